@@ -1,0 +1,377 @@
+"""Benchmark of the Mamba-2 recurrent-state decode step on B200.
+
+Workload (one "step" = one pass of the whole decode hot path over one batch):
+the Nemotron-H-8B mixer layer (H=128, P=64, N=128, G=8, K=4, conv_dim=10240),
+bf16 state (2 MiB per sequence) and activations, 64 active sequences
+scattered over a 256-slot cache, one fused launch per step (slot lookup, conv
+tap and roll, dt/dA, state update, C read-out, D skip, silu(z) gate).
+
+Metric: decode seq*layer-steps/s (whole job, all ranks), with the state GB/s
+and its fraction of HBM in the ``roofline`` object. Inputs are synthetic
+(seeded generators; no trained weights exist for this path) and resident in
+HBM when the timed region starts. L2 is flushed (a 512 MiB write) before every
+timed step, outside the kernel's own events.
+
+Usage: ``python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]``.
+With N > 1 the script runs under torchrun: each rank runs an independent
+replica of the workload on its own GPU (the path has no exchange step), and
+``value`` is the units of all ranks over the max-over-ranks device time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode seq*layer-steps/s"
+UNIT = "seq*layer-steps/s"
+WORKLOAD = "nemotron_h_layer decode: H=128 P=64 N=128 G=8 K=4, bf16 state+act, batch 64 / 256 slots"
+FLUSH_BYTES = 512 * 1024 * 1024
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "state_update_nemotron_h_layer.md")
+KERNEL_SOURCES = ["mamba_recurrent_state_b200/csrc/m2_state_update.cu",
+                  "mamba_recurrent_state_b200/csrc/m2_device.cuh"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="budget of the oracle CPU-baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks() -> tuple[float, str]:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+def profiled_traffic() -> float | None:
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source (null otherwise)."""
+    try:
+        text = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None
+    m_src = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
+    m_b = re.search(r"traffic_bytes_per_launch:\s*([0-9.e+]+)", text)
+    if not m_src or not m_b or m_src.group(1) != kernel_source_hash():
+        return None
+    return float(m_b.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    QUERY = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines: list[str] = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def oracle_sample(rows: int = 16):
+    """A bounded sample of the workload step for the oracle: ``rows`` of the 64
+    sequences, inputs generated up front. Returns (step function, rows, threads)."""
+    import numpy as np
+    import m2synth as S
+    import oracle as O
+    from m2synth import workloads as W
+    w = W.WORKLOADS[1]
+    orc = O.default()
+    p = W.layer_params(w)
+    f64 = S.storage_to_f64
+    idx = list(range(rows))
+    slots = W.slot_indices(w)
+    ssm_rows = [np.ascontiguousarray(f64(W.ssm_slot(w, int(slots[r])), w.state_dtype)) for r in idx]
+    conv_rows = [np.ascontiguousarray(f64(W.conv_slot(w, int(slots[r])), w.act_dtype)) for r in idx]
+    inp = {k: f64(v, w.act_dtype) for k, v in W.step_inputs(w, 0, rows=idx).items()}
+    params = (f64(p.conv_w, w.act_dtype), f64(p.conv_b, w.act_dtype), p.dt_bias.astype(np.float64),
+              p.A_log.astype(np.float64), p.D.astype(np.float64))
+    threads = os.cpu_count() or 1
+
+    def step():
+        O.decode_rows(orc, w.H, w.P, w.N, w.G, O.ROUND_BF16, ssm_rows, conv_rows, inp["xBC"],
+                      inp["dt"], inp["z"], *params, threads=threads)
+
+    return step, rows, threads
+
+
+def cpu_baseline(seconds: float) -> dict:
+    """The oracle, as it stands, on the host cores: one decode step over a
+    sample of the workload's sequences, repeated until the time budget is used."""
+    step, rows, threads = oracle_sample()
+    done = 0
+    t0 = time.perf_counter()
+    while True:
+        step()
+        done += rows
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return {"value": done / el, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{rows} of the 64 sequences of the workload step, decoded "
+                      f"{done // rows} times ({done} seq*layer-steps in {el:.1f} s)"}
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the oracle as it stands on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    step, rows, threads = oracle_sample()
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    value = rows * args.steps / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded generators)",
+        "config": {"workload": WORKLOAD, "sample_rows": rows},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{rows} of the 64 sequences per step, {args.steps} steps"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    import mamba_recurrent_state_b200 as m2
+    from m2synth import torch_inputs as TI
+    from m2synth import workloads as W
+
+    w = W.WORKLOADS[1]
+    shape = m2.Shape(w.H, w.P, w.N, w.G, w.K, w.state_dtype, w.act_dtype)
+    cache = m2.Cache(shape, w.num_slots)
+    TI.fill_caches(w, cache.ssm, cache.conv)
+    t = TI.layer_tensors(w)
+    ssm = m2.SSMParams(t["A_log"], t["dt_bias"], t["D"])
+    conv = m2.ConvParams(t["conv_w"], t["conv_b"], 1)
+    slots = t["slots"]
+    n_sets = 4  # distinct input sets, rotated
+    inputs = [TI.step_tensors(w, s) for s in range(n_sets)]
+    y = torch.empty((w.batch, w.H * w.P), dtype=torch.bfloat16, device="cuda")
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        inp = inputs[i % n_sets]
+        m2.state_update(cache, ssm, inp["xBC"], inp["dt"], slots, z=inp["z"], conv=conv, y=y)
+
+    for i in range(args.warmup):
+        flush.zero_()
+        step(i)
+    torch.cuda.synchronize()
+
+    # ---- device-resident timed region
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    sampler.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        step(i)
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    kern_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = max_over_ranks(sum(kern_ms), world)
+    if cache.device_error() != 0:
+        raise RuntimeError("device error word set during the benchmark")
+
+    # ---- end to end through the public API: pinned host inputs -> device ->
+    # step -> y back to pinned host memory, every step inside the events
+    host_in = [{k: v.cpu().pin_memory() for k, v in inp.items()} for inp in inputs]
+    dev_in = {k: torch.empty_like(v) for k, v in inputs[0].items()}
+    host_y = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host_in[0].values())
+    d2h = host_y.numel() * host_y.element_size()
+
+    def e2e_step(i):
+        for k, v in host_in[i % n_sets].items():
+            dev_in[k].copy_(v, non_blocking=True)
+        m2.state_update(cache, ssm, dev_in["xBC"], dev_in["dt"], slots, z=dev_in["z"], conv=conv,
+                        y=y)
+        host_y.copy_(y, non_blocking=True)
+
+    for i in range(args.warmup):
+        flush.zero_()
+        e2e_step(i)
+    torch.cuda.synchronize()
+    e_starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        e_starts[i].record(stream)
+        e2e_step(i)
+        e_ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_starts, e_ends)), world)
+
+    units = w.batch * args.steps * world
+    value = units / (total_ms / 1e3)
+    bytes_per_launch = W.bytes_per_unit(w) * w.batch + W.param_bytes_per_launch(w)
+    avg_s = (sum(kern_ms) / len(kern_ms)) / 1e3
+    achieved = bytes_per_launch / avg_s / 1e9
+    peak, peak_kind = measured_peaks()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded generators, random-init mixer parameters)",
+        "config": {"workload": WORKLOAD, "batch_per_gpu": w.batch, "num_slots": w.num_slots,
+                   "state_bytes_per_seq": w.state_bytes_per_slot(),
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "flushed (512 MiB write) before every timed step"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": profiled_traffic(),
+                     "peak_source": f"{peak_kind} hbm_gbs", "kernel": "m2 state_update (fused)",
+                     "algorithmic_bytes_per_launch": bytes_per_launch,
+                     "kernel_us_median": 1e3 * statistics.median(kern_ms)},
+        "e2e": {"value": units / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return
+    world, rank, local = dist_setup()
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,223 @@
+/*
+ * m2.h -- C ABI of libm2, the B200 (sm_100a) Mamba-2 recurrent-state library.
+ *
+ * The library runs the recurrent hot path of a Mamba-2 SSM mixer in hybrid
+ * Mamba-Transformer serving: the one-token decode step (causal conv update
+ * over a rolling conv cache, then the selective state update) and a chunked
+ * prefill scan that lands on the same state. It reads and writes a fixed-size
+ * per-sequence state cache in place at slot indices, with no gather/scatter.
+ *
+ * Passages that define the operations (cited by page title and section):
+ *  - vllm.cpp issue #1311 "NemotronH runs the PREFILL mamba kernels at decode",
+ *    section "The divergence": decode calls causal_conv1d_update and
+ *    selective_state_update, both taking state/conv slot indices and reading
+ *    and writing the cache in place at the slot.
+ *  - same issue, section "Confirm or refute": heads map to groups with
+ *    hpg = H/G, so n_groups = 8 is handled; a state update costs 1 launch and
+ *    0 allocations per layer per token (section "Cost, at T=1, ...").
+ *  - Nemotron-H-8B-Base-8K model record: ssm_state_size N, mamba_head_dim P,
+ *    mamba_num_heads H, n_groups G; 2 MiB of bf16 state per layer per
+ *    sequence, constant in context length; a fixed-size recurrent state
+ *    allocator.
+ *  - TensorRT-LLM issue #16976 (hybrid serving at concurrency 384): decode
+ *    must replay as a CUDA graph, so decode calls never allocate, never
+ *    synchronise and never read device status on the host.
+ *
+ * The recurrence, per head h with group g(h) = h / (H/G):
+ *     dt = softplus(dt_raw[h] + dt_bias[h]);  A = -exp(A_log[h]);  dA = exp(dt*A)
+ *     S[h,p,n] <- S[h,p,n]*dA + (dt*x[h,p]) * B[g,n]
+ *     y[h,p]    = sum_n S[h,p,n]*C[g,n] + D[h]*x[h,p],  times silu(z[h,p]) if z
+ * where x | B | C are the three parts of the post-conv xBC row
+ * (H*P, G*N and G*N channels; conv_dim = H*P + 2*G*N).
+ *
+ * Conventions for every call:
+ *  - Pointers are DEVICE pointers unless stated otherwise, on the device that
+ *    is current when the call is made. The caller owns every buffer except the
+ *    ones m2_cache_alloc creates.
+ *  - Tensor rows are contiguous (unit stride inside a row). Row strides are in
+ *    elements; every row start must be 16-byte aligned (pointer and stride).
+ *  - Slot indices are int32. A negative index marks a padding row: it is
+ *    skipped, its caches are not touched and its y row is written with zeros.
+ *    An index >= num_slots is a device error: the row is skipped, nothing is
+ *    written for it, and M2_ERR_BAD_SLOT is recorded in the cache's error
+ *    word. Slots must be unique within one call (checked on the host only when
+ *    the environment variable M2_VALIDATE=1 is set, which synchronises).
+ *  - All compute calls are asynchronous on `stream`, allocate nothing and never
+ *    synchronise (outside M2_VALIDATE mode), so they can be captured in CUDA
+ *    graphs. Argument errors are returned before anything is launched.
+ *  - There is no CPU fallback: without a usable sm_100 device the compute
+ *    calls fail with M2_ERR_CUDA.
+ */
+#ifndef M2_H_
+#define M2_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (CUstream); NULL is the legacy default stream. */
+typedef struct CUstream_st* m2_stream;
+
+typedef enum m2_dtype {
+    M2_F32 = 0,  /* IEEE binary32 */
+    M2_BF16 = 1  /* bfloat16 */
+} m2_dtype;
+
+typedef enum m2_status {
+    M2_OK = 0,
+    M2_ERR_INVALID_ARG = -1, /* NULL pointer, bad size, stride or alignment */
+    M2_ERR_UNSUPPORTED = -2, /* valid, but not a shape or dtype the kernels implement */
+    M2_ERR_CUDA = -3,        /* a CUDA runtime call or a launch failed */
+    M2_ERR_OOM = -4,         /* device allocation failed (m2_cache_alloc only) */
+    M2_ERR_BAD_SLOT = -5,    /* device: a slot index >= num_slots was seen */
+    M2_ERR_TIMEOUT = -6      /* device: a bounded wait inside a kernel ran out */
+} m2_status;
+
+/* Mixer shape (Nemotron-H-8B: H=128, P=64, N=128, G=8, K=4). */
+typedef struct m2_shape {
+    int32_t nheads;      /* H */
+    int32_t head_dim;    /* P */
+    int32_t d_state;     /* N */
+    int32_t ngroups;     /* G, divides H */
+    int32_t d_conv;      /* K, conv width (2..8) */
+    int32_t state_dtype; /* m2_dtype of the SSM cache */
+    int32_t act_dtype;   /* m2_dtype of activations, conv cache, conv weight/bias, dt_raw, y */
+} m2_shape;
+
+/* A slot-indexed cache of one mixer layer. */
+typedef struct m2_cache {
+    void* ssm;         /* [num_slots, H, P, N] state_dtype, N fastest */
+    void* conv;        /* [num_slots, K-1, conv_dim] act_dtype: the last K-1 RAW xBC
+                          inputs of each channel, oldest row first */
+    int32_t* error;    /* device int32 error word (0 = none), or NULL = not reported */
+    int64_t num_slots;
+    m2_shape shape;
+    int32_t owned;     /* 1 when m2_cache_alloc created ssm/conv/error */
+    int32_t device;    /* CUDA device ordinal of the buffers */
+} m2_cache;
+
+/* Depthwise causal conv parameters: weight [conv_dim, K] act_dtype (tap K-1
+ * multiplies the newest input), bias [conv_dim] act_dtype or NULL,
+ * activation 0 = none, 1 = SiLU. */
+typedef struct m2_conv_params {
+    const void* weight;
+    const void* bias;
+    int32_t activation;
+} m2_conv_params;
+
+/* Per-head SSM parameters, fp32 [H] each: A = -exp(A_log). */
+typedef struct m2_ssm_params {
+    const float* A_log;
+    const float* dt_bias;
+    const float* D;
+} m2_ssm_params;
+
+/* conv_dim = H*P + 2*G*N, or -1 for a NULL/invalid shape. Host only. */
+int64_t m2_conv_dim(const m2_shape* shape);
+
+/* M2_OK when the kernels implement `shape`; M2_ERR_INVALID_ARG for an
+ * inconsistent shape; M2_ERR_UNSUPPORTED otherwise. Host only, no CUDA. */
+m2_status m2_shape_check(const m2_shape* shape);
+
+/* Bytes of the SSM and conv caches for num_slots slots (Nemotron-H record:
+ * 2 MiB of bf16 state per slot at H=128, P=64, N=128). Host only, no CUDA. */
+m2_status m2_cache_bytes(const m2_shape* shape, int64_t num_slots, int64_t* ssm_bytes,
+                         int64_t* conv_bytes);
+
+/* The fixed-size recurrent state allocator (Nemotron-H record): allocates
+ * the SSM cache, the conv cache and the error word on the current device and
+ * zero-fills them on `stream` (then synchronises `stream`; not a hot call).
+ * Returns M2_ERR_OOM when the device is out of memory. */
+m2_status m2_cache_alloc(const m2_shape* shape, int64_t num_slots, m2_stream stream,
+                         m2_cache* out);
+
+/* Describes caller-owned buffers as a cache (for example torch tensors).
+ * ssm and conv must be 16-byte aligned; error_word may be NULL. Nothing is
+ * allocated or launched. */
+m2_status m2_cache_wrap(const m2_shape* shape, int64_t num_slots, void* ssm, void* conv,
+                        int32_t* error_word, m2_cache* out);
+
+/* Frees the buffers of a cache made by m2_cache_alloc (after synchronising
+ * `stream`); a wrapped cache is only cleared. */
+m2_status m2_cache_free(m2_cache* cache, m2_stream stream);
+
+/* Zero the SSM state and conv cache of n slots (start of new sequences) in one
+ * launch, without a host synchronisation. Negative indices are skipped; an
+ * index >= num_slots is a device error as above. */
+m2_status m2_cache_zero_slots(const m2_cache* cache, int32_t n, const int32_t* slot_idx,
+                              m2_stream stream);
+
+/*
+ * causal_conv1d_update over `seqlen` tokens per row (vllm.cpp issue, "The
+ * divergence"; seqlen > 1 is the prefill conv that precedes the chunk scan).
+ *   xBC      [batch, seqlen, conv_dim] act_dtype, raw; element (b,t,c) at
+ *            xBC[(b*seqlen + t)*xBC_row_stride + c]
+ *   xBC_out  [batch, seqlen, conv_dim] out_dtype (M2_F32 or M2_BF16), post-conv
+ *            (bias added, activation applied); same indexing with out_row_stride
+ *   slot_idx [batch] int32: row b reads its window history from, and writes
+ *            the last K-1 raw inputs back to, cache->conv[slot_idx[b]]
+ * The conv cache is rolled in place by exact copies. One launch.
+ */
+m2_status m2_conv1d_update(const m2_cache* cache, const m2_conv_params* conv, int32_t batch,
+                           int32_t seqlen, const void* xBC, int64_t xBC_row_stride,
+                           void* xBC_out, int32_t out_dtype, int64_t out_row_stride,
+                           const int32_t* slot_idx, m2_stream stream);
+
+/*
+ * selective_state_update for one token per row (vllm.cpp issue, "The
+ * divergence"), in place on cache->ssm at slot_idx[b].
+ *   conv     non-NULL: xBC is the RAW row and the conv tap + roll of
+ *            causal_conv1d_update run fused in the same launch (xBC_dtype must
+ *            then be act_dtype); NULL: xBC is already post-conv, in xBC_dtype
+ *   xBC      [batch, conv_dim], row stride xBC_row_stride
+ *   dt       [batch, H] act_dtype (dt_raw, before dt_bias and softplus)
+ *   z        [batch, H*P] act_dtype, or NULL for no gate
+ *   y        [batch, H*P] act_dtype, out
+ *   slot_idx [batch] int32
+ * The state is computed in fp32 and stored once, rounded to nearest even; y is
+ * computed from the unrounded new state. One launch, no scratch memory.
+ */
+m2_status m2_state_update(const m2_cache* cache, const m2_ssm_params* ssm,
+                          const m2_conv_params* conv, int32_t batch, const void* xBC,
+                          int32_t xBC_dtype, int64_t xBC_row_stride, const void* dt,
+                          int64_t dt_row_stride, const void* z, int64_t z_row_stride, void* y,
+                          int64_t y_row_stride, const int32_t* slot_idx, m2_stream stream);
+
+/*
+ * Chunked prefill scan (vllm.cpp issue, "The divergence": the chunk scan that
+ * follows CausalConv1dFwd at prefill). For each row, runs `seqlen` tokens of
+ * the recurrence starting from cache->ssm[slot_idx[b]] (or from zero when
+ * has_initial_state is NULL or has_initial_state[b] == 0), writes y for every
+ * token and stores the final state back to the same slot, rounded once.
+ *   xBC      [batch, seqlen, conv_dim] xBC_dtype, POST-conv, row stride
+ *            xBC_row_stride (token rows of a sequence are consecutive)
+ *   dt       [batch, seqlen, H] act_dtype, row stride dt_row_stride
+ *   z        [batch, seqlen, H*P] act_dtype or NULL, row stride z_row_stride
+ *   y        [batch, seqlen, H*P] act_dtype, row stride y_row_stride
+ *   chunk_size  tokens per chunk (the last chunk may be partial)
+ * No allocation, no scratch memory.
+ */
+m2_status m2_chunk_scan(const m2_cache* cache, const m2_ssm_params* ssm, int32_t batch,
+                        int32_t seqlen, int32_t chunk_size, const void* xBC, int32_t xBC_dtype,
+                        int64_t xBC_row_stride, const void* dt, int64_t dt_row_stride,
+                        const void* z, int64_t z_row_stride, void* y, int64_t y_row_stride,
+                        const int32_t* slot_idx, const uint8_t* has_initial_state,
+                        m2_stream stream);
+
+/* Debug/test path: synchronises `stream`, copies the cache's error word to
+ * *out_code (0 or an m2_status value) and clears it. Not for hot loops. */
+m2_status m2_get_device_error(const m2_cache* cache, m2_stream stream, int32_t* out_code);
+
+/* Static description of a status code. */
+const char* m2_status_string(m2_status status);
+
+/* Library version string, "m2 <major>.<minor>". */
+const char* m2_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* M2_H_ */

@@ -1,0 +1,342 @@
+"""B200-native Mamba-2 recurrent-state kernels: thin Python binding of libm2.
+
+Every step of the computation runs in ``libm2.so`` (hand-written sm_100a CUDA
+behind the C ABI of ``include/m2.h``); this module only marshals torch tensors
+into pointers, sizes and the current CUDA stream, and raises on a non-OK
+status. There is no CPU fallback: without the built library, importing the
+functions that compute raises immediately.
+
+Operations (vllm.cpp issue #1311 "NemotronH runs the PREFILL mamba kernels at
+decode", section "The divergence"; shapes from the Nemotron-H-8B-Base-8K
+record):
+
+* ``state_update``  -- one-token selective_state_update, optionally with the
+  causal_conv1d_update tap fused into the same launch, in place at slots.
+* ``conv1d_update`` -- causal_conv1d_update over seqlen >= 1 tokens.
+* ``chunk_scan``    -- prefill scan landing on the same state as sequential
+  updates.
+* ``Cache``         -- the fixed-size, slot-indexed state cache.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libm2.so")
+
+M2_F32 = 0
+M2_BF16 = 1
+
+STATUS = {
+    0: "ok",
+    -1: "invalid argument",
+    -2: "unsupported shape or dtype",
+    -3: "CUDA error",
+    -4: "out of device memory",
+    -5: "slot index out of range",
+    -6: "bounded wait timed out",
+}
+M2_OK = 0
+M2_ERR_INVALID_ARG = -1
+M2_ERR_UNSUPPORTED = -2
+M2_ERR_CUDA = -3
+M2_ERR_OOM = -4
+M2_ERR_BAD_SLOT = -5
+M2_ERR_TIMEOUT = -6
+
+
+class M2Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({status})")
+        self.status = status
+
+
+class m2_shape(ctypes.Structure):
+    _fields_ = [("nheads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("d_state", ctypes.c_int32), ("ngroups", ctypes.c_int32),
+                ("d_conv", ctypes.c_int32), ("state_dtype", ctypes.c_int32),
+                ("act_dtype", ctypes.c_int32)]
+
+
+class m2_cache(ctypes.Structure):
+    _fields_ = [("ssm", ctypes.c_void_p), ("conv", ctypes.c_void_p),
+                ("error", ctypes.c_void_p), ("num_slots", ctypes.c_int64),
+                ("shape", m2_shape), ("owned", ctypes.c_int32), ("device", ctypes.c_int32)]
+
+
+class m2_conv_params(ctypes.Structure):
+    _fields_ = [("weight", ctypes.c_void_p), ("bias", ctypes.c_void_p),
+                ("activation", ctypes.c_int32)]
+
+
+class m2_ssm_params(ctypes.Structure):
+    _fields_ = [("A_log", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p), ("D", ctypes.c_void_p)]
+
+
+# exported symbols and their signatures (mirrors include/m2.h)
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_I64 = ctypes.c_int64
+SIGNATURES = {
+    "m2_conv_dim": (_I64, [ctypes.POINTER(m2_shape)]),
+    "m2_shape_check": (_I32, [ctypes.POINTER(m2_shape)]),
+    "m2_cache_bytes": (_I32, [ctypes.POINTER(m2_shape), _I64, ctypes.POINTER(_I64),
+                              ctypes.POINTER(_I64)]),
+    "m2_cache_alloc": (_I32, [ctypes.POINTER(m2_shape), _I64, _P, ctypes.POINTER(m2_cache)]),
+    "m2_cache_wrap": (_I32, [ctypes.POINTER(m2_shape), _I64, _P, _P, _P,
+                             ctypes.POINTER(m2_cache)]),
+    "m2_cache_free": (_I32, [ctypes.POINTER(m2_cache), _P]),
+    "m2_cache_zero_slots": (_I32, [ctypes.POINTER(m2_cache), _I32, _P, _P]),
+    "m2_conv1d_update": (_I32, [ctypes.POINTER(m2_cache), ctypes.POINTER(m2_conv_params), _I32,
+                                _I32, _P, _I64, _P, _I32, _I64, _P, _P]),
+    "m2_state_update": (_I32, [ctypes.POINTER(m2_cache), ctypes.POINTER(m2_ssm_params),
+                               ctypes.POINTER(m2_conv_params), _I32, _P, _I32, _I64, _P, _I64,
+                               _P, _I64, _P, _I64, _P, _P]),
+    "m2_chunk_scan": (_I32, [ctypes.POINTER(m2_cache), ctypes.POINTER(m2_ssm_params), _I32, _I32,
+                             _I32, _P, _I32, _I64, _P, _I64, _P, _I64, _P, _I64, _P, _P, _P]),
+    "m2_get_device_error": (_I32, [ctypes.POINTER(m2_cache), _P, ctypes.POINTER(_I32)]),
+    "m2_status_string": (ctypes.c_char_p, [_I32]),
+    "m2_version": (ctypes.c_char_p, []),
+}
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libm2 (raises if it has not been built: no fallback exists)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing; build it with "
+                              "`python -m mamba_recurrent_state_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(status: int, what: str) -> None:
+    if status != M2_OK:
+        raise M2Error(status, what)
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return M2_F32
+    if t == torch.bfloat16:
+        return M2_BF16
+    raise TypeError(f"unsupported dtype {t} (float32 or bfloat16)")
+
+
+def torch_dtype(code: int) -> torch.dtype:
+    return torch.float32 if code == M2_F32 else torch.bfloat16
+
+
+def _stream_ptr() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _row_stride(t: torch.Tensor) -> int:
+    if t.stride(-1) != 1:
+        raise ValueError("rows must be contiguous (unit stride in the last dimension)")
+    return t.stride(-2) if t.dim() >= 2 else t.shape[-1]
+
+
+@dataclasses.dataclass(frozen=True)
+class Shape:
+    H: int
+    P: int
+    N: int
+    G: int
+    K: int = 4
+    state_dtype: int = M2_BF16
+    act_dtype: int = M2_BF16
+
+    @property
+    def conv_dim(self) -> int:
+        return self.H * self.P + 2 * self.G * self.N
+
+    def c(self) -> m2_shape:
+        return m2_shape(self.H, self.P, self.N, self.G, self.K, self.state_dtype, self.act_dtype)
+
+
+def shape_check(shape: Shape) -> int:
+    s = shape.c()
+    return lib().m2_shape_check(ctypes.byref(s))
+
+
+def cache_bytes(shape: Shape, num_slots: int) -> tuple[int, int]:
+    s = shape.c()
+    a, b = _I64(), _I64()
+    _check(lib().m2_cache_bytes(ctypes.byref(s), num_slots, ctypes.byref(a), ctypes.byref(b)),
+           "m2_cache_bytes")
+    return a.value, b.value
+
+
+class Cache:
+    """A slot-indexed state cache of one mixer layer.
+
+    ``ssm``  [num_slots, H, P, N] state dtype; ``conv`` [num_slots, K-1,
+    conv_dim] activation dtype (last K-1 raw inputs, oldest row first);
+    ``error`` a one-element int32 device word. The memory is owned by torch
+    (this object wraps it with ``m2_cache_wrap``) unless created with
+    ``native=True``, in which case ``m2_cache_alloc`` owns it.
+    """
+
+    def __init__(self, shape: Shape, num_slots: int, device="cuda", native: bool = False,
+                 ssm: Optional[torch.Tensor] = None, conv: Optional[torch.Tensor] = None):
+        self.shape = shape
+        self.num_slots = num_slots
+        self._c = m2_cache()
+        s = shape.c()
+        self.native = native
+        if native:
+            _check(lib().m2_cache_alloc(ctypes.byref(s), num_slots, _stream_ptr(),
+                                        ctypes.byref(self._c)), "m2_cache_alloc")
+            self.ssm = self.conv = self.error = None
+            return
+        dev = torch.device(device)
+        if ssm is None:
+            ssm = torch.zeros((num_slots, shape.H, shape.P, shape.N),
+                              dtype=torch_dtype(shape.state_dtype), device=dev)
+        if conv is None:
+            conv = torch.zeros((num_slots, shape.K - 1, shape.conv_dim),
+                               dtype=torch_dtype(shape.act_dtype), device=dev)
+        assert ssm.is_contiguous() and conv.is_contiguous()
+        self.ssm, self.conv = ssm, conv
+        self.error = torch.zeros(1, dtype=torch.int32, device=ssm.device)
+        _check(lib().m2_cache_wrap(ctypes.byref(s), num_slots, ssm.data_ptr(), conv.data_ptr(),
+                                   self.error.data_ptr(), ctypes.byref(self._c)), "m2_cache_wrap")
+
+    @property
+    def c(self) -> m2_cache:
+        return self._c
+
+    def zero_slots(self, slot_idx: torch.Tensor) -> None:
+        _check(lib().m2_cache_zero_slots(ctypes.byref(self._c), slot_idx.numel(),
+                                         slot_idx.data_ptr(), _stream_ptr()),
+               "m2_cache_zero_slots")
+
+    def device_error(self) -> int:
+        """Reads and clears the device error word (synchronises the stream)."""
+        code = _I32()
+        _check(lib().m2_get_device_error(ctypes.byref(self._c), _stream_ptr(), ctypes.byref(code)),
+               "m2_get_device_error")
+        return code.value
+
+    def free(self) -> None:
+        if self.native and self._c.ssm:
+            _check(lib().m2_cache_free(ctypes.byref(self._c), _stream_ptr()), "m2_cache_free")
+
+    def __del__(self):  # native caches only
+        try:
+            if self.native and self._c.ssm:
+                lib().m2_cache_free(ctypes.byref(self._c), None)
+        except Exception:
+            pass
+
+
+@dataclasses.dataclass
+class SSMParams:
+    """Per-head fp32 parameters [H]: A = -exp(A_log), dt_bias, D."""
+    A_log: torch.Tensor
+    dt_bias: torch.Tensor
+    D: torch.Tensor
+
+    def c(self) -> m2_ssm_params:
+        for t in (self.A_log, self.dt_bias, self.D):
+            if t.dtype != torch.float32 or not t.is_contiguous():
+                raise TypeError("SSM parameters must be contiguous float32")
+        return m2_ssm_params(self.A_log.data_ptr(), self.dt_bias.data_ptr(), self.D.data_ptr())
+
+
+@dataclasses.dataclass
+class ConvParams:
+    """Depthwise conv: weight [conv_dim, K], bias [conv_dim] or None, SiLU on/off."""
+    weight: torch.Tensor
+    bias: Optional[torch.Tensor] = None
+    activation: int = 1
+
+    def c(self) -> m2_conv_params:
+        if not self.weight.is_contiguous():
+            raise ValueError("conv weight must be contiguous [conv_dim, K]")
+        return m2_conv_params(self.weight.data_ptr(), _ptr(self.bias), self.activation)
+
+
+def state_update(cache: Cache, ssm: SSMParams, xBC: torch.Tensor, dt: torch.Tensor,
+                 slot_idx: torch.Tensor, z: Optional[torch.Tensor] = None,
+                 conv: Optional[ConvParams] = None, y: Optional[torch.Tensor] = None,
+                 stream: Optional[int] = None) -> torch.Tensor:
+    """One decode step for ``xBC.shape[0]`` rows, in place on ``cache``.
+
+    With ``conv`` given, ``xBC`` is the raw row and the conv tap is fused;
+    otherwise ``xBC`` is post-conv (float32 or bfloat16). Returns y
+    [batch, H*P] in the activation dtype.
+    """
+    sh = cache.shape
+    batch = xBC.shape[0]
+    if y is None:
+        y = torch.empty((batch, sh.H * sh.P), dtype=torch_dtype(sh.act_dtype), device=xBC.device)
+    sp = ssm.c()
+    cp = conv.c() if conv is not None else None
+    st = lib().m2_state_update(
+        ctypes.byref(cache.c), ctypes.byref(sp), ctypes.byref(cp) if cp is not None else None,
+        batch, xBC.data_ptr(), _dtype_code(xBC.dtype), _row_stride(xBC), dt.data_ptr(),
+        _row_stride(dt), _ptr(z), _row_stride(z) if z is not None else 0, y.data_ptr(),
+        _row_stride(y), slot_idx.data_ptr(), _stream_ptr() if stream is None else stream)
+    _check(st, "m2_state_update")
+    return y
+
+
+def conv1d_update(cache: Cache, conv: ConvParams, xBC: torch.Tensor, slot_idx: torch.Tensor,
+                  out: Optional[torch.Tensor] = None, out_dtype: Optional[torch.dtype] = None,
+                  stream: Optional[int] = None) -> torch.Tensor:
+    """causal_conv1d_update over xBC [batch, seqlen, conv_dim] (or [batch, conv_dim])."""
+    x3 = xBC if xBC.dim() == 3 else xBC.unsqueeze(1)
+    batch, seqlen, cd = x3.shape
+    if out is None:
+        out = torch.empty((batch, seqlen, cd), dtype=out_dtype or xBC.dtype, device=xBC.device)
+    o3 = out if out.dim() == 3 else out.unsqueeze(1)
+    cp = conv.c()
+    st = lib().m2_conv1d_update(ctypes.byref(cache.c), ctypes.byref(cp), batch, seqlen,
+                                x3.data_ptr(), x3.stride(1), o3.data_ptr(), _dtype_code(o3.dtype),
+                                o3.stride(1), slot_idx.data_ptr(),
+                                _stream_ptr() if stream is None else stream)
+    _check(st, "m2_conv1d_update")
+    return out
+
+
+def chunk_scan(cache: Cache, ssm: SSMParams, xBC: torch.Tensor, dt: torch.Tensor,
+               slot_idx: torch.Tensor, z: Optional[torch.Tensor] = None, chunk_size: int = 128,
+               has_initial_state: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
+               stream: Optional[int] = None) -> torch.Tensor:
+    """Prefill scan over xBC [batch, seqlen, conv_dim] (post-conv), dt [batch, seqlen, H]."""
+    sh = cache.shape
+    batch, seqlen, _ = xBC.shape
+    for t in (xBC, dt) + ((z,) if z is not None else ()):
+        if t.stride(0) != t.shape[1] * t.stride(1):
+            raise ValueError("token rows of a sequence must be consecutive")
+    if y is None:
+        y = torch.empty((batch, seqlen, sh.H * sh.P), dtype=torch_dtype(sh.act_dtype),
+                        device=xBC.device)
+    sp = ssm.c()
+    st = lib().m2_chunk_scan(
+        ctypes.byref(cache.c), ctypes.byref(sp), batch, seqlen, chunk_size, xBC.data_ptr(),
+        _dtype_code(xBC.dtype), xBC.stride(1), dt.data_ptr(), dt.stride(1), _ptr(z),
+        z.stride(1) if z is not None else 0, y.data_ptr(), y.stride(1), slot_idx.data_ptr(),
+        _ptr(has_initial_state), _stream_ptr() if stream is None else stream)
+    _check(st, "m2_chunk_scan")
+    return y

@@ -1,0 +1,376 @@
+// m2_api.cu -- the extern "C" entry points of libm2 (include/m2.h).
+//
+// Host-side only: argument validation, launch planning and error mapping. No
+// entry point on the hot path allocates, synchronises or reads device memory
+// on the host (the allocator and the error query are not hot-path calls).
+#include <cuda_runtime.h>
+
+#include <cstdlib>
+#include <cstring>
+#include <vector>
+
+#include "m2_internal.cuh"
+
+namespace {
+
+bool valid_dtype(int32_t d) { return d == M2_F32 || d == M2_BF16; }
+int dsize(int32_t d) { return d == M2_F32 ? 4 : 2; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool stride_ok(int64_t stride_elems, int elem_size, int64_t min_elems) {
+    return stride_elems >= min_elems && (stride_elems * elem_size) % 16 == 0;
+}
+
+m2_status shape_status(const m2_shape* s) {
+    if (!s) return M2_ERR_INVALID_ARG;
+    if (s->nheads <= 0 || s->head_dim <= 0 || s->d_state <= 0 || s->ngroups <= 0 || s->d_conv <= 0)
+        return M2_ERR_INVALID_ARG;
+    if (s->nheads % s->ngroups != 0) return M2_ERR_INVALID_ARG;
+    if (!valid_dtype(s->state_dtype) || !valid_dtype(s->act_dtype)) return M2_ERR_INVALID_ARG;
+    if (s->d_conv < 2 || s->d_conv > 8) return M2_ERR_UNSUPPORTED;
+    const int a = dsize(s->act_dtype);
+    const int64_t hp = static_cast<int64_t>(s->nheads) * s->head_dim;
+    const int64_t gn = static_cast<int64_t>(s->ngroups) * s->d_state;
+    // 16-byte vectors must tile the x, B and C segments of a row
+    if ((hp * a) % 16 != 0 || (gn * a) % 16 != 0 || (static_cast<int64_t>(s->head_dim) * a) % 16 != 0)
+        return M2_ERR_UNSUPPORTED;
+    m2::DecodePlan plan;
+    return m2::plan_state_update(s->nheads, s->head_dim, s->d_state, s->ngroups,
+                                 s->state_dtype == M2_BF16, 0, &plan);
+}
+
+m2_status cache_status(const m2_cache* c) {
+    if (!c || !c->ssm || !c->conv || c->num_slots <= 0) return M2_ERR_INVALID_ARG;
+    return shape_status(&c->shape);
+}
+
+m2_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return M2_OK;
+    if (e == cudaErrorMemoryAllocation) return M2_ERR_OOM;
+    return M2_ERR_CUDA;
+}
+
+// M2_VALIDATE=1: copy the slot indices to the host (synchronising) and reject
+// duplicates. Debug aid only; never used on a captured stream.
+bool validate_mode() {
+    const char* v = std::getenv("M2_VALIDATE");
+    return v && v[0] == '1';
+}
+
+m2_status validate_slots(const int32_t* slot_idx, int32_t n, int64_t num_slots, cudaStream_t s) {
+    std::vector<int32_t> h(static_cast<size_t>(n));
+    if (cudaMemcpyAsync(h.data(), slot_idx, sizeof(int32_t) * n, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return M2_ERR_CUDA;
+    std::vector<char> seen(static_cast<size_t>(num_slots), 0);
+    for (int32_t v : h) {
+        if (v < 0 || v >= num_slots) continue;  // padding / device-reported
+        if (seen[v]) return M2_ERR_INVALID_ARG;
+        seen[v] = 1;
+    }
+    return M2_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t m2_conv_dim(const m2_shape* s) {
+    if (!s || s->nheads <= 0 || s->head_dim <= 0 || s->d_state <= 0 || s->ngroups <= 0) return -1;
+    return static_cast<int64_t>(s->nheads) * s->head_dim + 2LL * s->ngroups * s->d_state;
+}
+
+m2_status m2_shape_check(const m2_shape* s) { return shape_status(s); }
+
+m2_status m2_cache_bytes(const m2_shape* s, int64_t num_slots, int64_t* ssm_bytes,
+                         int64_t* conv_bytes) {
+    const m2_status st = shape_status(s);
+    if (st == M2_ERR_INVALID_ARG) return st;
+    if (num_slots <= 0) return M2_ERR_INVALID_ARG;
+    const int64_t per_ssm = static_cast<int64_t>(s->nheads) * s->head_dim * s->d_state * dsize(s->state_dtype);
+    const int64_t per_conv = static_cast<int64_t>(s->d_conv - 1) * m2_conv_dim(s) * dsize(s->act_dtype);
+    if (ssm_bytes) *ssm_bytes = per_ssm * num_slots;
+    if (conv_bytes) *conv_bytes = per_conv * num_slots;
+    return M2_OK;
+}
+
+m2_status m2_cache_alloc(const m2_shape* s, int64_t num_slots, m2_stream stream, m2_cache* out) {
+    if (!out) return M2_ERR_INVALID_ARG;
+    const m2_status st = shape_status(s);
+    if (st != M2_OK) return st;
+    int64_t ssm_b = 0, conv_b = 0;
+    if (m2_cache_bytes(s, num_slots, &ssm_b, &conv_b) != M2_OK) return M2_ERR_INVALID_ARG;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return M2_ERR_CUDA;
+    void* ssm = nullptr;
+    void* conv = nullptr;
+    void* err = nullptr;
+    cudaError_t e = cudaMalloc(&ssm, static_cast<size_t>(ssm_b));
+    if (e == cudaSuccess) e = cudaMalloc(&conv, static_cast<size_t>(conv_b));
+    if (e == cudaSuccess) e = cudaMalloc(&err, sizeof(int32_t));
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    if (e == cudaSuccess) e = cudaMemsetAsync(ssm, 0, static_cast<size_t>(ssm_b), cs);
+    if (e == cudaSuccess) e = cudaMemsetAsync(conv, 0, static_cast<size_t>(conv_b), cs);
+    if (e == cudaSuccess) e = cudaMemsetAsync(err, 0, sizeof(int32_t), cs);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+    if (e != cudaSuccess) {
+        cudaFree(ssm);
+        cudaFree(conv);
+        cudaFree(err);
+        cudaGetLastError();
+        return from_cuda(e);
+    }
+    std::memset(out, 0, sizeof(*out));
+    out->ssm = ssm;
+    out->conv = conv;
+    out->error = static_cast<int32_t*>(err);
+    out->num_slots = num_slots;
+    out->shape = *s;
+    out->owned = 1;
+    out->device = dev;
+    return M2_OK;
+}
+
+m2_status m2_cache_wrap(const m2_shape* s, int64_t num_slots, void* ssm, void* conv,
+                        int32_t* error_word, m2_cache* out) {
+    if (!out || !ssm || !conv || num_slots <= 0) return M2_ERR_INVALID_ARG;
+    if (!aligned16(ssm) || !aligned16(conv)) return M2_ERR_INVALID_ARG;
+    if (error_word && (reinterpret_cast<uintptr_t>(error_word) & 3u)) return M2_ERR_INVALID_ARG;
+    const m2_status st = shape_status(s);
+    if (st != M2_OK) return st;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaGetLastError();
+    std::memset(out, 0, sizeof(*out));
+    out->ssm = ssm;
+    out->conv = conv;
+    out->error = error_word;
+    out->num_slots = num_slots;
+    out->shape = *s;
+    out->owned = 0;
+    out->device = dev;
+    return M2_OK;
+}
+
+m2_status m2_cache_free(m2_cache* c, m2_stream stream) {
+    if (!c) return M2_ERR_INVALID_ARG;
+    m2_status st = M2_OK;
+    if (c->owned) {
+        if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) st = M2_ERR_CUDA;
+        cudaFree(c->ssm);
+        cudaFree(c->conv);
+        cudaFree(c->error);
+    }
+    std::memset(c, 0, sizeof(*c));
+    return st;
+}
+
+m2_status m2_cache_zero_slots(const m2_cache* c, int32_t n, const int32_t* slot_idx, m2_stream stream) {
+    const m2_status st = cache_status(c);
+    if (st != M2_OK) return st;
+    if (n < 0 || (n > 0 && !slot_idx)) return M2_ERR_INVALID_ARG;
+    if (n == 0) return M2_OK;
+    m2::ZeroArgs a{};
+    a.ssm = c->ssm;
+    a.conv = c->conv;
+    a.error = c->error;
+    a.num_slots = c->num_slots;
+    m2_cache_bytes(&c->shape, 1, &a.ssm_bytes_per_slot, &a.conv_bytes_per_slot);
+    a.n = n;
+    a.slot_idx = slot_idx;
+    return from_cuda(m2::launch_zero_slots(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+m2_status m2_conv1d_update(const m2_cache* c, const m2_conv_params* conv, int32_t batch,
+                           int32_t seqlen, const void* xBC, int64_t xBC_row_stride, void* xBC_out,
+                           int32_t out_dtype, int64_t out_row_stride, const int32_t* slot_idx,
+                           m2_stream stream) {
+    const m2_status st = cache_status(c);
+    if (st != M2_OK) return st;
+    if (!conv || !conv->weight || batch < 0 || seqlen < 0 || !valid_dtype(out_dtype))
+        return M2_ERR_INVALID_ARG;
+    if (conv->activation != 0 && conv->activation != 1) return M2_ERR_INVALID_ARG;
+    if (batch == 0 || seqlen == 0) return M2_OK;
+    if (!xBC || !xBC_out || !slot_idx) return M2_ERR_INVALID_ARG;
+    const m2_shape& s = c->shape;
+    const int64_t cd = m2_conv_dim(&s);
+    const int as = dsize(s.act_dtype);
+    if (!aligned16(xBC) || !aligned16(xBC_out) || !stride_ok(xBC_row_stride, as, cd) ||
+        !stride_ok(out_row_stride, dsize(out_dtype), cd))
+        return M2_ERR_INVALID_ARG;
+    if (validate_mode()) {
+        const m2_status v = validate_slots(slot_idx, batch, c->num_slots, reinterpret_cast<cudaStream_t>(stream));
+        if (v != M2_OK) return v;
+    }
+    m2::ConvArgs a{};
+    a.conv = c->conv;
+    a.error = c->error;
+    a.num_slots = c->num_slots;
+    a.K = s.d_conv;
+    a.conv_dim = cd;
+    a.act_bf16 = s.act_dtype == M2_BF16;
+    a.out_bf16 = out_dtype == M2_BF16;
+    a.w = conv->weight;
+    a.b = conv->bias;
+    a.activation = conv->activation;
+    a.batch = batch;
+    a.seqlen = seqlen;
+    a.x = xBC;
+    a.x_stride = xBC_row_stride;
+    a.out = xBC_out;
+    a.out_stride = out_row_stride;
+    a.slot_idx = slot_idx;
+    return from_cuda(m2::launch_conv1d_update(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+m2_status m2_state_update(const m2_cache* c, const m2_ssm_params* ssm, const m2_conv_params* conv,
+                          int32_t batch, const void* xBC, int32_t xBC_dtype, int64_t xBC_row_stride,
+                          const void* dt, int64_t dt_row_stride, const void* z, int64_t z_row_stride,
+                          void* y, int64_t y_row_stride, const int32_t* slot_idx, m2_stream stream) {
+    const m2_status st = cache_status(c);
+    if (st != M2_OK) return st;
+    if (!ssm || !ssm->A_log || !ssm->dt_bias || !ssm->D || batch < 0 || !valid_dtype(xBC_dtype))
+        return M2_ERR_INVALID_ARG;
+    if (batch == 0) return M2_OK;
+    if (!xBC || !dt || !y || !slot_idx) return M2_ERR_INVALID_ARG;
+    const m2_shape& s = c->shape;
+    const int as = dsize(s.act_dtype);
+    const int64_t cd = m2_conv_dim(&s);
+    const int64_t hp = static_cast<int64_t>(s.nheads) * s.head_dim;
+    if (conv) {
+        if (!conv->weight || (conv->activation != 0 && conv->activation != 1)) return M2_ERR_INVALID_ARG;
+        if (xBC_dtype != s.act_dtype) return M2_ERR_INVALID_ARG;
+    }
+    if (!aligned16(xBC) || !aligned16(y) || !stride_ok(xBC_row_stride, dsize(xBC_dtype), cd) ||
+        !stride_ok(y_row_stride, as, hp) || dt_row_stride < s.nheads)
+        return M2_ERR_INVALID_ARG;
+    if (z && (!aligned16(z) || !stride_ok(z_row_stride, as, hp))) return M2_ERR_INVALID_ARG;
+    m2::DecodePlan plan;
+    const m2_status ps = m2::plan_state_update(s.nheads, s.head_dim, s.d_state, s.ngroups,
+                                               s.state_dtype == M2_BF16, conv != nullptr, &plan);
+    if (ps != M2_OK) return ps;
+    if (validate_mode()) {
+        const m2_status v = validate_slots(slot_idx, batch, c->num_slots, reinterpret_cast<cudaStream_t>(stream));
+        if (v != M2_OK) return v;
+    }
+    m2::StateUpdateArgs a{};
+    a.ssm = c->ssm;
+    a.conv = c->conv;
+    a.error = c->error;
+    a.num_slots = c->num_slots;
+    a.H = s.nheads;
+    a.P = s.head_dim;
+    a.N = s.d_state;
+    a.G = s.ngroups;
+    a.K = s.d_conv;
+    a.conv_dim = cd;
+    a.state_bf16 = s.state_dtype == M2_BF16;
+    a.act_bf16 = s.act_dtype == M2_BF16;
+    a.x_bf16 = xBC_dtype == M2_BF16;
+    a.A_log = ssm->A_log;
+    a.dt_bias = ssm->dt_bias;
+    a.D = ssm->D;
+    a.conv_w = conv ? conv->weight : nullptr;
+    a.conv_b = conv ? conv->bias : nullptr;
+    a.activation = conv ? conv->activation : 0;
+    a.fused = conv != nullptr;
+    a.batch = batch;
+    a.xBC = xBC;
+    a.xBC_stride = xBC_row_stride;
+    a.dt = dt;
+    a.dt_stride = dt_row_stride;
+    a.z = z;
+    a.z_stride = z_row_stride;
+    a.y = y;
+    a.y_stride = y_row_stride;
+    a.slot_idx = slot_idx;
+    return from_cuda(m2::launch_state_update(a, plan, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+m2_status m2_chunk_scan(const m2_cache* c, const m2_ssm_params* ssm, int32_t batch, int32_t seqlen,
+                        int32_t chunk_size, const void* xBC, int32_t xBC_dtype, int64_t xBC_row_stride,
+                        const void* dt, int64_t dt_row_stride, const void* z, int64_t z_row_stride,
+                        void* y, int64_t y_row_stride, const int32_t* slot_idx,
+                        const uint8_t* has_initial_state, m2_stream stream) {
+    const m2_status st = cache_status(c);
+    if (st != M2_OK) return st;
+    if (!ssm || !ssm->A_log || !ssm->dt_bias || !ssm->D || batch < 0 || seqlen < 0 ||
+        chunk_size <= 0 || !valid_dtype(xBC_dtype))
+        return M2_ERR_INVALID_ARG;
+    if (batch == 0 || seqlen == 0) return M2_OK;
+    if (!xBC || !dt || !y || !slot_idx) return M2_ERR_INVALID_ARG;
+    const m2_shape& s = c->shape;
+    const int as = dsize(s.act_dtype);
+    const int64_t cd = m2_conv_dim(&s);
+    const int64_t hp = static_cast<int64_t>(s.nheads) * s.head_dim;
+    if (!aligned16(xBC) || !aligned16(y) || !stride_ok(xBC_row_stride, dsize(xBC_dtype), cd) ||
+        !stride_ok(y_row_stride, as, hp) || dt_row_stride < s.nheads)
+        return M2_ERR_INVALID_ARG;
+    if (z && (!aligned16(z) || !stride_ok(z_row_stride, as, hp))) return M2_ERR_INVALID_ARG;
+    const m2_status ps = m2::plan_chunk_scan(s.nheads, s.head_dim, s.d_state, s.ngroups,
+                                             s.state_dtype == M2_BF16, s.act_dtype == M2_BF16,
+                                             xBC_dtype == M2_BF16, chunk_size);
+    if (ps != M2_OK) return ps;
+    if (validate_mode()) {
+        const m2_status v = validate_slots(slot_idx, batch, c->num_slots, reinterpret_cast<cudaStream_t>(stream));
+        if (v != M2_OK) return v;
+    }
+    m2::ScanArgs a{};
+    a.ssm = c->ssm;
+    a.error = c->error;
+    a.num_slots = c->num_slots;
+    a.H = s.nheads;
+    a.P = s.head_dim;
+    a.N = s.d_state;
+    a.G = s.ngroups;
+    a.state_bf16 = s.state_dtype == M2_BF16;
+    a.act_bf16 = s.act_dtype == M2_BF16;
+    a.x_bf16 = xBC_dtype == M2_BF16;
+    a.A_log = ssm->A_log;
+    a.dt_bias = ssm->dt_bias;
+    a.D = ssm->D;
+    a.batch = batch;
+    a.seqlen = seqlen;
+    a.chunk = chunk_size;
+    a.xBC = xBC;
+    a.xBC_stride = xBC_row_stride;
+    a.dt = dt;
+    a.dt_stride = dt_row_stride;
+    a.z = z;
+    a.z_stride = z_row_stride;
+    a.y = y;
+    a.y_stride = y_row_stride;
+    a.slot_idx = slot_idx;
+    a.has_init = has_initial_state;
+    return from_cuda(m2::launch_chunk_scan(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+m2_status m2_get_device_error(const m2_cache* c, m2_stream stream, int32_t* out_code) {
+    if (!c || !out_code) return M2_ERR_INVALID_ARG;
+    *out_code = 0;
+    if (!c->error) return M2_OK;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    int32_t h = 0;
+    cudaError_t e = cudaMemcpyAsync(&h, c->error, sizeof(h), cudaMemcpyDeviceToHost, cs);
+    if (e == cudaSuccess) e = cudaMemsetAsync(c->error, 0, sizeof(int32_t), cs);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
+    if (e != cudaSuccess) return M2_ERR_CUDA;
+    *out_code = h;
+    return M2_OK;
+}
+
+const char* m2_status_string(m2_status s) {
+    switch (s) {
+        case M2_OK: return "ok";
+        case M2_ERR_INVALID_ARG: return "invalid argument";
+        case M2_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case M2_ERR_CUDA: return "CUDA error";
+        case M2_ERR_OOM: return "out of device memory";
+        case M2_ERR_BAD_SLOT: return "slot index out of range";
+        case M2_ERR_TIMEOUT: return "bounded wait timed out";
+    }
+    return "unknown status";
+}
+
+const char* m2_version(void) { return "m2 0.1"; }
+
+}  // extern "C"

@@ -1,0 +1,192 @@
+// m2_conv1d.cu -- causal_conv1d_update over seqlen >= 1 tokens per row, and the
+// slot-zeroing kernel of the cache lifecycle.
+//
+// Operation: vllm.cpp issue #1311 "NemotronH runs the PREFILL mamba kernels at
+// decode", section "The divergence": causal_conv1d_update reads and writes the
+// conv cache in place at conv_state_indices; with seqlen > 1 it is the prefill
+// conv (CausalConv1dFwd) that feeds the chunk scan. For channel c and token t:
+//   window = (raw inputs t-K+1 .. t), older ones from the cache,
+//   out[t, c] = bias[c] + sum_k w[c, k] * window[k],  SiLU if requested,
+// and afterwards the cache holds the last K-1 raw inputs (exact copies).
+//
+// Layout: a thread owns VEC = 16 bytes of consecutive channels and TT
+// consecutive tokens; the raw-input history it needs before its first token
+// comes from the input itself (t >= 0) or from the cache (t < 0). Only the
+// CTAs of the first token tile read the cache, and those same CTAs write the
+// new cache rows afterwards, so no other CTA can observe a half-rolled cache.
+#include <cuda_runtime.h>
+
+#include "m2_device.cuh"
+#include "m2_internal.cuh"
+
+namespace m2 {
+namespace {
+
+constexpr int kConvThreads = 128;
+constexpr int kTT = 16;  // tokens per thread
+
+// Store VEC floats as OT at p (VEC * sizeof(OT) is 16 or 32 bytes, or 8 for
+// four bf16 outputs of fp32 inputs).
+template <typename OT, int VEC>
+__device__ __forceinline__ void store_vec(OT* p, const float* o) {
+    if constexpr (sizeof(OT) == 2 && VEC == 4) {
+        *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
+    } else {
+        constexpr int OVEC = Vec16<OT>::n;
+        static_assert(VEC % OVEC == 0, "whole 16-byte output vectors");
+#pragma unroll
+        for (int v = 0; v < VEC; v += OVEC) *reinterpret_cast<uint4*>(p + v) = pack16<OT>(o + v);
+    }
+}
+
+template <typename AT, typename OT, int K>
+__global__ void __launch_bounds__(kConvThreads) conv1d_kernel(const ConvArgs a) {
+    constexpr int VEC = Vec16<AT>::n;
+    const int b = blockIdx.z;
+    const int t0 = blockIdx.y * kTT;
+    const int64_t c0 = (static_cast<int64_t>(blockIdx.x) * kConvThreads + threadIdx.x) * VEC;
+    if (c0 >= a.conv_dim) return;
+    const int T = a.seqlen;
+    const int t_end = min(t0 + kTT, T);
+
+    const int32_t slot = a.slot_idx[b];
+    const AT* xb = static_cast<const AT*>(a.x) + static_cast<int64_t>(b) * T * a.x_stride;
+    OT* ob = static_cast<OT*>(a.out) + static_cast<int64_t>(b) * T * a.out_stride;
+    if (slot < 0) {  // padding row: zero output, cache untouched
+        float zeros[VEC];
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) zeros[v] = 0.f;
+        for (int t = t0; t < t_end; ++t) store_vec<OT, VEC>(ob + t * a.out_stride + c0, zeros);
+        return;
+    }
+    if (slot >= a.num_slots) {
+        if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) record_error(a.error, M2_ERR_BAD_SLOT);
+        return;
+    }
+    AT* cache = static_cast<AT*>(a.conv) + static_cast<int64_t>(slot) * (K - 1) * a.conv_dim;
+
+    // weights and bias of the VEC channels, as float
+    float w[VEC][K];
+    float bias[VEC];
+    {
+        const AT* wp = static_cast<const AT*>(a.w) + c0 * K;
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) {
+#pragma unroll
+            for (int k = 0; k < K; ++k) w[v][k] = to_f32(wp[v * K + k]);
+            bias[v] = a.b ? to_f32(static_cast<const AT*>(a.b)[c0 + v]) : 0.f;
+        }
+    }
+
+    // history: raw vectors of tokens t0-K+1 .. t0-1 (oldest first)
+    uint4 hist_raw[K - 1];
+#pragma unroll
+    for (int j = 0; j < K - 1; ++j) {
+        const int t = t0 - (K - 1) + j;
+        hist_raw[j] = t >= 0 ? *reinterpret_cast<const uint4*>(xb + t * a.x_stride + c0)
+                             : *reinterpret_cast<const uint4*>(cache + (K - 1 + t) * a.conv_dim + c0);
+    }
+    float hist[K - 1][VEC];
+#pragma unroll
+    for (int j = 0; j < K - 1; ++j) unpack16<AT>(hist_raw[j], hist[j]);
+
+#pragma unroll
+    for (int i = 0; i < kTT; ++i) {
+        const int t = t0 + i;
+        if (t < t_end) {
+            float cur[VEC];
+            unpack16<AT>(*reinterpret_cast<const uint4*>(xb + t * a.x_stride + c0), cur);
+            float o[VEC];
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) {
+                float acc = bias[v];
+#pragma unroll
+                for (int k = 0; k < K - 1; ++k) acc = fmaf(w[v][k], hist[k][v], acc);
+                acc = fmaf(w[v][K - 1], cur[v], acc);
+                o[v] = a.activation ? silu_f32(acc) : acc;
+            }
+            store_vec<OT, VEC>(ob + t * a.out_stride + c0, o);
+#pragma unroll
+            for (int k = 0; k < K - 2; ++k) {
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) hist[k][v] = hist[k + 1][v];
+            }
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) hist[K - 2][v] = cur[v];
+        }
+    }
+
+    if (blockIdx.y == 0) {
+        // new cache row k holds the raw input of token T-(K-1)+k: from the input
+        // when that token exists, else from the old cache rows read above
+        // (only possible when T < K-1, in which case this tile saw every token)
+#pragma unroll
+        for (int k = 0; k < K - 1; ++k) {
+            const int t = T - (K - 1) + k;
+            uint4 v;
+            if (t >= 0) {
+                v = *reinterpret_cast<const uint4*>(xb + t * a.x_stride + c0);
+            } else {
+#pragma unroll
+                for (int j = 0; j < K - 1; ++j) {
+                    if (j == k + T) v = hist_raw[j];  // old cache row k + T
+                }
+            }
+            *reinterpret_cast<uint4*>(cache + k * a.conv_dim + c0) = v;
+        }
+    }
+}
+
+template <typename AT, typename OT>
+cudaError_t conv_by_k(const ConvArgs& a, cudaStream_t s) {
+    constexpr int VEC = Vec16<AT>::n;
+    const dim3 grid(static_cast<unsigned>((a.conv_dim / VEC + kConvThreads - 1) / kConvThreads),
+                    static_cast<unsigned>((a.seqlen + kTT - 1) / kTT), static_cast<unsigned>(a.batch));
+    switch (a.K) {
+        case 2: conv1d_kernel<AT, OT, 2><<<grid, kConvThreads, 0, s>>>(a); break;
+        case 3: conv1d_kernel<AT, OT, 3><<<grid, kConvThreads, 0, s>>>(a); break;
+        case 4: conv1d_kernel<AT, OT, 4><<<grid, kConvThreads, 0, s>>>(a); break;
+        case 5: conv1d_kernel<AT, OT, 5><<<grid, kConvThreads, 0, s>>>(a); break;
+        case 6: conv1d_kernel<AT, OT, 6><<<grid, kConvThreads, 0, s>>>(a); break;
+        case 7: conv1d_kernel<AT, OT, 7><<<grid, kConvThreads, 0, s>>>(a); break;
+        case 8: conv1d_kernel<AT, OT, 8><<<grid, kConvThreads, 0, s>>>(a); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+// Zero the SSM and conv regions of n slots; one CTA row per slot.
+__global__ void __launch_bounds__(256) zero_slots_kernel(const ZeroArgs a) {
+    const int32_t slot = a.slot_idx[blockIdx.y];
+    if (slot < 0) return;
+    if (slot >= a.num_slots) {
+        if (threadIdx.x == 0 && blockIdx.x == 0) record_error(a.error, M2_ERR_BAD_SLOT);
+        return;
+    }
+    const uint4 zero = make_uint4(0, 0, 0, 0);
+    uint4* ssm = reinterpret_cast<uint4*>(static_cast<char*>(a.ssm) + slot * a.ssm_bytes_per_slot);
+    uint4* conv = reinterpret_cast<uint4*>(static_cast<char*>(a.conv) + slot * a.conv_bytes_per_slot);
+    const int64_t n_ssm = a.ssm_bytes_per_slot / 16;
+    const int64_t n_conv = a.conv_bytes_per_slot / 16;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_ssm; i += stride)
+        st_stream(ssm + i, zero);
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_conv; i += stride)
+        conv[i] = zero;
+}
+
+}  // namespace
+
+cudaError_t launch_conv1d_update(const ConvArgs& a, cudaStream_t s) {
+    if (a.act_bf16) return a.out_bf16 ? conv_by_k<bf16_t, bf16_t>(a, s) : conv_by_k<bf16_t, float>(a, s);
+    return a.out_bf16 ? conv_by_k<float, bf16_t>(a, s) : conv_by_k<float, float>(a, s);
+}
+
+cudaError_t launch_zero_slots(const ZeroArgs& a, cudaStream_t s) {
+    if (a.n == 0) return cudaSuccess;
+    const dim3 grid(32, static_cast<unsigned>(a.n));
+    zero_slots_kernel<<<grid, 256, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace m2

@@ -1,0 +1,115 @@
+// m2_internal.cuh -- declarations shared by the libm2 translation units.
+// Not installed; the public ABI is include/m2.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "m2.h"
+
+namespace m2 {
+
+// Everything a decode-step launch needs (host-validated).
+struct StateUpdateArgs {
+    void* ssm;
+    void* conv;
+    int32_t* error;
+    int64_t num_slots;
+    int H, P, N, G, K;
+    int64_t conv_dim;
+    int state_bf16, act_bf16, x_bf16;
+    const float* A_log;
+    const float* dt_bias;
+    const float* D;
+    const void* conv_w;
+    const void* conv_b;
+    int activation;
+    int fused;
+    int batch;
+    const void* xBC;
+    int64_t xBC_stride;
+    const void* dt;
+    int64_t dt_stride;
+    const void* z;
+    int64_t z_stride;
+    void* y;
+    int64_t y_stride;
+    const int32_t* slot_idx;
+};
+
+struct ConvArgs {
+    void* conv;
+    int32_t* error;
+    int64_t num_slots;
+    int K;
+    int64_t conv_dim;
+    int act_bf16, out_bf16;
+    const void* w;
+    const void* b;
+    int activation;
+    int batch, seqlen;
+    const void* x;
+    int64_t x_stride;
+    void* out;
+    int64_t out_stride;
+    const int32_t* slot_idx;
+};
+
+struct ZeroArgs {
+    void* ssm;
+    void* conv;
+    int32_t* error;
+    int64_t num_slots;
+    int64_t ssm_bytes_per_slot;
+    int64_t conv_bytes_per_slot;
+    int n;
+    const int32_t* slot_idx;
+};
+
+struct ScanArgs {
+    void* ssm;
+    int32_t* error;
+    int64_t num_slots;
+    int H, P, N, G;
+    int state_bf16, act_bf16, x_bf16;
+    const float* A_log;
+    const float* dt_bias;
+    const float* D;
+    int batch, seqlen, chunk;
+    const void* xBC;
+    int64_t xBC_stride;
+    const void* dt;
+    int64_t dt_stride;
+    const void* z;
+    int64_t z_stride;
+    void* y;
+    int64_t y_stride;
+    const int32_t* slot_idx;
+    const uint8_t* has_init;
+};
+
+// Launch-shape query for the decode kernels: M2_OK and the shape, or
+// M2_ERR_UNSUPPORTED. Pure host arithmetic.
+struct DecodePlan {
+    int loads;        // 16-byte loads per thread
+    int tile_rows;    // state rows (of N elements) per CTA
+    int ctas_per_seq; // H*P / tile_rows
+    int cluster;      // CTAs per group when the conv is fused (1 otherwise)
+};
+m2_status plan_state_update(int H, int P, int N, int G, int state_bf16, int fused,
+                            DecodePlan* plan);
+
+cudaError_t launch_state_update(const StateUpdateArgs& a, const DecodePlan& plan,
+                                cudaStream_t stream);
+cudaError_t launch_conv1d_update(const ConvArgs& a, cudaStream_t stream);
+cudaError_t launch_zero_slots(const ZeroArgs& a, cudaStream_t stream);
+m2_status plan_chunk_scan(int H, int P, int N, int G, int state_bf16, int act_bf16, int x_bf16,
+                          int chunk);
+cudaError_t launch_chunk_scan(const ScanArgs& a, cudaStream_t stream);
+
+// Records `code` in the error word unless an earlier error is already there.
+__device__ __forceinline__ void record_error(int32_t* error, int32_t code) {
+    if (error) atomicCAS(error, 0, code);
+}
+
+}  // namespace m2

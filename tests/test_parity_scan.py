@@ -1,0 +1,178 @@
+"""Chunked prefill scan against the oracle's definition (T sequential updates
+with the working state unrounded until the end), the T = 1 equivalence with
+the decode step, and the prefill-then-decode workload (8 x 2048 tokens, then
+32 decode steps continuing from the scanned state)."""
+
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+import pytest
+import torch
+
+import m2synth as S
+import mamba_recurrent_state_b200 as m2
+import oracle as O
+from m2synth import T_DT, T_XBC, T_Z
+from m2synth import torch_inputs as TI
+from m2synth import workloads as W
+from parity_util import OracleLayer, assert_close, f64, rel_err, TOL
+from test_parity_decode import layer_objs, make_cache, shape_of
+
+pytestmark = pytest.mark.gpu
+
+
+def wl(index, H=8, G=2, sd=S.BF16, ad=S.BF16, N=128, batch=3, slots=6, T=37, chunk=16):
+    return W.Workload(index, f"scan{index}", H, 64, N, G, 4, sd, ad, slots, batch, seqlen=T,
+                      chunk=chunk)
+
+
+def prefill_inputs(w, xdtype=None):
+    """Post-conv inputs are drawn directly here (the scan takes post-conv xBC)."""
+    rows = w.batch * w.seqlen
+    d = TI.step_tensors(w, 0, rows=rows)
+    x = d["xBC"] if xdtype is None else d["xBC"].to(xdtype)
+    return (x.view(w.batch, w.seqlen, -1), d["dt"].view(w.batch, w.seqlen, -1),
+            d["z"].view(w.batch, w.seqlen, -1))
+
+
+def oracle_scan_row(ol, w, b, s, init: bool, x_code):
+    rows = np.arange(b * w.seqlen, (b + 1) * w.seqlen)
+    xbc = f64(W.step_rows(w, T_XBC, 0, rows), w.act_dtype)
+    if x_code != w.act_dtype:  # xBC handed over in another precision
+        xbc = ol.orc.round_array(xbc, O.ROUND_F32 if x_code == S.F32 else O.ROUND_BF16)
+    dt = f64(W.step_rows(w, T_DT, 0, rows), w.act_dtype)
+    z = f64(W.step_rows(w, T_Z, 0, rows), w.act_dtype)
+    state = ol.initial_ssm(s) if init else np.zeros((w.H, w.P, w.N))
+    y = ol.orc.ssm_scan(state, O.round_mode_for(w.state_dtype), xbc, dt, ol.dt_bias, ol.A_log,
+                        ol.D, z, w.G)
+    return state, y
+
+
+@pytest.mark.parametrize("w", [
+    wl(300),
+    wl(301, T=1),
+    wl(302, T=200, chunk=64),
+    wl(303, sd=S.F32, ad=S.BF16, T=50),
+    wl(304, sd=S.F32, ad=S.F32, T=20, N=64),
+    wl(305, H=16, G=16, T=33, batch=2),
+], ids=lambda w: f"H{w.H}G{w.G}N{w.N}s{w.state_dtype}a{w.act_dtype}T{w.seqlen}")
+def test_scan_small(w):
+    cache = make_cache(w)
+    ssm0 = cache.ssm.clone()
+    t, ssm, _ = layer_objs(w)
+    slot_list = [5, -1, 2][: w.batch]
+    init_list = [1, 0, 0][: w.batch]
+    slots = torch.tensor(slot_list, dtype=torch.int32, device="cuda")
+    init = torch.tensor(init_list, dtype=torch.uint8, device="cuda")
+    x, dt, z = prefill_inputs(w)
+    y = m2.chunk_scan(cache, ssm, x, dt, slots, z=z, chunk_size=w.chunk, has_initial_state=init)
+    torch.cuda.synchronize()
+    ol = OracleLayer(w)
+    for b, s in enumerate(slot_list):
+        if s < 0:
+            assert torch.count_nonzero(y[b]) == 0
+            continue
+        state, y_ref = oracle_scan_row(ol, w, b, s, bool(init_list[b]), w.act_dtype)
+        assert_close(f64(TI.to_storage_np(y[b]), w.act_dtype), y_ref, w.act_dtype, f"y row {b}")
+        assert_close(f64(TI.to_storage_np(cache.ssm[s]), w.state_dtype), state, w.state_dtype,
+                     f"final state row {b}")
+    keep = [q for q in range(w.num_slots) if q not in slot_list]
+    assert torch.equal(cache.ssm[keep], ssm0[keep])
+    assert cache.device_error() == 0
+
+
+def test_scan_fp32_xbc_input():
+    w = wl(306, T=24)
+    cache = make_cache(w)
+    t, ssm, _ = layer_objs(w)
+    slots = torch.tensor([0, 3, 4], dtype=torch.int32, device="cuda")
+    x, dt, z = prefill_inputs(w, xdtype=torch.float32)
+    y = m2.chunk_scan(cache, ssm, x, dt, slots, z=z)
+    torch.cuda.synchronize()
+    ol = OracleLayer(w)
+    for b, s in enumerate([0, 3, 4]):
+        state, y_ref = oracle_scan_row(ol, w, b, s, False, S.F32)
+        assert_close(f64(TI.to_storage_np(y[b]), w.act_dtype), y_ref, w.act_dtype, "y")
+        assert_close(f64(TI.to_storage_np(cache.ssm[s]), w.state_dtype), state, w.state_dtype, "S")
+
+
+@pytest.mark.parametrize("G", [1, 8])
+def test_scan_T1_equals_state_update(G):
+    """A one-token scan from the cached state equals one decode step on the
+    same post-conv input (including n_groups = 8): the state bit for bit (same
+    fp32 arithmetic per element), y within tolerance."""
+    w = W.Workload(310 + G, "t1", 128, 64, 128, G, 4, S.BF16, S.BF16, 16, 8, seqlen=1)
+    a = make_cache(w)
+    b = m2.Cache(shape_of(w), w.num_slots, ssm=a.ssm.clone(), conv=a.conv.clone())
+    t, ssm, _ = layer_objs(w)
+    x, dt, z = prefill_inputs(w)
+    ones = torch.ones(w.batch, dtype=torch.uint8, device="cuda")
+    y_scan = m2.chunk_scan(a, ssm, x, dt, t["slots"], z=z, chunk_size=128, has_initial_state=ones)
+    y_dec = m2.state_update(b, ssm, x[:, 0], dt[:, 0], t["slots"], z=z[:, 0])
+    torch.cuda.synchronize()
+    assert torch.equal(a.ssm, b.ssm)
+    e = rel_err(f64(TI.to_storage_np(y_scan[:, 0]), S.BF16), f64(TI.to_storage_np(y_dec), S.BF16))
+    assert e <= TOL[S.BF16], e
+
+
+def test_workload4_prefill_then_decode():
+    """Zero initial state; prefill conv over 2048 tokens (bf16 post-conv buffer),
+    chunk scan, then 32 fused decode steps continuing from the scanned state.
+    Every y and the final states of all 8 sequences are checked."""
+    w = W.WORKLOADS[4]
+    cache = make_cache(w)
+    t, ssm, conv = layer_objs(w)
+    cache.zero_slots(t["slots"])
+    T = w.seqlen
+    d = TI.step_tensors(w, 0, rows=w.batch * T)
+    xr = d["xBC"].view(w.batch, T, -1)
+    xp = m2.conv1d_update(cache, conv, xr, t["slots"], out_dtype=torch.bfloat16)
+    y_pre = m2.chunk_scan(cache, ssm, xp, d["dt"].view(w.batch, T, -1), t["slots"],
+                          z=d["z"].view(w.batch, T, -1), chunk_size=w.chunk)
+    state_after_prefill = TI.to_storage_np(cache.ssm[t["slots"].long()])
+    y_dec = []
+    for step in range(1, w.decode_after + 1):
+        inp = TI.step_tensors(w, step)
+        y_dec.append(m2.state_update(cache, ssm, inp["xBC"], inp["dt"], t["slots"], z=inp["z"],
+                                     conv=conv))
+    torch.cuda.synchronize()
+    y_pre_np = TI.to_storage_np(y_pre)
+    y_dec_np = np.stack([TI.to_storage_np(y) for y in y_dec])
+    ssm_np = TI.to_storage_np(cache.ssm)
+    conv_np = TI.to_storage_np(cache.conv)
+    ol = OracleLayer(w)
+
+    def one(b):
+        s = int(ol.slots[b])
+        rows = np.arange(b * T, (b + 1) * T)
+        conv_state = np.zeros((w.K - 1, w.conv_dim))
+        xraw = f64(W.step_rows(w, T_XBC, 0, rows), w.act_dtype)
+        xpost = ol.orc.conv1d(conv_state, xraw, ol.conv_w, ol.conv_b, 1)
+        xpost = ol.orc.round_array(xpost, O.ROUND_BF16)  # the bf16 buffer between the launches
+        dt = f64(W.step_rows(w, T_DT, 0, rows), w.act_dtype)
+        z = f64(W.step_rows(w, T_Z, 0, rows), w.act_dtype)
+        state = np.zeros((w.H, w.P, w.N))
+        y = ol.orc.ssm_scan(state, O.ROUND_BF16, xpost, dt, ol.dt_bias, ol.A_log, ol.D, z, w.G)
+        errs = {"prefill_y": rel_err(f64(y_pre_np[b], w.act_dtype), y),
+                "prefill_state": rel_err(f64(state_after_prefill[b], w.state_dtype), state)}
+        dec = []
+        for step in range(1, w.decode_after + 1):
+            inp = ol.inputs(step, [b])
+            yd = O.decode_rows(ol.orc, w.H, w.P, w.N, w.G, O.ROUND_BF16, [state], [conv_state],
+                               inp["xBC"], inp["dt"], inp["z"], ol.conv_w, ol.conv_b, ol.dt_bias,
+                               ol.A_log, ol.D, threads=1)
+            dec.append(rel_err(f64(y_dec_np[step - 1][b], w.act_dtype), yd))
+        errs["decode_y"] = max(dec)
+        errs["final_state"] = rel_err(f64(ssm_np[s], w.state_dtype), state)
+        errs["conv_exact"] = bool(np.array_equal(conv_np[s], S.to_storage(conv_state, w.act_dtype)))
+        return errs
+
+    with ThreadPoolExecutor(max_workers=8) as ex:
+        results = list(ex.map(one, range(w.batch)))
+    for b, e in enumerate(results):
+        assert e["prefill_y"] <= TOL[S.BF16], (b, e)
+        assert e["prefill_state"] <= TOL[S.BF16], (b, e)
+        assert e["decode_y"] <= TOL[S.BF16], (b, e)
+        assert e["final_state"] <= TOL[S.BF16], (b, e)
+        assert e["conv_exact"], (b, e)
+    assert cache.device_error() == 0
