@@ -46,7 +46,7 @@ KERNEL_SOURCES = ["mamba_recurrent_state_b200/csrc/m2_state_update.cu",
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -87,37 +87,43 @@ def profiled_traffic() -> float | None:
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """nvidia-smi clocks and throttle reasons, sampled every 50 ms while the
+    benchmark runs; only samples that arrive inside the timed region count."""
 
     QUERY = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.lines: list[str] = []
+        self.samples: list[tuple[float, str]] = []
         self.thread = None
 
     def start(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
             return
         self.thread = threading.Thread(target=self._read, daemon=True)
         self.thread.start()
+        t0 = time.monotonic()  # wait for the first sample (nvidia-smi start-up)
+        while not self.samples and time.monotonic() - t0 < 5.0:
+            time.sleep(0.05)
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.samples.append((time.monotonic(), line.strip()))
 
-    def stop(self) -> dict | None:
+    def stop(self, t_begin: float, t_end: float) -> dict | None:
         if self.proc is None:
             return None
+        time.sleep(0.1)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -125,8 +131,9 @@ class ClockSampler:
             self.proc.kill()
         self.thread.join(timeout=2)
         sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ts, ln in self.samples:
+            if not (t_begin <= ts <= t_end + 0.06):
+                continue
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 7:
                 continue
@@ -135,11 +142,12 @@ class ClockSampler:
                 mx.append(float(parts[1]))
             except ValueError:
                 continue
-            for n, v in zip(names, parts[3:7]):
+            for n, v in zip(self.REASONS, parts[3:7]):
                 if v.lower() == "active":
                     reasons.add(n)
         if not sm:
-            return None
+            return {"sm_mhz": None, "sm_max_mhz": None, "samples": 0, "reasons": [],
+                    "note": "no nvidia-smi sample landed inside the timed region"}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
                 "reasons": sorted(reasons)}
 
@@ -281,14 +289,16 @@ def run_ours(args, world, rank, local):
     sampler.start()
     barrier(world)
     torch.cuda.synchronize()
+    t_begin = time.monotonic()
     for i in range(args.steps):
         flush.zero_()
         starts[i].record(stream)
         step(i)
         ends[i].record(stream)
     torch.cuda.synchronize()
+    t_end = time.monotonic()
     barrier(world)
-    clocks = sampler.stop()
+    clocks = sampler.stop(t_begin, t_end)
     kern_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = max_over_ranks(sum(kern_ms), world)
     if cache.device_error() != 0:

@@ -10,15 +10,22 @@
 //
 // Work decomposition (HBM-bound: ~96% of the bytes are the state stream).
 //  * A sequence's state [H, P, N] is a run of H*P rows of N elements. One CTA
-//    of 256 threads owns TILE = 8 warps x RPW rows x LOADS consecutive rows, so
-//    its slice of the cache is one contiguous block (64 KB with LOADS = 16).
-//  * A row is read by LPR = N*sizeof(state)/16 lanes, one 16-byte vector each,
-//    so every lane keeps the same EPV state columns n for all of its rows and
-//    holds B[g, n] and C[g, n] for those columns in registers. A warp load
-//    instruction covers 512 contiguous bytes.
-//  * Each thread issues all LOADS 16-byte loads of the tile before any
-//    arithmetic (up to 64 KB in flight per CTA), then updates, stores and
-//    reduces y over its LPR lanes with xor shuffles.
+//    of 256 threads owns TILE consecutive rows, one contiguous block of the
+//    cache (64 KB in the main configuration), split in CHUNKS chunks.
+//  * Right after reading its slot index, one thread issues the whole tile as
+//    bulk asynchronous copies (cp.async.bulk) into shared memory, one
+//    mbarrier per chunk, so the tile's bytes are in flight while the CTA runs
+//    the conv tap and the per-head scalars. Registers are not used as the
+//    staging buffer, which lets three CTAs share an SM.
+//  * A state row is handled by LPR = N*sizeof(state)/16 lanes, one 16-byte
+//    vector each, so every lane keeps the same EPV state columns n for all of
+//    its rows and holds B[g, n] and C[g, n] for those columns in registers.
+//    Shared-memory reads are linear (conflict free); the new state goes
+//    straight from registers to global memory with 16-byte streaming stores.
+//    y is reduced over the LPR lanes with xor shuffles.
+//  * Waits on the copies are bounded (one second of %globaltimer); on a
+//    timeout the CTA records M2_ERR_TIMEOUT, waits once more (bounded) for its
+//    copies and skips the rest of its tile.
 //  * Fused conv: the CTA computes the conv tap for its own x channels (and
 //    rolls their conv-cache rows, which no other CTA touches) and for the
 //    group's B and C channels, which every CTA of the group needs. Those CTAs
@@ -33,9 +40,17 @@
 namespace m2 {
 namespace {
 
+// Tuning knobs (compile-time): resident CTAs per SM the register budget is
+// sized for, and 16 KB chunks per CTA tile in the main configuration.
+#ifndef M2_DECODE_MIN_BLOCKS
+#define M2_DECODE_MIN_BLOCKS 3
+#endif
+#ifndef M2_DECODE_MAIN_CHUNKS
+#define M2_DECODE_MAIN_CHUNKS 4
+#endif
+
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kMaxK = 8;
 constexpr int kMaxHeadsPerTile = 33;
 
 __device__ __forceinline__ void cluster_arrive() {
@@ -50,62 +65,144 @@ __device__ __forceinline__ uint32_t cluster_rank() {
     return r;
 }
 
-// Conv tap for channel c of one row: reads the K-1 cached raw inputs and the
-// new raw input, returns the post-conv value (bias, activation) and leaves the
-// raw window in win[] (oldest first, newest at K-1).
-template <typename AT>
-__device__ __forceinline__ float conv_tap(const AT* conv_row0, int64_t conv_dim, int K,
-                                          const AT* w, const AT* bias, int activation,
-                                          AT new_in, int64_t c, AT* win) {
-    float acc = bias ? to_f32(bias[c]) : 0.f;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // bounded waits: one second
+
+// Sums VPT row partials over the LPR lanes that share each row. For VPT = 4
+// the first two levels exchange only the halves each lane keeps
+// (reduce-scatter), so 4 rows cost 5 shuffles instead of 16. On return the
+// lanes with (lane % (LPR/VPT)) == 0 hold the sum of row `which`.
+template <int LPR, int VPT>
+__device__ __forceinline__ float reduce_rows(const float (&acc)[VPT], int lane, int& which) {
+    static_assert(VPT == 1 || VPT == 4, "one or four rows per thread");
+    static_assert(LPR >= VPT, "reduce-scatter needs at least one lane per row");
+    if constexpr (VPT == 1) {
+        float v = acc[0];
 #pragma unroll
-    for (int k = 0; k < kMaxK; ++k) {
-        if (k < K) {
-            const AT v = (k < K - 1) ? conv_row0[static_cast<int64_t>(k) * conv_dim + c] : new_in;
-            win[k] = v;
-            acc = fmaf(to_f32(w[c * K + k]), to_f32(v), acc);
+        for (int off = LPR / 2; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        which = 0;
+        return v;
+    } else {
+        const bool hi1 = (lane & (LPR / 2)) != 0;   // keeps rows 2,3 instead of 0,1
+        const float s0 = hi1 ? acc[0] : acc[2];
+        const float s1 = hi1 ? acc[1] : acc[3];
+        const float k0 = (hi1 ? acc[2] : acc[0]) + __shfl_xor_sync(0xffffffffu, s0, LPR / 2);
+        const float k1 = (hi1 ? acc[3] : acc[1]) + __shfl_xor_sync(0xffffffffu, s1, LPR / 2);
+        const bool hi2 = (lane & (LPR / 4)) != 0;   // keeps the odd row of the pair
+        float v = (hi2 ? k1 : k0) + __shfl_xor_sync(0xffffffffu, hi2 ? k0 : k1, LPR / 4);
+#pragma unroll
+        for (int off = LPR / 8; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        which = (hi1 ? 2 : 0) + (hi2 ? 1 : 0);
+        return v;
+    }
+}
+
+// Conv tap of AV consecutive channels c0.. for one row: the K-1 cached raw
+// inputs (staged in shared memory at `rows`, row pitch `pitch` elements,
+// oldest first) and the raw input `xin`; tap K-1 multiplies the newest input.
+// Weights and bias are loaded before waiting for the staged rows. Returns
+// false if the bounded wait for the rows ran out.
+template <typename AT, int AV>
+__device__ __forceinline__ bool conv_vec_k4(const uint4& xin, const AT* w, const AT* bias, int64_t c0,
+                                            const AT* rows, int64_t pitch, int activation,
+                                            uint64_t* bar, float (&out)[AV]) {
+    constexpr int K = 4;
+    // the AV x K weight block is exactly K 16-byte vectors; (e, k) sits at e*K + k
+    uint4 wv[K];
+#pragma unroll
+    for (int q = 0; q < K; ++q) wv[q] = __ldg(reinterpret_cast<const uint4*>(w + c0 * K) + q);
+    float wf[AV * K];
+#pragma unroll
+    for (int q = 0; q < K; ++q) unpack16<AT>(wv[q], wf + q * AV);
+#pragma unroll
+    for (int e = 0; e < AV; ++e) out[e] = bias ? to_f32(__ldg(bias + c0 + e)) : 0.f;
+    if (!mbar_wait_bounded(bar, 0, kWaitLimitNs)) return false;
+    float xv[AV];
+    unpack16<AT>(xin, xv);
+#pragma unroll
+    for (int k = 0; k < K - 1; ++k) {
+        float rv[AV];
+        unpack16<AT>(*reinterpret_cast<const uint4*>(rows + k * pitch), rv);
+#pragma unroll
+        for (int e = 0; e < AV; ++e) out[e] = fmaf(wf[e * K + k], rv[e], out[e]);
+    }
+#pragma unroll
+    for (int e = 0; e < AV; ++e) {
+        out[e] = fmaf(wf[e * K + K - 1], xv[e], out[e]);
+        if (activation) out[e] = silu_f32(out[e]);
+    }
+    return true;
+}
+
+// Same for any width K (2..8): weights read one by one (cached).
+template <typename AT, int AV>
+__device__ __forceinline__ bool conv_vec_any(const uint4& xin, const AT* w, const AT* bias, int64_t c0,
+                                             int K, const AT* rows, int64_t pitch, int activation,
+                                             uint64_t* bar, float (&out)[AV]) {
+#pragma unroll
+    for (int e = 0; e < AV; ++e) out[e] = bias ? to_f32(__ldg(bias + c0 + e)) : 0.f;
+    if (!mbar_wait_bounded(bar, 0, kWaitLimitNs)) return false;
+    float xv[AV];
+    unpack16<AT>(xin, xv);
+#pragma unroll
+    for (int e = 0; e < AV; ++e) {
+        for (int k = 0; k < K; ++k) {
+            const float in = (k < K - 1) ? to_f32(rows[k * pitch + e]) : xv[e];
+            out[e] = fmaf(to_f32(__ldg(w + (c0 + e) * K + k)), in, out[e]);
         }
+        if (activation) out[e] = silu_f32(out[e]);
     }
-    return activation ? silu_f32(acc) : acc;
+    return true;
 }
 
-// Roll: conv[k] <- win[k+1] for k < K-1 (exact copies of raw inputs).
-template <typename AT>
-__device__ __forceinline__ void conv_roll(AT* conv_row0, int64_t conv_dim, int K, int64_t c,
-                                          const AT* win) {
-#pragma unroll
-    for (int k = 0; k < kMaxK - 1; ++k) {
-        if (k < K - 1) conv_row0[static_cast<int64_t>(k) * conv_dim + c] = win[k + 1];
-    }
-}
-
-template <typename ST, typename AT, typename XT, int N, int LOADS, bool FUSED>
-__global__ void __launch_bounds__(kThreads)
+template <typename ST, typename AT, typename XT, int N, int CHUNKS, int VPT, bool FUSED>
+__global__ void __launch_bounds__(kThreads, M2_DECODE_MIN_BLOCKS)
 state_update_kernel(const StateUpdateArgs a) {
     constexpr int EPV = Vec16<ST>::n;       // state elements per 16-byte vector
     constexpr int LPR = N / EPV;            // lanes per state row
     static_assert(LPR >= 1 && LPR <= 32 && (32 % LPR) == 0, "row must fit a warp");
-    constexpr int RPW = 32 / LPR;           // rows per warp load instruction
-    constexpr int TILE = kWarps * RPW * LOADS;
+    constexpr int RPP = kThreads / LPR;     // rows per pass of the CTA
+    constexpr int RC = RPP * VPT;           // rows per chunk
+    constexpr int TILE = RC * CHUNKS;       // rows per CTA
+    constexpr uint32_t CHUNK_BYTES = RC * N * sizeof(ST);
+    constexpr uint32_t TILE_BYTES = CHUNK_BYTES * CHUNKS;
+    static_assert(CHUNK_BYTES % 16 == 0, "bulk copies move multiples of 16 bytes");
+    constexpr int AV = Vec16<AT>::n;        // activation elements per 16-byte vector
+    constexpr int XV = TILE / AV;           // 16-byte vectors of x channels in the tile
+    constexpr int BV = N / AV;              // 16-byte vectors of one B (or C) segment
+    static_assert(TILE % AV == 0 && N % AV == 0, "whole activation vectors");
+    constexpr uint32_t XROW_BYTES = TILE * sizeof(AT);
+    constexpr uint32_t BROW_BYTES = N * sizeof(AT);
+    constexpr int kHalf = kThreads / 2;     // x-conv threads | B/C-conv threads
 
-    __shared__ float s_x[TILE];
-    __shared__ float s_B[N];
-    __shared__ float s_C[N];
+    // dynamic: [state tile | conv rows of the tile's x channels | conv rows of B, C]
+    extern __shared__ __align__(128) uint8_t s_dyn[];
+    uint8_t* s_tile = s_dyn;
+    const AT* s_cx = reinterpret_cast<const AT*>(s_dyn + TILE_BYTES);                 // [K-1][TILE]
+    const AT* s_cbc = reinterpret_cast<const AT*>(s_dyn + TILE_BYTES + (a.K - 1) * XROW_BYTES);  // [K-1][2][N]
+    __shared__ __align__(8) uint64_t s_bar[CHUNKS + 1];  // one per state chunk, one for the conv rows
+    __shared__ __align__(16) float4 s_rp[TILE];          // per row: dt*x, dA, D*x
+    __shared__ __align__(16) float s_B[N];
+    __shared__ __align__(16) float s_C[N];
     __shared__ float s_y[TILE];
     __shared__ float s_dt[kMaxHeadsPerTile];
     __shared__ float s_dA[kMaxHeadsPerTile];
     __shared__ float s_D[kMaxHeadsPerTile];
+    __shared__ int s_fail;
 
     const int tid = threadIdx.x;
     const int b = blockIdx.y;
     const int64_t r0 = static_cast<int64_t>(blockIdx.x) * TILE;  // first row (h*P + p)
     const int P = a.P;
     const int H = a.H;
+    const int K = a.K;
     const int64_t HP = static_cast<int64_t>(H) * P;
     const int hpg = H / a.G;
     const int h_first = static_cast<int>(r0 / P);
     const int g = h_first / hpg;
     const int n_heads_tile = static_cast<int>((r0 + TILE - 1) / P) - h_first + 1;
+    const int64_t cd = a.conv_dim;
+    const int64_t cB = HP + static_cast<int64_t>(g) * N;                        // first B channel
+    const int64_t cC = HP + static_cast<int64_t>(a.G) * N + static_cast<int64_t>(g) * N;
 
     const int32_t slot = a.slot_idx[b];
     const AT* zrow = a.z ? static_cast<const AT*>(a.z) + b * a.z_stride : nullptr;
@@ -120,129 +217,219 @@ state_update_kernel(const StateUpdateArgs a) {
         return;
     }
 
-    // ---- phase 1: per-head scalars, post-conv x / B / C into shared memory
-    if (tid < n_heads_tile) {
-        const int h = h_first + tid;
+    // ---- phase 0: the slot's conv rows, then the whole state tile, go in flight
+    ST* tile = static_cast<ST*>(a.ssm) + (static_cast<int64_t>(slot) * HP + r0) * N;
+    AT* conv0 = static_cast<AT*>(a.conv) + static_cast<int64_t>(slot) * (K - 1) * cd;
+    uint64_t* bar_conv = &s_bar[CHUNKS];
+    if (tid == 0) {
+        s_fail = 0;
+#pragma unroll
+        for (int c = 0; c <= CHUNKS; ++c) mbar_init(&s_bar[c], 1);
+        fence_mbar_init();
+        if constexpr (FUSED) {
+            mbar_arrive_expect_tx(bar_conv, (K - 1) * (XROW_BYTES + 2 * BROW_BYTES));
+            uint8_t* dst = s_dyn + TILE_BYTES;
+            for (int k = 0; k < K - 1; ++k)
+                bulk_g2s(dst + k * XROW_BYTES, conv0 + k * cd + r0, XROW_BYTES, bar_conv);
+            dst += (K - 1) * XROW_BYTES;
+            for (int k = 0; k < K - 1; ++k) {
+                bulk_g2s(dst + (2 * k) * BROW_BYTES, conv0 + k * cd + cB, BROW_BYTES, bar_conv);
+                bulk_g2s(dst + (2 * k + 1) * BROW_BYTES, conv0 + k * cd + cC, BROW_BYTES, bar_conv);
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < CHUNKS; ++c) {
+            mbar_arrive_expect_tx(&s_bar[c], CHUNK_BYTES);
+            bulk_g2s(s_tile + c * CHUNK_BYTES, reinterpret_cast<const uint8_t*>(tile) + c * CHUNK_BYTES,
+                     CHUNK_BYTES, &s_bar[c]);
+        }
+    }
+    // per-head scalars
+    for (int i = tid; i < n_heads_tile; i += kThreads) {
+        const int h = h_first + i;
         const float dtr = to_f32(static_cast<const AT*>(a.dt)[b * a.dt_stride + h]);
         const float dt = softplus_f32(dtr + a.dt_bias[h]);
         const float A = -expf(a.A_log[h]);
-        s_dt[tid] = dt;
-        s_dA[tid] = expf(dt * A);
-        s_D[tid] = a.D[h];
+        s_dt[i] = dt;
+        s_dA[i] = expf(dt * A);
+        s_D[i] = a.D[h];
     }
+    __syncthreads();  // barrier initialisation and head scalars visible to all threads
 
-    const int64_t cd = a.conv_dim;
-    const int64_t cB = HP + static_cast<int64_t>(g) * N;                        // first B channel
-    const int64_t cC = HP + static_cast<int64_t>(a.G) * N + static_cast<int64_t>(g) * N;
-    // raw windows of this thread's (at most two) B/C channels, kept for the roll
-    AT bc_win[2][kMaxK];
-
+    // ---- phase 1: post-conv x (into the row parameters) and B, C
     if constexpr (FUSED) {
         const AT* xrow = static_cast<const AT*>(a.xBC) + b * a.xBC_stride;
-        AT* conv0 = static_cast<AT*>(a.conv) + static_cast<int64_t>(slot) * (a.K - 1) * cd;
         const AT* w = static_cast<const AT*>(a.conv_w);
         const AT* bias = static_cast<const AT*>(a.conv_b);
-        for (int i = tid; i < TILE; i += kThreads) {  // private x channels
-            const int64_t c = r0 + i;
-            AT win[kMaxK];
-            s_x[i] = conv_tap(conv0, cd, a.K, w, bias, a.activation, xrow[c], c, win);
-            conv_roll(conv0, cd, a.K, c, win);
-        }
-        static_assert(2 * N <= 2 * kThreads, "B/C channels: at most two per thread");
+        const bool first_half = tid < kHalf;
+        const int nvec = first_half ? XV : 2 * BV;
+        for (int v = first_half ? tid : tid - kHalf; v < nvec; v += kHalf) {
+            // channel c0 .. c0+AV-1 and where its cached rows sit in shared memory
+            int64_t c0;
+            const AT* rows;
+            int64_t row_pitch;
+            if (first_half) {
+                c0 = r0 + static_cast<int64_t>(v) * AV;
+                rows = s_cx + v * AV;
+                row_pitch = TILE;
+            } else {
+                const int seg = v / BV;                        // 0 = B, 1 = C
+                const int j0 = (v % BV) * AV;
+                c0 = (seg ? cC : cB) + j0;
+                rows = s_cbc + seg * N + j0;
+                row_pitch = 2 * N;
+            }
+            // inputs that do not depend on the slot (raw x, weights, bias) are
+            // loaded before waiting for the slot's staged conv rows
+            const uint4 xin = *reinterpret_cast<const uint4*>(xrow + c0);
+            float out[AV];
+            bool got;
+            if (K == 4) {
+                got = conv_vec_k4<AT, AV>(xin, w, bias, c0, rows, row_pitch, a.activation, bar_conv, out);
+            } else {
+                got = conv_vec_any<AT, AV>(xin, w, bias, c0, K, rows, row_pitch, a.activation, bar_conv, out);
+            }
+            if (!got) {
+                record_error(a.error, M2_ERR_TIMEOUT);
+                s_fail = 1;
+                break;
+            }
+            if (first_half) {
+                // roll the private x rows: row k <- row k+1, last row <- raw input
+                for (int k = 0; k < K - 1; ++k) {
+                    const uint4 nv = (k < K - 2) ? *reinterpret_cast<const uint4*>(rows + (k + 1) * row_pitch) : xin;
+                    *reinterpret_cast<uint4*>(conv0 + k * cd + c0) = nv;
+                }
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {  // shared B / C channels
-            const int j = tid + q * kThreads;
-            if (j < 2 * N) {
-                const int64_t c = j < N ? cB + j : cC + (j - N);
-                const float v =
-                    conv_tap(conv0, cd, a.K, w, bias, a.activation, xrow[c], c, bc_win[q]);
-                if (j < N) s_B[j] = v; else s_C[j - N] = v;
+                for (int e = 0; e < AV; ++e) {
+                    const int r = v * AV + e;
+                    const int hl = static_cast<int>((r0 + r) / P) - h_first;
+                    s_rp[r] = make_float4(s_dt[hl] * out[e], s_dA[hl], s_D[hl] * out[e], 0.f);
+                }
+            } else {
+                float* dstf = (v / BV) ? s_C : s_B;
+#pragma unroll
+                for (int e = 0; e < AV; ++e) dstf[(v % BV) * AV + e] = out[e];
             }
         }
         // every CTA of the group has read the B/C conv rows once it arrives here
         cluster_arrive();
     } else {
         const XT* xrow = static_cast<const XT*>(a.xBC) + b * a.xBC_stride;
-        for (int i = tid; i < TILE; i += kThreads) s_x[i] = to_f32(xrow[r0 + i]);
+        for (int i = tid; i < TILE; i += kThreads) {
+            const int hl = static_cast<int>((r0 + i) / P) - h_first;
+            const float xv = to_f32(xrow[r0 + i]);
+            s_rp[i] = make_float4(s_dt[hl] * xv, s_dA[hl], s_D[hl] * xv, 0.f);
+        }
         for (int j = tid; j < N; j += kThreads) {
             s_B[j] = to_f32(xrow[cB + j]);
             s_C[j] = to_f32(xrow[cC + j]);
         }
     }
     __syncthreads();
+    bool ok = s_fail == 0;
 
-    // ---- phase 2: stream the state tile
-    const int warp = tid >> 5;
+    // ---- phase 2: update the tile chunk by chunk as the copies land
     const int lane = tid & 31;
-    const int sub = lane / LPR;          // row within a warp load
-    const int e0 = (lane % LPR) * EPV;   // first state column of this lane
-    float Bv[EPV], Cv[EPV];
+    const int e0 = (lane % LPR) * EPV;   // first state column of this thread (same in every pass)
+    static_assert(EPV % 2 == 0, "pairs of state columns");
+    float2 B2[EPV / 2], C2[EPV / 2];
 #pragma unroll
-    for (int e = 0; e < EPV; ++e) {
-        Bv[e] = s_B[e0 + e];
-        Cv[e] = s_C[e0 + e];
+    for (int e = 0; e < EPV / 2; ++e) {
+        B2[e] = make_float2(s_B[e0 + 2 * e], s_B[e0 + 2 * e + 1]);
+        C2[e] = make_float2(s_C[e0 + 2 * e], s_C[e0 + 2 * e + 1]);
     }
-
-    ST* tile = static_cast<ST*>(a.ssm) + (static_cast<int64_t>(slot) * HP + r0) * N;
-    uint4 v[LOADS];
-#pragma unroll
-    for (int i = 0; i < LOADS; ++i) {
-        const int row = (i * kWarps + warp) * RPW + sub;
-        v[i] = ld_stream(tile + static_cast<int64_t>(row) * N + e0);
-    }
-#pragma unroll
-    for (int i = 0; i < LOADS; ++i) {
-        const int row = (i * kWarps + warp) * RPW + sub;
-        const int hl = static_cast<int>((r0 + row) / P) - h_first;
-        const float xv = s_x[row];
-        const float dtx = s_dt[hl] * xv;
-        const float dA = s_dA[hl];
-        float s[EPV];
-        unpack16<ST>(v[i], s);
-        float acc = 0.f;
-#pragma unroll
-        for (int e = 0; e < EPV; ++e) {
-            s[e] = fmaf(s[e], dA, dtx * Bv[e]);
-            acc = fmaf(s[e], Cv[e], acc);
+#pragma unroll 1
+    for (int c = 0; c < CHUNKS && ok; ++c) {
+        if (!mbar_wait_bounded(&s_bar[c], 0, kWaitLimitNs)) {
+            record_error(a.error, M2_ERR_TIMEOUT);
+            ok = false;
+            break;
         }
-        st_stream(tile + static_cast<int64_t>(row) * N + e0, pack16<ST>(s));
+        const uint8_t* src = s_tile + c * CHUNK_BYTES;
+        float acc[VPT];
 #pragma unroll
-        for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if ((lane % LPR) == 0) s_y[row] = fmaf(s_D[hl], xv, acc);
+        for (int i = 0; i < VPT; ++i) {
+            const int v = i * kThreads + tid;          // vector index within the chunk
+            const int row = c * RC + v / LPR;          // row within the tile
+            const float4 rp = s_rp[row];
+            const float2 dtx2 = make_float2(rp.x, rp.x);
+            const float2 dA2 = make_float2(rp.y, rp.y);
+            float st[EPV];
+            unpack16<ST>(*reinterpret_cast<const uint4*>(src + static_cast<uint32_t>(v) * 16u), st);
+            float2 a2 = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int e = 0; e < EPV / 2; ++e) {
+                float2 s2 = make_float2(st[2 * e], st[2 * e + 1]);
+                s2 = __ffma2_rn(s2, dA2, __fmul2_rn(dtx2, B2[e]));  // S*dA + (dt*x)*B
+                a2 = __ffma2_rn(s2, C2[e], a2);                      // partial sum of S'*C
+                st[2 * e] = s2.x;
+                st[2 * e + 1] = s2.y;
+            }
+            st_stream(tile + static_cast<int64_t>(row) * N + e0, pack16<ST>(st));
+            acc[i] = a2.x + a2.y;
+        }
+        int which;
+        const float sum = reduce_rows<LPR, VPT>(acc, lane, which);
+        if ((lane % (LPR / VPT)) == 0) {
+            const int row = c * RC + which * RPP + tid / LPR;
+            s_y[row] = sum + s_rp[row].z;
+        }
+    }
+    if (!ok) {
+        // let this CTA's own copies land (bounded) before its shared memory is released
+        for (int c = 0; c <= CHUNKS; ++c) mbar_wait_bounded(&s_bar[c], 0, kWaitLimitNs);
     }
     __syncthreads();
 
     // ---- y (gated), contiguous over the tile's rows
-    for (int i = tid; i < TILE; i += kThreads) {
-        float yv = s_y[i];
-        if (zrow) yv *= silu_f32(to_f32(zrow[r0 + i]));
-        yrow[r0 + i] = from_f32<AT>(yv);
+    if (ok) {
+        for (int i = tid; i < TILE; i += kThreads) {
+            float yv = s_y[i];
+            if (zrow) yv *= silu_f32(to_f32(zrow[r0 + i]));
+            yrow[r0 + i] = from_f32<AT>(yv);
+        }
     }
 
     if constexpr (FUSED) {
-        // ---- phase 3: cluster rank 0 rolls the shared B/C conv rows
+        // ---- phase 3: cluster rank 0 rolls the shared B/C conv rows (from the
+        // staged copy of the old rows and the raw inputs)
         cluster_wait();
-        if (cluster_rank() == 0) {
-            AT* conv0 = static_cast<AT*>(a.conv) + static_cast<int64_t>(slot) * (a.K - 1) * cd;
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                const int j = tid + q * kThreads;
-                if (j < 2 * N) {
-                    const int64_t c = j < N ? cB + j : cC + (j - N);
-                    conv_roll(conv0, cd, a.K, c, bc_win[q]);
+        if (ok && cluster_rank() == 0) {
+            const AT* xrow = static_cast<const AT*>(a.xBC) + b * a.xBC_stride;
+            for (int v = tid; v < 2 * BV; v += kThreads) {
+                const int seg = v / BV;
+                const int j0 = (v % BV) * AV;
+                const int64_t c0 = (seg ? cC : cB) + j0;
+                const AT* rows = s_cbc + seg * N + j0;
+                for (int k = 0; k < K - 1; ++k) {
+                    const uint4 nv = (k < K - 2) ? *reinterpret_cast<const uint4*>(rows + (k + 1) * 2 * N)
+                                                 : *reinterpret_cast<const uint4*>(xrow + c0);
+                    *reinterpret_cast<uint4*>(conv0 + k * cd + c0) = nv;
                 }
             }
         }
     }
 }
 
-template <typename ST, typename AT, typename XT, int N, int LOADS, bool FUSED>
+template <typename ST, typename AT, typename XT, int N, int CHUNKS, int VPT, bool FUSED>
 cudaError_t launch_one(const StateUpdateArgs& a, const DecodePlan& plan, cudaStream_t stream) {
-    auto kern = state_update_kernel<ST, AT, XT, N, LOADS, FUSED>;
+    auto kern = state_update_kernel<ST, AT, XT, N, CHUNKS, VPT, FUSED>;
+    constexpr int LPR = N / Vec16<ST>::n;
+    constexpr int TILE = CHUNKS * (kThreads / LPR) * VPT;
+    size_t smem = static_cast<size_t>(TILE) * N * sizeof(ST);
+    if (FUSED) smem += static_cast<size_t>(a.K - 1) * (TILE + 2 * N) * sizeof(AT);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    if (FUSED && plan.cluster > 8) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(plan.ctas_per_seq, a.batch, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -251,19 +438,16 @@ cudaError_t launch_one(const StateUpdateArgs& a, const DecodePlan& plan, cudaStr
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (FUSED && plan.cluster > 8) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return e;
-    }
     return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 template <typename ST, typename AT, typename XT, int N, bool FUSED>
 cudaError_t by_loads(const StateUpdateArgs& a, const DecodePlan& p, cudaStream_t s) {
+    // loads = 16-byte vectors per thread per tile = CHUNKS * VPT
     switch (p.loads) {
-        case 16: return launch_one<ST, AT, XT, N, 16, FUSED>(a, p, s);
-        case 4: return launch_one<ST, AT, XT, N, 4, FUSED>(a, p, s);
-        case 1: return launch_one<ST, AT, XT, N, 1, FUSED>(a, p, s);
+        case 4 * M2_DECODE_MAIN_CHUNKS: return launch_one<ST, AT, XT, N, M2_DECODE_MAIN_CHUNKS, 4, FUSED>(a, p, s);
+        case 4: return launch_one<ST, AT, XT, N, 1, 4, FUSED>(a, p, s);
+        case 1: return launch_one<ST, AT, XT, N, 1, 1, FUSED>(a, p, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -298,7 +482,7 @@ m2_status plan_state_update(int H, int P, int N, int G, int state_bf16, int fuse
     const int lpr = N / epv;
     const int rpw = 32 / lpr;
     const int64_t group_rows = static_cast<int64_t>(H / G) * P;
-    static const int kLoads[3] = {16, 4, 1};
+    static const int kLoads[3] = {4 * M2_DECODE_MAIN_CHUNKS, 4, 1};
     for (int li = 0; li < 3; ++li) {
         const int tile = kWarps * rpw * kLoads[li];
         if (group_rows % tile != 0) continue;
