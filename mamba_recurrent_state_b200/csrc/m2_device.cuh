@@ -152,7 +152,11 @@ __device__ __forceinline__ float softplus_f32(float v) {
     return v > 20.f ? v : log1pf(expf(v));
 }
 
-// silu(v) = v / (1 + exp(-v)).
-__device__ __forceinline__ float silu_f32(float v) { return v / (1.f + expf(-v)); }
+// silu(v) = v / (1 + exp(-v)), with the hardware exponential and the fast
+// division (a few ulp for the |v| < 20 the activations take; the limits 0 and v
+// come out right: exp overflows to inf and the quotient to 0 for v -> -inf).
+// Every kernel uses this one definition, so fused and unfused paths agree
+// bit for bit.
+__device__ __forceinline__ float silu_f32(float v) { return __fdividef(v, 1.f + __expf(-v)); }
 
 }  // namespace m2

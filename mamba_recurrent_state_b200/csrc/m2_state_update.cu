@@ -30,8 +30,8 @@
 //    rolls their conv-cache rows, which no other CTA touches) and for the
 //    group's B and C channels, which every CTA of the group needs. Those CTAs
 //    form one thread-block cluster; each arrives on the cluster barrier after
-//    reading the B/C conv rows, and only cluster rank 0 writes the rolled B/C
-//    rows, after waiting on the barrier at the very end.
+//    reading the B/C conv rows, and only cluster rank 0 waits on it (at the
+//    very end) and then writes the rolled B/C rows.
 #include <cuda_runtime.h>
 
 #include "m2_device.cuh"
@@ -53,8 +53,11 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxHeadsPerTile = 33;
 
+// Relaxed arrive: the only cross-CTA hazard it orders is WAR on the group's
+// B/C conv rows, and those rows were read by bulk copies whose completion every
+// reading thread has already observed on its mbarrier before arriving.
 __device__ __forceinline__ void cluster_arrive() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;\n" ::: "memory");
 }
 __device__ __forceinline__ void cluster_wait() {
     asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
@@ -393,8 +396,10 @@ state_update_kernel(const StateUpdateArgs a) {
 
     if constexpr (FUSED) {
         // ---- phase 3: cluster rank 0 rolls the shared B/C conv rows (from the
-        // staged copy of the old rows and the raw inputs)
-        cluster_wait();
+        // staged copy of the old rows and the raw inputs). Only rank 0 writes
+        // after the barrier, so only rank 0 waits; the other CTAs have arrived
+        // and may exit (exited threads never hold up a cluster wait).
+        if (cluster_rank() == 0) cluster_wait();
         if (ok && cluster_rank() == 0) {
             const AT* xrow = static_cast<const AT*>(a.xBC) + b * a.xBC_stride;
             for (int v = tid; v < 2 * BV; v += kThreads) {
