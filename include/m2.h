@@ -72,7 +72,9 @@ typedef enum m2_status {
     M2_ERR_CUDA = -3,        /* a CUDA runtime call or a launch failed */
     M2_ERR_OOM = -4,         /* device allocation failed (m2_cache_alloc only) */
     M2_ERR_BAD_SLOT = -5,    /* device: a slot index >= num_slots was seen */
-    M2_ERR_TIMEOUT = -6      /* device: a bounded wait inside a kernel ran out */
+    M2_ERR_TIMEOUT = -6,     /* device: a bounded wait inside a kernel ran out */
+    M2_ERR_RANGE = -7        /* device: a value exceeded the fp16 range of the tensor-core
+                                scan's operands (|v| >= 65520); that row's results are not valid */
 } m2_status;
 
 /* Mixer shape (Nemotron-H-8B: H=128, P=64, N=128, G=8, K=4). */
@@ -197,6 +199,12 @@ m2_status m2_state_update(const m2_cache* cache, const m2_ssm_params* ssm,
  *   z        [batch, seqlen, H*P] act_dtype or NULL, row stride z_row_stride
  *   y        [batch, seqlen, H*P] act_dtype, row stride y_row_stride
  *   chunk_size  tokens per chunk (the last chunk may be partial)
+ * With bf16 state and activations at P = 64, N = 128 the scan runs on the
+ * tensor cores in chunks of 128 tokens, with fp16 MMA operands (inputs converted
+ * exactly, derived operands rounded once, fp32 accumulation); any operand that
+ * leaves the fp16 range sets M2_ERR_RANGE in the error word. The result does
+ * not depend on chunk_size, which must be positive (the kernels choose their own
+ * tiling). Other dtypes and shapes run token by token on the CUDA cores.
  * No allocation, no scratch memory.
  */
 m2_status m2_chunk_scan(const m2_cache* cache, const m2_ssm_params* ssm, int32_t batch,

@@ -41,6 +41,7 @@ STATUS = {
     -4: "out of device memory",
     -5: "slot index out of range",
     -6: "bounded wait timed out",
+    -7: "operand outside the fp16 range of the tensor-core scan",
 }
 M2_OK = 0
 M2_ERR_INVALID_ARG = -1
@@ -49,6 +50,7 @@ M2_ERR_CUDA = -3
 M2_ERR_OOM = -4
 M2_ERR_BAD_SLOT = -5
 M2_ERR_TIMEOUT = -6
+M2_ERR_RANGE = -7
 
 
 class M2Error(RuntimeError):

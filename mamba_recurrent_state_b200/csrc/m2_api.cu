@@ -367,6 +367,7 @@ const char* m2_status_string(m2_status s) {
         case M2_ERR_OOM: return "out of device memory";
         case M2_ERR_BAD_SLOT: return "slot index out of range";
         case M2_ERR_TIMEOUT: return "bounded wait timed out";
+        case M2_ERR_RANGE: return "operand outside the fp16 range of the tensor-core scan";
     }
     return "unknown status";
 }

@@ -8,7 +8,9 @@
 //   S <- S*exp(dt_t*A) + (dt_t*x_t) B_t^T,   y_t = S C_t + D x_t,  y_t *= silu(z_t)
 // from the slot's state (or zero), with the final S stored back once.
 //
-// This file holds the token-sequential kernel on the CUDA cores: one CTA per
+// bf16 state and activations at P = 64, N = 128 go to the tensor-core kernel
+// (m2_chunk_scan_tc.cu). This file holds the token-sequential kernel on the
+// CUDA cores used for the other dtypes and shapes: one CTA per
 // (sequence, head), the head's P x N state in registers (TPR threads per state
 // row), inputs staged through shared memory a tile of tokens at a time. It
 // allocates nothing and keeps the state on chip for the whole sequence.
@@ -162,6 +164,7 @@ m2_status plan_chunk_scan(int H, int P, int N, int G, int state_bf16, int act_bf
 
 cudaError_t launch_chunk_scan(const ScanArgs& a, cudaStream_t s) {
     if (a.batch == 0 || a.seqlen == 0) return cudaSuccess;
+    if (chunk_scan_tc_supported(a)) return launch_chunk_scan_tc(a, s);
     if (a.state_bf16) return a.act_bf16 ? scan_by_x<bf16_t, bf16_t>(a, s) : scan_by_x<bf16_t, float>(a, s);
     return a.act_bf16 ? scan_by_x<float, bf16_t>(a, s) : scan_by_x<float, float>(a, s);
 }

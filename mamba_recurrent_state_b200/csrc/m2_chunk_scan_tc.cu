@@ -1,0 +1,517 @@
+// m2_chunk_scan_tc.cu -- chunked prefill scan on the 5th-generation tensor
+// cores (tcgen05 + TMEM, operands staged by TMA), bf16 state and activations.
+//
+// Operation: vllm.cpp issue #1311 "NemotronH runs the PREFILL mamba kernels at
+// decode", section "The divergence" (the chunk scan that follows the prefill
+// conv) and section "Confirm or refute" (it must land on the state of the
+// sequential updates). The Mamba-2 recurrence over a chunk of Q = 128 tokens
+// t = 0..Q-1 of one head, with c_t = sum_{r<=t} dt_r * A (A = -exp(A_log)),
+// written in its chunked (state-space dual) form:
+//   Y      = (C B^T o L o dt_u) X + diag(exp(c_t)) C S^T + D x      (y before the gate)
+//   S_next = exp(c_end) S + X^T (w o B),   w_u = exp(c_end - c_u) dt_u
+// with L[t,u] = exp(c_t - c_u) for u <= t, else 0. The four products run as
+// tcgen05 MMAs (M = 128, fp16 operands, fp32 accumulators in TMEM):
+//   MMA1  CB     [t,u] = C . B^T        A = C (K-major), B = B (K-major)
+//   MMA3  Yoff   [t,p] = C . S^T        A = C (K-major), B = S (K-major, bf16 copy)
+//   MMA2  Ydiag  [t,p] = M . X          A = M = CB o L o dt (K-major), B = X (MN-major)
+//   MMA4  dS^T   [n,p] = W^T . X        A = W = w o B (MN-major), B = X (MN-major)
+// The state itself is carried exactly in fp32 registers (thread n holds column
+// n of S) and rounded once when the sequence ends. Only the chunk-to-chunk carry
+// is sequential.
+//
+// Operand precision. The intra-chunk terms dt_u (C_t . B_u) x_u are often an
+// order of magnitude larger than y itself, so rounding M, W and the state copy
+// to bf16 (8-bit significand) leaves absolute errors of a few percent of
+// rms(y). The MMAs therefore take fp16 operands (11-bit significand, the same
+// A/B type in every MMA): the bf16 inputs C, B, X are converted exactly in
+// shared memory after each load, and M, W, S are rounded once to fp16. Any value
+// outside the fp16 range (|v| >= 65520) records M2_ERR_RANGE.
+//
+// One CTA of 256 threads per (sequence, head). Thread t owns TMEM lane
+// r = t % 128 (row r of every accumulator; warps w and w+4 share a lane quarter)
+// and the column half h2 = t / 128 of that row. Shared memory (1024-byte
+// aligned, 128-byte swizzle):
+//   C tile  32 KB [2 atoms of 64 n][128 t][128 B]   later overwritten by M
+//   B tile  32 KB [2 atoms of 64 n][128 u][128 B]   later scaled in place to W
+//   X tile  16 KB [128 u][64 p]
+//   S copy  16 KB [2 atoms of 64 n][64 p][128 B]    fp16 state for MMA3
+// TMEM (256 columns): CB at 0..127 (then dS^T at 0..63), Yoff at 128..191,
+// Ydiag at 192..255. Tokens past the sequence end arrive as zeros from TMA and
+// get dt = 0, so they neither decay nor feed the state.
+//
+// Every wait is bounded (one second of %globaltimer); the CTA takes the
+// timeout decision together (__syncthreads_and), records M2_ERR_TIMEOUT, waits
+// once more for its own copies and MMAs, frees its TMEM and returns.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "m2_device.cuh"
+#include "m2_internal.cuh"
+
+namespace m2 {
+namespace {
+
+constexpr int kQ = 128;   // tokens per chunk = MMA M
+constexpr int kP = 64;    // head dim
+constexpr int kN = 128;   // state dim
+constexpr int kTC = 256;  // threads per CTA: two threads per TMEM lane (row)
+constexpr uint32_t kOffC = 0, kOffB = 32768, kOffX = 65536, kOffS = 81920, kSmemUsed = 98304;
+constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // + alignment slack
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColCB = 0, kColDS = 0, kColYoff = 128, kColYdiag = 192;
+constexpr uint64_t kLimitNs = 1000000000ull;
+
+// ---- tcgen05 / TMA helpers -----------------------------------------------
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm100 version field.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1) << 46;  // descriptor version (sm100)
+    d |= static_cast<uint64_t>(2) << 61;  // SWIZZLE_128B
+    return d;
+}
+
+// Instruction descriptor, kind::f16: fp16 A and B (format 0), fp32 D, dense.
+constexpr uint32_t idesc_f16(int M, int N, bool a_mn_major, bool b_mn_major) {
+    return (1u << 4) | ((a_mn_major ? 1u : 0u) << 15) |
+           ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+           (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrives on `bar` once every MMA this thread issued so far has completed.
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
+                     smem_addr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane. The wait for the
+// load sits in the same asm statement, so no use of the registers can be
+// scheduled before the data has arrived.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+        "tcgen05.wait::ld.sync.aligned;\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+          "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+          "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Generic-proxy shared-memory writes become visible to the async proxy
+// (tensor cores, TMA).
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];\n" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
+// Byte offset of 16-byte chunk j of row r in a 128-byte-swizzled tile.
+__device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t j) { return r * 128u + ((j ^ (r & 7u)) << 4); }
+
+constexpr float kF16Limit = 65520.f;  // smallest magnitude that rounds to fp16 infinity
+
+// Converts a 16-byte chunk of 8 bf16 values in shared memory to fp16 in place;
+// returns the largest magnitude seen.
+__device__ __forceinline__ float bf16_chunk_to_f16(uint8_t* p) {
+    float v[8];
+    unpack16<bf16_t>(*reinterpret_cast<const uint4*>(p), v);
+    float mx = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(v[e]));
+    *reinterpret_cast<uint4*>(p) = pack16_f16(v);
+    return mx;
+}
+
+template <typename ST>
+__global__ void __launch_bounds__(kTC, 2)
+chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs a) {
+    extern __shared__ uint8_t s_raw[];
+    __shared__ __align__(8) uint64_t s_bar_ld;
+    __shared__ __align__(8) uint64_t s_bar_mma;
+    __shared__ uint32_t s_tmem;
+    __shared__ float s_cum[kQ];
+    __shared__ float s_dt[kQ];
+    __shared__ float s_wsum[kQ / 32];
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int r = tid & (kQ - 1);   // TMEM lane / tile row of this thread
+    const int h2 = tid >> 7;        // column half of this thread
+    const int h = blockIdx.x;
+    const int b = blockIdx.y;
+    const int H = a.H;
+    const int G = a.G;
+    const int g = h / (H / G);
+    const int T = a.seqlen;
+    const int64_t HP = static_cast<int64_t>(H) * kP;
+    const int32_t slot = a.slot_idx[b];
+    bf16_t* y = static_cast<bf16_t*>(a.y);
+    const int64_t row0 = static_cast<int64_t>(b) * T;
+
+    if (slot < 0) {  // padding row: y = 0, cache untouched
+        for (int64_t i = tid; i < static_cast<int64_t>(T) * (kP / 8); i += kTC) {
+            const int64_t t = i / (kP / 8);
+            *reinterpret_cast<uint4*>(y + (row0 + t) * a.y_stride + h * kP + (i % (kP / 8)) * 8) =
+                make_uint4(0, 0, 0, 0);
+        }
+        return;
+    }
+    if (slot >= a.num_slots) {
+        if (tid == 0) record_error(a.error, M2_ERR_BAD_SLOT);
+        return;
+    }
+
+    // 1024-byte aligned base for the swizzled tiles
+    const uint32_t raw_addr = smem_addr(s_raw);
+    const uint32_t base = (raw_addr + 1023u) & ~1023u;
+    uint8_t* sm = s_raw + (base - raw_addr);
+
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
+                         smem_addr(&s_tmem)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+    }
+    if (tid == 0) {
+        mbar_init(&s_bar_ld, 1);
+        mbar_init(&s_bar_mma, 1);
+        fence_mbar_init();
+        asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;  // this warp's TMEM lanes
+
+    const float A = -expf(a.A_log[h]);
+    const float dt_bias = a.dt_bias[h];
+    const float Dh = a.D[h];
+    const int xcol = h * kP;
+    const int bcol = static_cast<int>(HP) + g * kN;
+    const int ccol = static_cast<int>(HP) + G * kN + g * kN;
+
+    // running state: thread (n = r, h2) holds S[p][n] for p = 32*h2 .. 32*h2+31 (fp32)
+    constexpr int kPH = kP / 2;
+    const int n = r;
+    const int p0 = h2 * kPH;
+    ST* state = static_cast<ST*>(a.ssm) + (static_cast<int64_t>(slot) * HP + static_cast<int64_t>(h) * kP) * kN;
+    float S[kPH];
+    float range_max = 0.f;  // largest magnitude handed to an fp16 operand
+    const bool init = a.has_init != nullptr && a.has_init[b] != 0;
+#pragma unroll
+    for (int i = 0; i < kPH; ++i) S[i] = init ? to_f32(state[(p0 + i) * kN + n]) : 0.f;
+    // fp16 copy for MMA3: element (p, n) of the K-major [2 atoms][64 p][64 n] tile
+    auto write_state_copy = [&]() {
+        uint8_t* sS = sm + kOffS + (n >> 6) * 8192;
+        const uint32_t j = (n & 63) >> 3;
+#pragma unroll
+        for (int i = 0; i < kPH; ++i) {
+            *reinterpret_cast<__half*>(sS + sw128(p0 + i, j) + (n & 7) * 2) = __float2half_rn(S[i]);
+            range_max = fmaxf(range_max, fabsf(S[i]));
+        }
+    };
+    write_state_copy();
+
+    const int nchunks = (T + kQ - 1) / kQ;
+    const uint32_t id_cb = idesc_f16(128, 128, false, false);
+    const uint32_t id_yoff = idesc_f16(128, 64, false, false);
+    const uint32_t id_ydiag = idesc_f16(128, 64, false, true);
+    const uint32_t id_ds = idesc_f16(128, 64, true, true);
+    auto issue_loads = [&](int c) {
+        const int t0 = c * kQ;
+        mbar_arrive_expect_tx(&s_bar_ld, 5u * 16384u);
+        tma_load_3d(base + kOffX, &tmap_x, xcol, t0, b, &s_bar_ld);
+        tma_load_3d(base + kOffB, &tmap_x, bcol, t0, b, &s_bar_ld);
+        tma_load_3d(base + kOffB + 16384, &tmap_x, bcol + 64, t0, b, &s_bar_ld);
+        tma_load_3d(base + kOffC, &tmap_x, ccol, t0, b, &s_bar_ld);
+        tma_load_3d(base + kOffC + 16384, &tmap_x, ccol + 64, t0, b, &s_bar_ld);
+    };
+    if (tid == 0) issue_loads(0);
+
+    bool ok = true;
+    int loads_issued = 1, loads_done = 0, mma_issued = 0, mma_done = 0;
+    for (int c = 0; c < nchunks; ++c) {
+        const int t0 = c * kQ;
+        const int valid = min(kQ, T - t0);
+
+        // ---- dt and the cumulative decay c_t for the chunk (threads 0..127: token t)
+        const int t = r;
+        {
+            float dt = 0.f;
+            if (h2 == 0 && t < valid) {
+                const float raw = to_f32(static_cast<const bf16_t*>(a.dt)[(row0 + t0 + t) * a.dt_stride + h]);
+                dt = softplus_f32(raw + dt_bias);
+            }
+            float cum = dt * A;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float o = __shfl_up_sync(0xffffffffu, cum, off);
+                if (lane >= off) cum += o;
+            }
+            if (h2 == 0 && lane == 31) s_wsum[warp] = cum;
+            __syncthreads();
+            if (h2 == 0) {
+                for (int w = 0; w < warp; ++w) cum += s_wsum[w];
+                s_cum[t] = cum;
+                s_dt[t] = dt;
+            }
+        }
+
+        // ---- wait for X, B, C; MMA1 (CB) and MMA3 (Yoff)
+        bool got = mbar_wait_bounded(&s_bar_ld, loads_done & 1, kLimitNs);
+        if (!__syncthreads_and(got)) { ok = false; break; }
+        ++loads_done;
+        // bf16 -> fp16 in place (exact within range): row t of C and B (atom h2)
+        // and half of row t of X
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            range_max = fmaxf(range_max, bf16_chunk_to_f16(sm + kOffC + h2 * 16384 + t * 128 + j * 16));
+            range_max = fmaxf(range_max, bf16_chunk_to_f16(sm + kOffB + h2 * 16384 + t * 128 + j * 16));
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            range_max = fmaxf(range_max, bf16_chunk_to_f16(sm + kOffX + t * 128 + (4 * h2 + j) * 16));
+        fence_proxy_async();
+        __syncthreads();
+        const float cum_end = s_cum[kQ - 1];
+        if (tid == 0) {
+            tc_fence_after();
+            for (int k = 0; k < kN / 16; ++k) {
+                const uint32_t koff = (k >> 2) * 16384u + (k & 3) * 32u;
+                mma_f16(tmem + kColCB, sw128_desc(base + kOffC + koff, 16, 1024),
+                         sw128_desc(base + kOffB + koff, 16, 1024), id_cb, k > 0);
+            }
+            for (int k = 0; k < kN / 16; ++k) {
+                const uint32_t koff = (k >> 2) * 16384u + (k & 3) * 32u;
+                const uint32_t soff = (k >> 2) * 8192u + (k & 3) * 32u;
+                mma_f16(tmem + kColYoff, sw128_desc(base + kOffC + koff, 16, 1024),
+                         sw128_desc(base + kOffS + soff, 16, 1024), id_yoff, k > 0);
+            }
+            mma_commit(&s_bar_mma);
+        }
+        ++mma_issued;
+        got = mbar_wait_bounded(&s_bar_mma, mma_done & 1, kLimitNs);
+        if (!__syncthreads_and(got)) { ok = false; break; }
+        ++mma_done;
+        tc_fence_after();
+
+        // ---- epilogue 1: M = CB o L o dt (row t, bf16, into the C tile) and
+        // W = w o B (row u = t of the B tile, scaled in place)
+        {
+            const float cum_t = s_cum[t];
+#pragma unroll 1
+            for (int q = 2 * h2; q < 2 * h2 + 2; ++q) {  // columns u = 64*h2 .. 64*h2+63
+                float cb[32];
+                tmem_ld32(tmem + lane_base + kColCB + q * 32, cb);
+                float m[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int u = q * 32 + i;
+                    m[i] = (u <= t) ? cb[i] * __expf(cum_t - s_cum[u]) * s_dt[u] : 0.f;
+                    range_max = fmaxf(range_max, fabsf(m[i]));
+                }
+                // 32 columns = 4 chunks of 8 in atom (q >> 1), chunks 4*(q&1) ..
+                uint8_t* dst = sm + kOffC + (q >> 1) * 16384;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const uint32_t j = (q & 1) * 4 + jj;
+                    *reinterpret_cast<uint4*>(dst + sw128(t, j)) = pack16_f16(m + 8 * jj);
+                }
+            }
+            const float wu = (t < valid) ? __expf(cum_end - cum_t) * s_dt[t] : 0.f;
+            {
+                const int atom = h2;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    uint4* p = reinterpret_cast<uint4*>(sm + kOffB + atom * 16384 + t * 128 + j * 16);
+                    float v[8];
+                    unpack16_f16(*p, v);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        v[e] *= wu;
+                        range_max = fmaxf(range_max, fabsf(v[e]));
+                    }
+                    *p = pack16_f16(v);
+                }
+            }
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+
+        // ---- MMA2 (Ydiag = M X) and MMA4 (dS^T = W^T X)
+        if (tid == 0) {
+            tc_fence_after();
+            for (int k = 0; k < kQ / 16; ++k) {
+                const uint32_t koff = (k >> 2) * 16384u + (k & 3) * 32u;
+                mma_f16(tmem + kColYdiag, sw128_desc(base + kOffC + koff, 16, 1024),
+                         sw128_desc(base + kOffX + k * 2048u, 16384, 1024), id_ydiag, k > 0);
+            }
+            for (int k = 0; k < kQ / 16; ++k) {
+                mma_f16(tmem + kColDS, sw128_desc(base + kOffB + k * 2048u, 16384, 1024),
+                         sw128_desc(base + kOffX + k * 2048u, 16384, 1024), id_ds, k > 0);
+            }
+            mma_commit(&s_bar_mma);
+        }
+        ++mma_issued;
+        got = mbar_wait_bounded(&s_bar_mma, mma_done & 1, kLimitNs);
+        if (!__syncthreads_and(got)) { ok = false; break; }
+        ++mma_done;
+        tc_fence_after();
+
+        // ---- epilogue 2: y row t, then the state carry (thread n = t)
+        {
+            const float et = __expf(s_cum[t]);
+            const bool row_ok = t < valid;
+            const bf16_t* zrow = a.z ? static_cast<const bf16_t*>(a.z) + (row0 + t0 + t) * a.z_stride + xcol : nullptr;
+            bf16_t* yrow = y + (row0 + t0 + t) * a.y_stride + xcol;
+            {
+                const int q = h2;  // columns p = 32*h2 .. 32*h2+31
+                float yd[32], yo[32];
+                tmem_ld32(tmem + lane_base + kColYdiag + q * 32, yd);
+                tmem_ld32(tmem + lane_base + kColYoff + q * 32, yo);
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const uint32_t j = q * 4 + jj;  // chunk of 8 p values
+                    float xv[8], out[8];
+                    unpack16_f16(*reinterpret_cast<const uint4*>(sm + kOffX + sw128(t, j)), xv);
+                    float zv[8];
+                    if (zrow && row_ok) unpack16<bf16_t>(*reinterpret_cast<const uint4*>(zrow + 8 * j), zv);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        float v = fmaf(et, yo[8 * jj + e], yd[8 * jj + e]);
+                        v = fmaf(Dh, xv[e], v);
+                        if (zrow) v *= silu_f32(zv[e]);
+                        out[e] = v;
+                    }
+                    if (row_ok) *reinterpret_cast<uint4*>(yrow + 8 * j) = pack16<bf16_t>(out);
+                }
+            }
+            const float eend = __expf(cum_end);
+            {
+                float ds[32];
+                tmem_ld32(tmem + lane_base + kColDS + p0, ds);
+#pragma unroll
+                for (int i = 0; i < kPH; ++i) S[i] = fmaf(eend, S[i], ds[i]);
+            }
+            write_state_copy();
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0 && c + 1 < nchunks) {
+            issue_loads(c + 1);
+            ++loads_issued;
+        }
+    }
+    if (ok) {
+#pragma unroll
+        for (int i = 0; i < kPH; ++i) state[(p0 + i) * kN + n] = from_f32<ST>(S[i]);
+        if (range_max >= kF16Limit) record_error(a.error, M2_ERR_RANGE);
+    } else {
+        if (tid == 0) record_error(a.error, M2_ERR_TIMEOUT);
+        // let this CTA's own copies and MMAs finish (bounded) before freeing
+        if (loads_done < loads_issued) mbar_wait_bounded(&s_bar_ld, loads_done & 1, kLimitNs);
+        if (mma_done < mma_issued) mbar_wait_bounded(&s_bar_mma, mma_done & 1, kLimitNs);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn encode_fn() {
+    static std::once_flag once;
+    static EncodeFn fn = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeFn>(p);
+        cudaGetLastError();
+    });
+    return fn;
+}
+
+}  // namespace
+
+bool chunk_scan_tc_supported(const ScanArgs& a) {
+    return a.P == kP && a.N == kN && a.state_bf16 && a.act_bf16 && a.x_bf16 && (a.xBC_stride * 2) % 16 == 0;
+}
+
+cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t stream) {
+    EncodeFn enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    // xBC as a 3-D tensor (channel, token, sequence), 64 x 128 x 1 boxes of bf16,
+    // 128-byte swizzle; out-of-range tokens read as zeros
+    CUtensorMap map;
+    const int64_t cd = static_cast<int64_t>(a.H) * a.P + 2LL * a.G * a.N;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(cd), static_cast<cuuint64_t>(a.seqlen),
+                                static_cast<cuuint64_t>(a.batch)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(a.xBC_stride) * 2,
+                                   static_cast<cuuint64_t>(a.xBC_stride) * 2 * a.seqlen};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kQ), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a.xBC), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    auto kern = chunk_scan_tc_kernel<bf16_t>;
+    static const cudaError_t attr_err =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
+    if (attr_err != cudaSuccess) return attr_err;
+    const dim3 grid(static_cast<unsigned>(a.H), static_cast<unsigned>(a.batch));
+    kern<<<grid, kTC, kSmemBytes, stream>>>(map, a);
+    return cudaGetLastError();
+}
+
+}  // namespace m2

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace m2 {
@@ -76,6 +77,29 @@ template <>
 __device__ __forceinline__ uint4 pack16<bf16_t>(const float* in) {
     return make_uint4(pack_bf16x2(in[0], in[1]), pack_bf16x2(in[2], in[3]),
                       pack_bf16x2(in[4], in[5]), pack_bf16x2(in[6], in[7]));
+}
+
+// fp16 (IEEE binary16) carried as its raw 16-bit pattern.
+using f16_t = uint16_t;
+
+// Eight fp16 values <-> one 16-byte vector (round to nearest even).
+__device__ __forceinline__ void unpack16_f16(const uint4& v, float* out) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+        out[2 * i] = f.x;
+        out[2 * i + 1] = f.y;
+    }
+}
+__device__ __forceinline__ uint4 pack16_f16(const float* in) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __half2 h = __floats2half2_rn(in[2 * i], in[2 * i + 1]);
+        w[i] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 // Streaming 16-byte global load / store (data touched once per call).

@@ -106,6 +106,9 @@ cudaError_t launch_zero_slots(const ZeroArgs& a, cudaStream_t stream);
 m2_status plan_chunk_scan(int H, int P, int N, int G, int state_bf16, int act_bf16, int x_bf16,
                           int chunk);
 cudaError_t launch_chunk_scan(const ScanArgs& a, cudaStream_t stream);
+// Tensor-core (tcgen05) scan: bf16 state, activations and xBC, P = 64, N = 128.
+bool chunk_scan_tc_supported(const ScanArgs& a);
+cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t stream);
 
 // Records `code` in the error word unless an earlier error is already there.
 __device__ __forceinline__ void record_error(int32_t* error, int32_t code) {

@@ -99,8 +99,9 @@ def test_scan_fp32_xbc_input():
 @pytest.mark.parametrize("G", [1, 8])
 def test_scan_T1_equals_state_update(G):
     """A one-token scan from the cached state equals one decode step on the
-    same post-conv input (including n_groups = 8): the state bit for bit (same
-    fp32 arithmetic per element), y within tolerance."""
+    same post-conv input (including n_groups = 8), state and y within the bf16
+    tolerance (the scan's tensor-core path forms its state increment from bf16
+    MMA operands, the decode step element by element in fp32)."""
     w = W.Workload(310 + G, "t1", 128, 64, 128, G, 4, S.BF16, S.BF16, 16, 8, seqlen=1)
     a = make_cache(w)
     b = m2.Cache(shape_of(w), w.num_slots, ssm=a.ssm.clone(), conv=a.conv.clone())
@@ -110,7 +111,11 @@ def test_scan_T1_equals_state_update(G):
     y_scan = m2.chunk_scan(a, ssm, x, dt, t["slots"], z=z, chunk_size=128, has_initial_state=ones)
     y_dec = m2.state_update(b, ssm, x[:, 0], dt[:, 0], t["slots"], z=z[:, 0])
     torch.cuda.synchronize()
-    assert torch.equal(a.ssm, b.ssm)
+    rows = t["slots"].long()
+    es = rel_err(f64(TI.to_storage_np(a.ssm[rows]), S.BF16), f64(TI.to_storage_np(b.ssm[rows]), S.BF16))
+    assert es <= TOL[S.BF16], es
+    others = [q for q in range(w.num_slots) if q not in rows.tolist()]
+    assert torch.equal(a.ssm[others], b.ssm[others])
     e = rel_err(f64(TI.to_storage_np(y_scan[:, 0]), S.BF16), f64(TI.to_storage_np(y_dec), S.BF16))
     assert e <= TOL[S.BF16], e
 
@@ -118,7 +123,15 @@ def test_scan_T1_equals_state_update(G):
 def test_workload4_prefill_then_decode():
     """Zero initial state; prefill conv over 2048 tokens (bf16 post-conv buffer),
     chunk scan, then 32 fused decode steps continuing from the scanned state.
-    Every y and the final states of all 8 sequences are checked."""
+    Every y and the states of all 8 sequences are checked.
+
+    Each kernel is held to the oracle on its own inputs: the prefill against the
+    oracle's 2048 sequential updates from zero, and the decode steps against the
+    oracle continuing from the state the prefill stored (bf16, exact) and the
+    conv cache it left (checked bit for bit). Chaining the two would compare a
+    trajectory that rounds the state to bf16 at every decode step from a start
+    that may differ by one ulp; such differences random-walk under per-step
+    rounding, so the chained figure is printed, not asserted."""
     w = W.WORKLOADS[4]
     cache = make_cache(w)
     t, ssm, conv = layer_objs(w)
@@ -155,24 +168,50 @@ def test_workload4_prefill_then_decode():
         y = ol.orc.ssm_scan(state, O.ROUND_BF16, xpost, dt, ol.dt_bias, ol.A_log, ol.D, z, w.G)
         errs = {"prefill_y": rel_err(f64(y_pre_np[b], w.act_dtype), y),
                 "prefill_state": rel_err(f64(state_after_prefill[b], w.state_dtype), state)}
+        # decode continued from the stored prefill state (the GPU's bf16 bits)
+        dstate = np.ascontiguousarray(f64(state_after_prefill[b], w.state_dtype))
+        chained = state
+        dconv = conv_state.copy()
         dec = []
         for step in range(1, w.decode_after + 1):
             inp = ol.inputs(step, [b])
-            yd = O.decode_rows(ol.orc, w.H, w.P, w.N, w.G, O.ROUND_BF16, [state], [conv_state],
+            yd = O.decode_rows(ol.orc, w.H, w.P, w.N, w.G, O.ROUND_BF16, [dstate], [dconv],
                                inp["xBC"], inp["dt"], inp["z"], ol.conv_w, ol.conv_b, ol.dt_bias,
                                ol.A_log, ol.D, threads=1)
+            O.decode_rows(ol.orc, w.H, w.P, w.N, w.G, O.ROUND_BF16, [chained], [conv_state],
+                          inp["xBC"], inp["dt"], inp["z"], ol.conv_w, ol.conv_b, ol.dt_bias,
+                          ol.A_log, ol.D, threads=1)
             dec.append(rel_err(f64(y_dec_np[step - 1][b], w.act_dtype), yd))
         errs["decode_y"] = max(dec)
-        errs["final_state"] = rel_err(f64(ssm_np[s], w.state_dtype), state)
+        errs["final_state"] = rel_err(f64(ssm_np[s], w.state_dtype), dstate)
+        errs["chained_final_state"] = rel_err(f64(ssm_np[s], w.state_dtype), chained)
         errs["conv_exact"] = bool(np.array_equal(conv_np[s], S.to_storage(conv_state, w.act_dtype)))
         return errs
 
     with ThreadPoolExecutor(max_workers=8) as ex:
         results = list(ex.map(one, range(w.batch)))
+    print("workload 4 errors per sequence:", results)
     for b, e in enumerate(results):
         assert e["prefill_y"] <= TOL[S.BF16], (b, e)
         assert e["prefill_state"] <= TOL[S.BF16], (b, e)
         assert e["decode_y"] <= TOL[S.BF16], (b, e)
         assert e["final_state"] <= TOL[S.BF16], (b, e)
         assert e["conv_exact"], (b, e)
+    assert cache.device_error() == 0
+
+
+def test_scan_operand_range_error_is_reported():
+    """A value beyond the fp16 range of the tensor-core scan's operands sets
+    M2_ERR_RANGE in the error word (the launch itself completes normally)."""
+    w = wl(320, H=8, G=2, T=64, batch=1, slots=2)
+    cache = make_cache(w)
+    t, ssm, _ = layer_objs(w)
+    x, dt, z = prefill_inputs(w)
+    x = x.clone()
+    x[0, 5, 3] = 1.0e5  # an x channel of head 0
+    slots = torch.tensor([1], dtype=torch.int32, device="cuda")
+    m2.chunk_scan(cache, ssm, x, dt, slots, z=z)
+    assert cache.device_error() == m2.M2_ERR_RANGE
+    x[0, 5, 3] = 1.0
+    m2.chunk_scan(cache, ssm, x, dt, slots, z=z)
     assert cache.device_error() == 0
