@@ -52,6 +52,9 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="budget of the oracle CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sections", default="decode,prefill,stack48",
+                    help="comma list: decode (the headline, always run), prefill (workload 4: "
+                         "prefill conv and tensor-core scan), stack48 (workload 2: 48-layer token)")
     return ap.parse_args()
 
 
@@ -63,13 +66,24 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def measured_peaks() -> tuple[float, str]:
+def _peak(key: str, fallback: float) -> tuple[float, str]:
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
-            return float(json.load(f)["hbm_gbs"]), "measured"
+            return float(json.load(f)[key]), "measured"
     except (OSError, KeyError, ValueError):
-        return 6650.0, "fallback"
+        return fallback, "fallback"
+
+
+def measured_peaks() -> tuple[float, str]:
+    """HBM copy bandwidth, GB/s (measured on this machine, else the fallback)."""
+    return _peak("hbm_gbs", 6650.0)
+
+
+def measured_tensor_peak() -> tuple[float, str]:
+    """Dense 16-bit tensor throughput, TFLOP/s (the cuBLAS bf16 burst figure;
+    fp16 and bf16 share the nominal dense rate)."""
+    return _peak("bf16_tflops", 1590.0)
 
 
 def profiled_traffic() -> float | None:
@@ -253,6 +267,122 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def _time_us(fn, flush, reps: int) -> list[float]:
+    """Device time of fn() per rep (CUDA events on the current stream), L2
+    flushed before every rep, outside the events."""
+    import torch
+    stream = torch.cuda.current_stream()
+    out = []
+    for _ in range(reps):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        b.synchronize()
+        out.append(1e3 * a.elapsed_time(b))
+    return out
+
+
+def measure_prefill(flush, peak_gbs: float, peak_tflops: float, reps: int = 10) -> dict:
+    """Workload 4's prefill: conv over 8 x 2048 tokens, then the tensor-core
+    chunk scan (fp16 operands, fp32 accumulate, 128-token chunks)."""
+    import torch
+    import mamba_recurrent_state_b200 as m2
+    from m2synth import torch_inputs as TI
+    from m2synth import workloads as W
+    w = W.WORKLOADS[4]
+    shape = m2.Shape(w.H, w.P, w.N, w.G, w.K, w.state_dtype, w.act_dtype)
+    cache = m2.Cache(shape, w.num_slots)
+    t = TI.layer_tensors(w)
+    ssm = m2.SSMParams(t["A_log"], t["dt_bias"], t["D"])
+    conv = m2.ConvParams(t["conv_w"], t["conv_b"], 1)
+    T = w.seqlen
+    d = TI.step_tensors(w, 0, rows=w.batch * T)
+    xr = d["xBC"].view(w.batch, T, -1)
+    dt = d["dt"].view(w.batch, T, -1)
+    z = d["z"].view(w.batch, T, -1)
+    xp = torch.empty_like(xr)
+    y = torch.empty((w.batch, T, w.H * w.P), dtype=torch.bfloat16, device="cuda")
+
+    def conv_step():
+        m2.conv1d_update(cache, conv, xr, t["slots"], out=xp)
+
+    def scan_step():
+        m2.chunk_scan(cache, ssm, xp, dt, t["slots"], z=z, chunk_size=w.chunk, y=y)
+
+    for _ in range(3):
+        conv_step()
+        scan_step()
+    conv_us = statistics.median(_time_us(conv_step, flush, reps))
+    scan_us = statistics.median(_time_us(scan_step, flush, reps))
+    if cache.device_error() != 0:
+        raise RuntimeError("device error word set during the prefill benchmark")
+    tokens = w.batch * T
+    hp, cd = w.H * w.P, w.conv_dim
+    # scan algorithmic bytes: post-conv xBC, dt, z in; y out; final state out
+    scan_bytes = tokens * (cd + w.H + hp + hp) * 2 + w.batch * w.H * w.P * w.N * 2
+    conv_bytes = tokens * cd * 2 * 2 + w.batch * (w.K - 1) * cd * 2 * 2
+    # SSD form with C.B^T shared by the heads of a group, per (sequence, chunk):
+    # G * 2Q^2N + H * (2Q^2P + 2QNP (C.S^T) + 2QNP (state increment))
+    chunks = w.batch * (T // w.chunk)
+    q = w.chunk
+    alg_flops = chunks * (w.G * 2 * q * q * w.N + w.H * (2 * q * q * w.P + 4 * q * w.N * w.P))
+    exec_flops = chunks * w.H * (2 * q * q * w.N + 2 * q * q * w.P + 4 * q * w.N * w.P)
+    return {
+        "workload": "prefill: 8 seqs x 2048 tokens, Nemotron-H layer, bf16, zero initial state",
+        "conv_us": conv_us, "conv_GBs": conv_bytes / conv_us / 1e3,
+        "conv_frac_hbm": conv_bytes / conv_us / 1e3 / peak_gbs,
+        "scan_us": scan_us, "scan_bytes": scan_bytes, "scan_GBs": scan_bytes / scan_us / 1e3,
+        "scan_frac_hbm": scan_bytes / scan_us / 1e3 / peak_gbs,
+        "scan_alg_flops": alg_flops, "scan_exec_flops": exec_flops,
+        "scan_alg_TFLOPs": alg_flops / scan_us / 1e6,
+        "scan_frac_fp16_tensor_peak": alg_flops / scan_us / 1e6 / peak_tflops,
+        "tokens_per_s": tokens / (scan_us + conv_us) * 1e6,
+    }
+
+
+def measure_stack48(flush, reps: int = 10) -> dict:
+    """Workload 2: one decode token for 384 sequences through 48 layers
+    (36 GiB of bf16 state), one CUDA graph of 48 fused launches per token."""
+    import torch
+    import mamba_recurrent_state_b200 as m2
+    from m2synth import torch_inputs as TI
+    from m2synth import workloads as W
+    w = W.WORKLOADS[2]
+    shape = m2.Shape(w.H, w.P, w.N, w.G, w.K, w.state_dtype, w.act_dtype)
+    caches, objs, inps = [], [], []
+    for layer in range(w.layers):
+        c = m2.Cache(shape, w.num_slots)
+        TI.fill_caches(w, c.ssm, c.conv, layer)
+        caches.append(c)
+        t = TI.layer_tensors(w, layer)
+        objs.append((t, m2.SSMParams(t["A_log"], t["dt_bias"], t["D"]),
+                     m2.ConvParams(t["conv_w"], t["conv_b"], 1)))
+        inps.append(TI.step_tensors(w, 0, layer))
+    ys = [torch.empty((w.batch, w.H * w.P), dtype=torch.bfloat16, device="cuda") for _ in caches]
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for layer in range(w.layers):
+            t, ssm, conv = objs[layer]
+            m2.state_update(caches[layer], ssm, inps[layer]["xBC"], inps[layer]["dt"], t["slots"],
+                            z=inps[layer]["z"], conv=conv, y=ys[layer])
+    for _ in range(3):
+        g.replay()
+    token_us = statistics.median(_time_us(g.replay, flush, reps))
+    for c in caches:
+        if c.device_error() != 0:
+            raise RuntimeError("device error word set during the 48-layer benchmark")
+    del g
+    bytes_tok = w.layers * (W.bytes_per_unit(w) * w.batch + W.param_bytes_per_launch(w))
+    return {"workload": "48 layers x 384 sequences, one token, CUDA graph of 48 launches",
+            "per_token_us": token_us, "per_layer_us": token_us / w.layers,
+            "bytes_per_token": bytes_tok, "GBs": bytes_tok / token_us / 1e3,
+            "seq_layer_steps_per_s": w.layers * w.batch / token_us * 1e6}
+
+
 def run_ours(args, world, rank, local):
     import torch
     import mamba_recurrent_state_b200 as m2
@@ -361,6 +491,15 @@ def run_ours(args, world, rank, local):
         "gpu_launches": args.steps,
         "clocks": clocks,
     }
+    sections = set(args.sections.split(","))
+    del cache, inputs, host_in
+    torch.cuda.empty_cache()
+    if "prefill" in sections:
+        tpeak, tkind = measured_tensor_peak()
+        line["prefill"] = measure_prefill(flush, peak, tpeak)
+        line["prefill"]["tensor_peak"] = f"{tpeak} TFLOP/s ({tkind} bf16_tflops)"
+    if "stack48" in sections:
+        line["stack48"] = measure_stack48(flush)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     if rank == 0:

@@ -90,12 +90,21 @@ __global__ void __launch_bounds__(kConvThreads) conv1d_kernel(const ConvArgs a) 
 #pragma unroll
     for (int j = 0; j < K - 1; ++j) unpack16<AT>(hist_raw[j], hist[j]);
 
+    // all of the tile's raw inputs are loaded before any output is stored, so
+    // the loads are in flight together (the output may alias nothing, but the
+    // compiler cannot know that)
+    uint4 raw[kTT];
+#pragma unroll
+    for (int i = 0; i < kTT; ++i) {
+        const int t = t0 + i;
+        raw[i] = t < t_end ? *reinterpret_cast<const uint4*>(xb + t * a.x_stride + c0) : make_uint4(0, 0, 0, 0);
+    }
 #pragma unroll
     for (int i = 0; i < kTT; ++i) {
         const int t = t0 + i;
         if (t < t_end) {
             float cur[VEC];
-            unpack16<AT>(*reinterpret_cast<const uint4*>(xb + t * a.x_stride + c0), cur);
+            unpack16<AT>(raw[i], cur);
             float o[VEC];
 #pragma unroll
             for (int v = 0; v < VEC; ++v) {
