@@ -303,7 +303,7 @@ def measure_prefill(flush, peak_gbs: float, peak_tflops: float, reps: int = 10) 
     xr = d["xBC"].view(w.batch, T, -1)
     dt = d["dt"].view(w.batch, T, -1)
     z = d["z"].view(w.batch, T, -1)
-    xp = torch.empty_like(xr)
+    xp = torch.empty(xr.shape, dtype=torch.float16, device="cuda")  # fp16 post-conv buffer
     y = torch.empty((w.batch, T, w.H * w.P), dtype=torch.bfloat16, device="cuda")
 
     def conv_step():

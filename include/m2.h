@@ -62,7 +62,12 @@ typedef struct CUstream_st* m2_stream;
 
 typedef enum m2_dtype {
     M2_F32 = 0,  /* IEEE binary32 */
-    M2_BF16 = 1  /* bfloat16 */
+    M2_BF16 = 1, /* bfloat16 */
+    M2_F16 = 2   /* IEEE binary16: only for the post-conv xBC buffer between
+                    m2_conv1d_update (out_dtype) and m2_state_update /
+                    m2_chunk_scan (xBC_dtype); its 11-bit significand keeps the
+                    post-conv values more precisely than bfloat16 and feeds the
+                    tensor-core scan without conversion */
 } m2_dtype;
 
 typedef enum m2_status {
@@ -156,7 +161,8 @@ m2_status m2_cache_zero_slots(const m2_cache* cache, int32_t n, const int32_t* s
  * divergence"; seqlen > 1 is the prefill conv that precedes the chunk scan).
  *   xBC      [batch, seqlen, conv_dim] act_dtype, raw; element (b,t,c) at
  *            xBC[(b*seqlen + t)*xBC_row_stride + c]
- *   xBC_out  [batch, seqlen, conv_dim] out_dtype (M2_F32 or M2_BF16), post-conv
+ *   xBC_out  [batch, seqlen, conv_dim] out_dtype (M2_F32, M2_BF16 or M2_F16),
+ *            post-conv (an fp16 value beyond 65504 records M2_ERR_RANGE)
  *            (bias added, activation applied); same indexing with out_row_stride
  *   slot_idx [batch] int32: row b reads its window history from, and writes
  *            the last K-1 raw inputs back to, cache->conv[slot_idx[b]]
@@ -173,6 +179,7 @@ m2_status m2_conv1d_update(const m2_cache* cache, const m2_conv_params* conv, in
  *   conv     non-NULL: xBC is the RAW row and the conv tap + roll of
  *            causal_conv1d_update run fused in the same launch (xBC_dtype must
  *            then be act_dtype); NULL: xBC is already post-conv, in xBC_dtype
+ *            (M2_F32, M2_BF16 or M2_F16)
  *   xBC      [batch, conv_dim], row stride xBC_row_stride
  *   dt       [batch, H] act_dtype (dt_raw, before dt_bias and softplus)
  *   z        [batch, H*P] act_dtype, or NULL for no gate
@@ -193,7 +200,8 @@ m2_status m2_state_update(const m2_cache* cache, const m2_ssm_params* ssm,
  * the recurrence starting from cache->ssm[slot_idx[b]] (or from zero when
  * has_initial_state is NULL or has_initial_state[b] == 0), writes y for every
  * token and stores the final state back to the same slot, rounded once.
- *   xBC      [batch, seqlen, conv_dim] xBC_dtype, POST-conv, row stride
+ *   xBC      [batch, seqlen, conv_dim] xBC_dtype (M2_F32, M2_BF16 or M2_F16),
+ *            POST-conv, row stride
  *            xBC_row_stride (token rows of a sequence are consecutive)
  *   dt       [batch, seqlen, H] act_dtype, row stride dt_row_stride
  *   z        [batch, seqlen, H*P] act_dtype or NULL, row stride z_row_stride

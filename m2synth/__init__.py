@@ -37,6 +37,7 @@ _MASK = (1 << 64) - 1
 
 F32 = 0
 BF16 = 1
+F16 = 2  # IEEE binary16 (only as a post-conv buffer; never drawn by the generator)
 
 # Tensor ids mixed into the per-tensor stream key.
 T_SSM = 1
@@ -143,6 +144,8 @@ def storage_to_f64(a: np.ndarray, dtype: int) -> np.ndarray:
         return np.asarray(a, dtype=np.float32).astype(np.float64)
     if dtype == BF16:
         return bf16_bits_to_f64(a)
+    if dtype == F16:
+        return np.asarray(a, dtype=np.float16).astype(np.float64)
     raise ValueError(f"unknown storage dtype {dtype}")
 
 

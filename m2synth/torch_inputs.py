@@ -31,6 +31,8 @@ def to_storage_np(t: torch.Tensor) -> np.ndarray:
         return t.numpy()
     if t.dtype == torch.bfloat16:
         return t.view(torch.int16).numpy().view(np.uint16)
+    if t.dtype == torch.float16:
+        return t.numpy()
     raise TypeError(t.dtype)
 
 

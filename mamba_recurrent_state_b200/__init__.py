@@ -32,6 +32,7 @@ LIB_PATH = os.path.join(_HERE, "libm2.so")
 
 M2_F32 = 0
 M2_BF16 = 1
+M2_F16 = 2  # post-conv xBC buffer only
 
 STATUS = {
     0: "ok",
@@ -136,7 +137,9 @@ def _dtype_code(t: torch.dtype) -> int:
         return M2_F32
     if t == torch.bfloat16:
         return M2_BF16
-    raise TypeError(f"unsupported dtype {t} (float32 or bfloat16)")
+    if t == torch.float16:
+        return M2_F16
+    raise TypeError(f"unsupported dtype {t} (float32, bfloat16, or float16 for a post-conv buffer)")
 
 
 def torch_dtype(code: int) -> torch.dtype:

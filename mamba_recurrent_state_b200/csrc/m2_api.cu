@@ -13,7 +13,9 @@
 
 namespace {
 
+// Storage dtypes of caches and activations; the post-conv buffer may also be fp16.
 bool valid_dtype(int32_t d) { return d == M2_F32 || d == M2_BF16; }
+bool valid_buffer_dtype(int32_t d) { return valid_dtype(d) || d == M2_F16; }
 int dsize(int32_t d) { return d == M2_F32 ? 4 : 2; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool stride_ok(int64_t stride_elems, int elem_size, int64_t min_elems) {
@@ -186,7 +188,7 @@ m2_status m2_conv1d_update(const m2_cache* c, const m2_conv_params* conv, int32_
                            m2_stream stream) {
     const m2_status st = cache_status(c);
     if (st != M2_OK) return st;
-    if (!conv || !conv->weight || batch < 0 || seqlen < 0 || !valid_dtype(out_dtype))
+    if (!conv || !conv->weight || batch < 0 || seqlen < 0 || !valid_buffer_dtype(out_dtype))
         return M2_ERR_INVALID_ARG;
     if (conv->activation != 0 && conv->activation != 1) return M2_ERR_INVALID_ARG;
     if (batch == 0 || seqlen == 0) return M2_OK;
@@ -208,7 +210,7 @@ m2_status m2_conv1d_update(const m2_cache* c, const m2_conv_params* conv, int32_
     a.K = s.d_conv;
     a.conv_dim = cd;
     a.act_bf16 = s.act_dtype == M2_BF16;
-    a.out_bf16 = out_dtype == M2_BF16;
+    a.out_dtype = out_dtype;
     a.w = conv->weight;
     a.b = conv->bias;
     a.activation = conv->activation;
@@ -228,7 +230,7 @@ m2_status m2_state_update(const m2_cache* c, const m2_ssm_params* ssm, const m2_
                           void* y, int64_t y_row_stride, const int32_t* slot_idx, m2_stream stream) {
     const m2_status st = cache_status(c);
     if (st != M2_OK) return st;
-    if (!ssm || !ssm->A_log || !ssm->dt_bias || !ssm->D || batch < 0 || !valid_dtype(xBC_dtype))
+    if (!ssm || !ssm->A_log || !ssm->dt_bias || !ssm->D || batch < 0 || !valid_buffer_dtype(xBC_dtype))
         return M2_ERR_INVALID_ARG;
     if (batch == 0) return M2_OK;
     if (!xBC || !dt || !y || !slot_idx) return M2_ERR_INVALID_ARG;
@@ -265,7 +267,7 @@ m2_status m2_state_update(const m2_cache* c, const m2_ssm_params* ssm, const m2_
     a.conv_dim = cd;
     a.state_bf16 = s.state_dtype == M2_BF16;
     a.act_bf16 = s.act_dtype == M2_BF16;
-    a.x_bf16 = xBC_dtype == M2_BF16;
+    a.x_dtype = xBC_dtype;
     a.A_log = ssm->A_log;
     a.dt_bias = ssm->dt_bias;
     a.D = ssm->D;
@@ -294,7 +296,7 @@ m2_status m2_chunk_scan(const m2_cache* c, const m2_ssm_params* ssm, int32_t bat
     const m2_status st = cache_status(c);
     if (st != M2_OK) return st;
     if (!ssm || !ssm->A_log || !ssm->dt_bias || !ssm->D || batch < 0 || seqlen < 0 ||
-        chunk_size <= 0 || !valid_dtype(xBC_dtype))
+        chunk_size <= 0 || !valid_buffer_dtype(xBC_dtype))
         return M2_ERR_INVALID_ARG;
     if (batch == 0 || seqlen == 0) return M2_OK;
     if (!xBC || !dt || !y || !slot_idx) return M2_ERR_INVALID_ARG;
@@ -306,9 +308,7 @@ m2_status m2_chunk_scan(const m2_cache* c, const m2_ssm_params* ssm, int32_t bat
         !stride_ok(y_row_stride, as, hp) || dt_row_stride < s.nheads)
         return M2_ERR_INVALID_ARG;
     if (z && (!aligned16(z) || !stride_ok(z_row_stride, as, hp))) return M2_ERR_INVALID_ARG;
-    const m2_status ps = m2::plan_chunk_scan(s.nheads, s.head_dim, s.d_state, s.ngroups,
-                                             s.state_dtype == M2_BF16, s.act_dtype == M2_BF16,
-                                             xBC_dtype == M2_BF16, chunk_size);
+    const m2_status ps = m2::plan_chunk_scan(s.nheads, s.head_dim, s.d_state, s.ngroups, chunk_size);
     if (ps != M2_OK) return ps;
     if (validate_mode()) {
         const m2_status v = validate_slots(slot_idx, batch, c->num_slots, reinterpret_cast<cudaStream_t>(stream));
@@ -324,7 +324,7 @@ m2_status m2_chunk_scan(const m2_cache* c, const m2_ssm_params* ssm, int32_t bat
     a.G = s.ngroups;
     a.state_bf16 = s.state_dtype == M2_BF16;
     a.act_bf16 = s.act_dtype == M2_BF16;
-    a.x_bf16 = xBC_dtype == M2_BF16;
+    a.x_dtype = xBC_dtype;
     a.A_log = ssm->A_log;
     a.dt_bias = ssm->dt_bias;
     a.D = ssm->D;

@@ -149,14 +149,15 @@ cudaError_t scan_by_shape(const ScanArgs& a, cudaStream_t s) {
 
 template <typename ST, typename AT>
 cudaError_t scan_by_x(const ScanArgs& a, cudaStream_t s) {
-    return a.x_bf16 ? scan_by_shape<ST, AT, bf16_t>(a, s) : scan_by_shape<ST, AT, float>(a, s);
+    if (a.x_dtype == M2_BF16) return scan_by_shape<ST, AT, bf16_t>(a, s);
+    if (a.x_dtype == M2_F16) return scan_by_shape<ST, AT, f16_t>(a, s);
+    return scan_by_shape<ST, AT, float>(a, s);
 }
 
 }  // namespace
 
-m2_status plan_chunk_scan(int H, int P, int N, int G, int state_bf16, int act_bf16, int x_bf16,
-                          int chunk) {
-    (void)H; (void)G; (void)state_bf16; (void)act_bf16; (void)x_bf16;
+m2_status plan_chunk_scan(int H, int P, int N, int G, int chunk) {
+    (void)H; (void)G;
     if (chunk <= 0) return M2_ERR_INVALID_ARG;
     if (P == 64 && (N == 128 || N == 64)) return M2_OK;
     return M2_ERR_UNSUPPORTED;

@@ -23,9 +23,10 @@
 // order of magnitude larger than y itself, so rounding M, W and the state copy
 // to bf16 (8-bit significand) leaves absolute errors of a few percent of
 // rms(y). The MMAs therefore take fp16 operands (11-bit significand, the same
-// A/B type in every MMA): the bf16 inputs C, B, X are converted exactly in
-// shared memory after each load, and M, W, S are rounded once to fp16. Any value
-// outside the fp16 range (|v| >= 65520) records M2_ERR_RANGE.
+// A/B type in every MMA): an fp16 post-conv buffer is used as loaded, a bf16 one
+// is converted exactly in shared memory after each load, and M, W, S are
+// rounded once to fp16. Any value outside the fp16 range (|v| >= 65520)
+// records M2_ERR_RANGE.
 //
 // One CTA of 256 threads per (sequence, head). Thread t owns TMEM lane
 // r = t % 128 (row r of every accumulator; warps w and w+4 share a lane quarter)
@@ -46,6 +47,7 @@
 #include <cuda_runtime.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "m2_device.cuh"
 #include "m2_internal.cuh"
@@ -159,7 +161,9 @@ __device__ __forceinline__ float bf16_chunk_to_f16(uint8_t* p) {
     return mx;
 }
 
-template <typename ST>
+// XT: element type of the post-conv xBC tiles (bf16_t: converted to fp16 in
+// shared memory after each load; f16_t: used as loaded).
+template <typename ST, typename XT>
 __global__ void __launch_bounds__(kTC, 2)
 chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs a) {
     extern __shared__ uint8_t s_raw[];
@@ -301,18 +305,20 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
         bool got = mbar_wait_bounded(&s_bar_ld, loads_done & 1, kLimitNs);
         if (!__syncthreads_and(got)) { ok = false; break; }
         ++loads_done;
-        // bf16 -> fp16 in place (exact within range): row t of C and B (atom h2)
-        // and half of row t of X
+        if constexpr (std::is_same<XT, bf16_t>::value) {
+            // bf16 -> fp16 in place (exact within range): row t of C and B
+            // (atom h2) and half of row t of X
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            range_max = fmaxf(range_max, bf16_chunk_to_f16(sm + kOffC + h2 * 16384 + t * 128 + j * 16));
-            range_max = fmaxf(range_max, bf16_chunk_to_f16(sm + kOffB + h2 * 16384 + t * 128 + j * 16));
+            for (int j = 0; j < 8; ++j) {
+                range_max = fmaxf(range_max, bf16_chunk_to_f16(sm + kOffC + h2 * 16384 + t * 128 + j * 16));
+                range_max = fmaxf(range_max, bf16_chunk_to_f16(sm + kOffB + h2 * 16384 + t * 128 + j * 16));
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                range_max = fmaxf(range_max, bf16_chunk_to_f16(sm + kOffX + t * 128 + (4 * h2 + j) * 16));
+            fence_proxy_async();
+            __syncthreads();
         }
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-            range_max = fmaxf(range_max, bf16_chunk_to_f16(sm + kOffX + t * 128 + (4 * h2 + j) * 16));
-        fence_proxy_async();
-        __syncthreads();
         const float cum_end = s_cum[kQ - 1];
         if (tid == 0) {
             tc_fence_after();
@@ -485,7 +491,8 @@ EncodeFn encode_fn() {
 }  // namespace
 
 bool chunk_scan_tc_supported(const ScanArgs& a) {
-    return a.P == kP && a.N == kN && a.state_bf16 && a.act_bf16 && a.x_bf16 && (a.xBC_stride * 2) % 16 == 0;
+    return a.P == kP && a.N == kN && a.state_bf16 && a.act_bf16 &&
+           (a.x_dtype == M2_BF16 || a.x_dtype == M2_F16) && (a.xBC_stride * 2) % 16 == 0;
 }
 
 cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t stream) {
@@ -501,13 +508,22 @@ cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t stream) {
                                    static_cast<cuuint64_t>(a.xBC_stride) * 2 * a.seqlen};
     const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kQ), 1};
     const cuuint32_t estr[3] = {1, 1, 1};
-    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(a.xBC), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    const bool f16_in = a.x_dtype == M2_F16;
+    if (enc(&map, f16_in ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+            const_cast<void*>(a.xBC), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    auto kern = chunk_scan_tc_kernel<bf16_t>;
-    static const cudaError_t attr_err =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
+    auto kern = f16_in ? chunk_scan_tc_kernel<bf16_t, f16_t> : chunk_scan_tc_kernel<bf16_t, bf16_t>;
+    static const cudaError_t attr_err = [] {
+        cudaError_t e = cudaFuncSetAttribute(chunk_scan_tc_kernel<bf16_t, f16_t>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(kSmemBytes));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(chunk_scan_tc_kernel<bf16_t, bf16_t>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
+        return e;
+    }();
     if (attr_err != cudaSuccess) return attr_err;
     const dim3 grid(static_cast<unsigned>(a.H), static_cast<unsigned>(a.batch));
     kern<<<grid, kTC, kSmemBytes, stream>>>(map, a);

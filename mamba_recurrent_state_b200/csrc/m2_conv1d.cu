@@ -16,6 +16,8 @@
 // new cache rows afterwards, so no other CTA can observe a half-rolled cache.
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "m2_device.cuh"
 #include "m2_internal.cuh"
 
@@ -30,7 +32,9 @@ constexpr int kTT = 16;  // tokens per thread
 template <typename OT, int VEC>
 __device__ __forceinline__ void store_vec(OT* p, const float* o) {
     if constexpr (sizeof(OT) == 2 && VEC == 4) {
-        *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
+        float t[8] = {o[0], o[1], o[2], o[3], 0.f, 0.f, 0.f, 0.f};
+        const uint4 v = pack16<OT>(t);
+        *reinterpret_cast<uint2*>(p) = make_uint2(v.x, v.y);
     } else {
         constexpr int OVEC = Vec16<OT>::n;
         static_assert(VEC % OVEC == 0, "whole 16-byte output vectors");
@@ -90,6 +94,7 @@ __global__ void __launch_bounds__(kConvThreads) conv1d_kernel(const ConvArgs a) 
 #pragma unroll
     for (int j = 0; j < K - 1; ++j) unpack16<AT>(hist_raw[j], hist[j]);
 
+    float out_max = 0.f;  // largest post-conv magnitude (checked for fp16 outputs)
     // all of the tile's raw inputs are loaded before any output is stored, so
     // the loads are in flight together (the output may alias nothing, but the
     // compiler cannot know that)
@@ -114,6 +119,10 @@ __global__ void __launch_bounds__(kConvThreads) conv1d_kernel(const ConvArgs a) 
                 acc = fmaf(w[v][K - 1], cur[v], acc);
                 o[v] = a.activation ? silu_f32(acc) : acc;
             }
+            if constexpr (std::is_same<OT, f16_t>::value) {
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) out_max = fmaxf(out_max, fabsf(o[v]));
+            }
             store_vec<OT, VEC>(ob + t * a.out_stride + c0, o);
 #pragma unroll
             for (int k = 0; k < K - 2; ++k) {
@@ -125,6 +134,7 @@ __global__ void __launch_bounds__(kConvThreads) conv1d_kernel(const ConvArgs a) 
         }
     }
 
+    if (out_max >= 65520.f) record_error(a.error, M2_ERR_RANGE);  // beyond fp16 (rounds to inf)
     if (blockIdx.y == 0) {
         // new cache row k holds the raw input of token T-(K-1)+k: from the input
         // when that token exists, else from the old cache rows read above
@@ -187,8 +197,14 @@ __global__ void __launch_bounds__(256) zero_slots_kernel(const ZeroArgs a) {
 }  // namespace
 
 cudaError_t launch_conv1d_update(const ConvArgs& a, cudaStream_t s) {
-    if (a.act_bf16) return a.out_bf16 ? conv_by_k<bf16_t, bf16_t>(a, s) : conv_by_k<bf16_t, float>(a, s);
-    return a.out_bf16 ? conv_by_k<float, bf16_t>(a, s) : conv_by_k<float, float>(a, s);
+    if (a.act_bf16) {
+        if (a.out_dtype == M2_BF16) return conv_by_k<bf16_t, bf16_t>(a, s);
+        if (a.out_dtype == M2_F16) return conv_by_k<bf16_t, f16_t>(a, s);
+        return conv_by_k<bf16_t, float>(a, s);
+    }
+    if (a.out_dtype == M2_BF16) return conv_by_k<float, bf16_t>(a, s);
+    if (a.out_dtype == M2_F16) return conv_by_k<float, f16_t>(a, s);
+    return conv_by_k<float, float>(a, s);
 }
 
 cudaError_t launch_zero_slots(const ZeroArgs& a, cudaStream_t s) {

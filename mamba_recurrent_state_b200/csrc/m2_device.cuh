@@ -7,8 +7,10 @@
 
 namespace m2 {
 
-// Storage types: bf16 is carried as its raw 16-bit pattern.
+// Storage types: bf16 is carried as its raw 16-bit pattern; fp16 (IEEE
+// binary16) as the CUDA __half type, so the two stay distinct C++ types.
 using bf16_t = uint16_t;
+using f16_t = __half;
 
 __device__ __forceinline__ float bf16_to_f32(bf16_t v) {
     return __uint_as_float(static_cast<uint32_t>(v) << 16);
@@ -32,12 +34,17 @@ __device__ __forceinline__ float to_f32<float>(float v) { return v; }
 template <>
 __device__ __forceinline__ float to_f32<bf16_t>(bf16_t v) { return bf16_to_f32(v); }
 
+template <>
+__device__ __forceinline__ float to_f32<f16_t>(f16_t v) { return __half2float(v); }
+
 template <typename T>
 __device__ __forceinline__ T from_f32(float v);
 template <>
 __device__ __forceinline__ float from_f32<float>(float v) { return v; }
 template <>
 __device__ __forceinline__ bf16_t from_f32<bf16_t>(float v) { return f32_to_bf16(v); }
+template <>
+__device__ __forceinline__ f16_t from_f32<f16_t>(float v) { return __float2half_rn(v); }
 
 // Elements of T per 16-byte vector.
 template <typename T>
@@ -79,9 +86,6 @@ __device__ __forceinline__ uint4 pack16<bf16_t>(const float* in) {
                       pack_bf16x2(in[4], in[5]), pack_bf16x2(in[6], in[7]));
 }
 
-// fp16 (IEEE binary16) carried as its raw 16-bit pattern.
-using f16_t = uint16_t;
-
 // Eight fp16 values <-> one 16-byte vector (round to nearest even).
 __device__ __forceinline__ void unpack16_f16(const uint4& v, float* out) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -101,6 +105,11 @@ __device__ __forceinline__ uint4 pack16_f16(const float* in) {
     }
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
+
+template <>
+__device__ __forceinline__ void unpack16<f16_t>(const uint4& v, float* out) { unpack16_f16(v, out); }
+template <>
+__device__ __forceinline__ uint4 pack16<f16_t>(const float* in) { return pack16_f16(in); }
 
 // Streaming 16-byte global load / store (data touched once per call).
 __device__ __forceinline__ uint4 ld_stream(const void* p) {

@@ -17,7 +17,8 @@ struct StateUpdateArgs {
     int64_t num_slots;
     int H, P, N, G, K;
     int64_t conv_dim;
-    int state_bf16, act_bf16, x_bf16;
+    int state_bf16, act_bf16;
+    int x_dtype;  // m2_dtype of xBC when it is post-conv (the unfused path)
     const float* A_log;
     const float* dt_bias;
     const float* D;
@@ -43,7 +44,8 @@ struct ConvArgs {
     int64_t num_slots;
     int K;
     int64_t conv_dim;
-    int act_bf16, out_bf16;
+    int act_bf16;
+    int out_dtype;  // m2_dtype of the post-conv output
     const void* w;
     const void* b;
     int activation;
@@ -71,7 +73,8 @@ struct ScanArgs {
     int32_t* error;
     int64_t num_slots;
     int H, P, N, G;
-    int state_bf16, act_bf16, x_bf16;
+    int state_bf16, act_bf16;
+    int x_dtype;  // m2_dtype of the post-conv xBC
     const float* A_log;
     const float* dt_bias;
     const float* D;
@@ -103,8 +106,7 @@ cudaError_t launch_state_update(const StateUpdateArgs& a, const DecodePlan& plan
                                 cudaStream_t stream);
 cudaError_t launch_conv1d_update(const ConvArgs& a, cudaStream_t stream);
 cudaError_t launch_zero_slots(const ZeroArgs& a, cudaStream_t stream);
-m2_status plan_chunk_scan(int H, int P, int N, int G, int state_bf16, int act_bf16, int x_bf16,
-                          int chunk);
+m2_status plan_chunk_scan(int H, int P, int N, int G, int chunk);
 cudaError_t launch_chunk_scan(const ScanArgs& a, cudaStream_t stream);
 // Tensor-core (tcgen05) scan: bf16 state, activations and xBC, P = 64, N = 128.
 bool chunk_scan_tc_supported(const ScanArgs& a);

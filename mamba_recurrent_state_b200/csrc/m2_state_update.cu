@@ -472,7 +472,8 @@ cudaError_t by_n(const StateUpdateArgs& a, const DecodePlan& p, cudaStream_t s) 
 template <typename ST, typename AT>
 cudaError_t by_mode(const StateUpdateArgs& a, const DecodePlan& p, cudaStream_t s) {
     if (a.fused) return by_n<ST, AT, AT, true>(a, p, s);
-    if (a.x_bf16) return by_n<ST, AT, bf16_t, false>(a, p, s);
+    if (a.x_dtype == M2_BF16) return by_n<ST, AT, bf16_t, false>(a, p, s);
+    if (a.x_dtype == M2_F16) return by_n<ST, AT, f16_t, false>(a, p, s);
     return by_n<ST, AT, float, false>(a, p, s);
 }
 

@@ -27,6 +27,7 @@ _LIB_PATH = os.path.join(_HERE, "libm2_oracle.so")
 ROUND_F32 = 0
 ROUND_BF16 = 1
 ROUND_NONE = 2
+ROUND_F16 = 3
 
 _dp = ctypes.POINTER(ctypes.c_double)
 
@@ -55,6 +56,8 @@ class Oracle:
         L.m2o_round_f32.argtypes = [ctypes.c_double]
         L.m2o_round_bf16.restype = ctypes.c_double
         L.m2o_round_bf16.argtypes = [ctypes.c_double]
+        L.m2o_round_f16.restype = ctypes.c_double
+        L.m2o_round_f16.argtypes = [ctypes.c_double]
         L.m2o_softplus.restype = ctypes.c_double
         L.m2o_softplus.argtypes = [ctypes.c_double]
         L.m2o_silu.restype = ctypes.c_double
@@ -80,6 +83,9 @@ class Oracle:
 
     def round_bf16(self, x: float) -> float:
         return self.lib.m2o_round_bf16(float(x))
+
+    def round_f16(self, x: float) -> float:
+        return self.lib.m2o_round_f16(float(x))
 
     def round_array(self, x, mode: int) -> np.ndarray:
         """Rounded copy of x (float64) in the given mode."""

@@ -46,6 +46,7 @@
 #define M2O_ROUND_F32 0
 #define M2O_ROUND_BF16 1
 #define M2O_ROUND_NONE 2
+#define M2O_ROUND_F16 3
 
 /* ---------------------------------------------------------------- rounding */
 
@@ -73,9 +74,24 @@ double m2o_round_bf16(double x) {
     return r;
 }
 
+/* Round to the nearest IEEE binary16 (11-bit significand, exponents -14..15,
+ * subnormal spacing 2^-24), ties to even, straight from double; beyond the
+ * largest finite value (65504) the result is an infinity. */
+double m2o_round_f16(double x) {
+    if (!isfinite(x) || x == 0.0) return x;
+    int e;
+    frexp(x, &e);
+    int ulp_exp = (e - 1) - 10;
+    if (ulp_exp < -24) ulp_exp = -24;
+    double r = ldexp(nearbyint(ldexp(x, -ulp_exp)), ulp_exp);
+    if (fabs(r) > 65504.0) r = copysign(INFINITY, x);
+    return r;
+}
+
 double m2o_round(double x, int mode) {
     if (mode == M2O_ROUND_F32) return m2o_round_f32(x);
     if (mode == M2O_ROUND_BF16) return m2o_round_bf16(x);
+    if (mode == M2O_ROUND_F16) return m2o_round_f16(x);
     return x;
 }
 

@@ -89,6 +89,39 @@ def pin_round_bf16_brute(orc: O.Oracle) -> None:
         assert got == want, (x, got, want)
 
 
+def _nearest_f16_brute(x: float) -> float:
+    """Exact nearest binary16 (ties to even) by searching the neighbours of
+    numpy's conversion over rationals."""
+    h = np.array([x], dtype=np.float64).astype(np.float16)
+    u = int(h.view(np.uint16)[0])
+    fx = Fraction(x)
+    best = None
+    for d in (-2, -1, 0, 1, 2):
+        b = (u + d) & 0xFFFF
+        v = float(np.array([b], dtype=np.uint16).view(np.float16)[0])
+        if not math.isfinite(v):
+            continue
+        key = (abs(Fraction(v) - fx), b & 1)
+        if best is None or key < best[0]:
+            best = (key, v)
+    return best[1]
+
+
+def pin_round_f16_brute(orc: O.Oracle) -> None:
+    """fp16 rounding = exact nearest binary16, ties to even, subnormals
+    included (brute force), and numpy's float64 -> float16 in range."""
+    rng = _rng(13)
+    xs = list(rng.normal(size=300) * 10.0 ** rng.integers(-7, 5, size=300))
+    for base in (1.0, 1.0009765625, -3.140625, 6.103515625e-05, 2.0 ** -20):
+        ulp = 2.0 ** max(math.frexp(abs(base))[1] - 1 - 10, -24)
+        xs += [base + ulp / 2, base - ulp / 2, base + 1.5 * ulp]
+    for x in xs:
+        got = orc.round_f16(float(x))
+        assert got == _nearest_f16_brute(float(x)), x
+        assert got == float(np.float16(x)), x
+    assert math.isinf(orc.round_f16(70000.0)) and orc.round_f16(65504.0) == 65504.0
+
+
 def pin_round_f32_library(orc: O.Oracle) -> None:
     """float32 rounding agrees with numpy's float64 -> float32 conversion."""
     rng = _rng(2)
@@ -412,6 +445,7 @@ def pin_state_rounding_on_store(orc: O.Oracle) -> None:
 
 ALL_PINS = [
     pin_round_bf16_brute,
+    pin_round_f16_brute,
     pin_round_f32_library,
     pin_softplus,
     pin_silu,

@@ -125,20 +125,23 @@ def test_fused_equals_conv_then_update_bitwise():
     assert torch.equal(a.ssm, b.ssm)
 
 
-def test_bf16_conv_output_between_launches():
-    """Unfused path with the conv output stored in bf16: the oracle rounds there too."""
+@pytest.mark.parametrize("buf", [torch.bfloat16, torch.float16], ids=["bf16", "f16"])
+def test_16bit_conv_output_between_launches(buf):
+    """Unfused path with the conv output stored in bf16 or fp16: the oracle
+    rounds there too."""
     w = W.WORKLOADS[1]
     cache = make_cache(w)
     t, ssm, conv = layer_objs(w)
     inp = TI.step_tensors(w, 0)
-    xp = m2.conv1d_update(cache, conv, inp["xBC"], t["slots"], out_dtype=torch.bfloat16)
+    xp = m2.conv1d_update(cache, conv, inp["xBC"], t["slots"], out_dtype=buf)
     y = m2.state_update(cache, ssm, xp, inp["dt"], t["slots"], z=inp["z"])
     torch.cuda.synchronize()
     ol = OracleLayer(w)
     rows = [0, 17, 63]
     ssm_rows = [ol.initial_ssm(ol.slots[r]) for r in rows]
     conv_rows = [ol.initial_conv(ol.slots[r]) for r in rows]
-    y_ref = ol.decode(ssm_rows, conv_rows, ol.inputs(0, rows), post_conv_round=O.ROUND_BF16)
+    rnd = O.ROUND_BF16 if buf == torch.bfloat16 else O.ROUND_F16
+    y_ref = ol.decode(ssm_rows, conv_rows, ol.inputs(0, rows), post_conv_round=rnd)
     assert_close(f64(TI.to_storage_np(y[rows]), w.act_dtype), y_ref, w.act_dtype, "y")
     for i, r in enumerate(rows):
         assert_close(f64(TI.to_storage_np(cache.ssm[int(ol.slots[r])]), w.state_dtype), ssm_rows[i],

@@ -39,7 +39,8 @@ def oracle_scan_row(ol, w, b, s, init: bool, x_code):
     rows = np.arange(b * w.seqlen, (b + 1) * w.seqlen)
     xbc = f64(W.step_rows(w, T_XBC, 0, rows), w.act_dtype)
     if x_code != w.act_dtype:  # xBC handed over in another precision
-        xbc = ol.orc.round_array(xbc, O.ROUND_F32 if x_code == S.F32 else O.ROUND_BF16)
+        mode = {S.F32: O.ROUND_F32, S.BF16: O.ROUND_BF16, S.F16: O.ROUND_F16}[x_code]
+        xbc = ol.orc.round_array(xbc, mode)
     dt = f64(W.step_rows(w, T_DT, 0, rows), w.act_dtype)
     z = f64(W.step_rows(w, T_Z, 0, rows), w.act_dtype)
     state = ol.initial_ssm(s) if init else np.zeros((w.H, w.P, w.N))
@@ -81,17 +82,21 @@ def test_scan_small(w):
     assert cache.device_error() == 0
 
 
-def test_scan_fp32_xbc_input():
-    w = wl(306, T=24)
+@pytest.mark.parametrize("xdt,code,T", [(torch.float32, S.F32, 24), (torch.float16, S.F16, 24),
+                                       (torch.float16, S.F16, 300)], ids=["f32", "f16", "f16_T300"])
+def test_scan_other_xbc_dtypes(xdt, code, T):
+    """Post-conv xBC handed over in fp32 (CUDA-core scan) or fp16 (tensor-core
+    scan, used as loaded)."""
+    w = wl(306 + T, T=T)
     cache = make_cache(w)
     t, ssm, _ = layer_objs(w)
     slots = torch.tensor([0, 3, 4], dtype=torch.int32, device="cuda")
-    x, dt, z = prefill_inputs(w, xdtype=torch.float32)
+    x, dt, z = prefill_inputs(w, xdtype=xdt)
     y = m2.chunk_scan(cache, ssm, x, dt, slots, z=z)
     torch.cuda.synchronize()
     ol = OracleLayer(w)
     for b, s in enumerate([0, 3, 4]):
-        state, y_ref = oracle_scan_row(ol, w, b, s, False, S.F32)
+        state, y_ref = oracle_scan_row(ol, w, b, s, False, code)
         assert_close(f64(TI.to_storage_np(y[b]), w.act_dtype), y_ref, w.act_dtype, "y")
         assert_close(f64(TI.to_storage_np(cache.ssm[s]), w.state_dtype), state, w.state_dtype, "S")
 
@@ -121,7 +126,7 @@ def test_scan_T1_equals_state_update(G):
 
 
 def test_workload4_prefill_then_decode():
-    """Zero initial state; prefill conv over 2048 tokens (bf16 post-conv buffer),
+    """Zero initial state; prefill conv over 2048 tokens (fp16 post-conv buffer),
     chunk scan, then 32 fused decode steps continuing from the scanned state.
     Every y and the states of all 8 sequences are checked.
 
@@ -139,7 +144,7 @@ def test_workload4_prefill_then_decode():
     T = w.seqlen
     d = TI.step_tensors(w, 0, rows=w.batch * T)
     xr = d["xBC"].view(w.batch, T, -1)
-    xp = m2.conv1d_update(cache, conv, xr, t["slots"], out_dtype=torch.bfloat16)
+    xp = m2.conv1d_update(cache, conv, xr, t["slots"], out_dtype=torch.float16)
     y_pre = m2.chunk_scan(cache, ssm, xp, d["dt"].view(w.batch, T, -1), t["slots"],
                           z=d["z"].view(w.batch, T, -1), chunk_size=w.chunk)
     state_after_prefill = TI.to_storage_np(cache.ssm[t["slots"].long()])
@@ -161,7 +166,7 @@ def test_workload4_prefill_then_decode():
         conv_state = np.zeros((w.K - 1, w.conv_dim))
         xraw = f64(W.step_rows(w, T_XBC, 0, rows), w.act_dtype)
         xpost = ol.orc.conv1d(conv_state, xraw, ol.conv_w, ol.conv_b, 1)
-        xpost = ol.orc.round_array(xpost, O.ROUND_BF16)  # the bf16 buffer between the launches
+        xpost = ol.orc.round_array(xpost, O.ROUND_F16)  # the fp16 buffer between the launches
         dt = f64(W.step_rows(w, T_DT, 0, rows), w.act_dtype)
         z = f64(W.step_rows(w, T_Z, 0, rows), w.act_dtype)
         state = np.zeros((w.H, w.P, w.N))
