@@ -170,8 +170,8 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
     __shared__ __align__(8) uint64_t s_bar_ld;
     __shared__ __align__(8) uint64_t s_bar_mma;
     __shared__ uint32_t s_tmem;
-    __shared__ float s_cum[kQ];
-    __shared__ float s_dt[kQ];
+    __shared__ __align__(16) float s_cum[kQ];
+    __shared__ __align__(16) float s_dt[kQ];
     __shared__ float s_wsum[kQ / 32];
 
     const int tid = threadIdx.x;
@@ -274,18 +274,30 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
 
     bool ok = true;
     int loads_issued = 1, loads_done = 0, mma_issued = 0, mma_done = 0;
+    float dt_raw_next = 0.f;  // raw dt of this thread's token in the next chunk
+    if (tid < kQ && tid < T) dt_raw_next = to_f32(static_cast<const bf16_t*>(a.dt)[(row0 + tid) * a.dt_stride + h]);
     for (int c = 0; c < nchunks; ++c) {
         const int t0 = c * kQ;
         const int valid = min(kQ, T - t0);
 
         // ---- dt and the cumulative decay c_t for the chunk (threads 0..127: token t)
         const int t = r;
+        // z of this thread's row half, loaded now so its latency overlaps the
+        // MMAs and epilogue 1 (used in epilogue 2)
+        uint4 zpre[4];
+        {
+            const bool zok = a.z != nullptr && t < valid;
+            const bf16_t* zr = zok ? static_cast<const bf16_t*>(a.z) + (row0 + t0 + t) * a.z_stride + xcol + 32 * h2
+                                   : nullptr;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) zpre[j] = zok ? *reinterpret_cast<const uint4*>(zr + 8 * j) : make_uint4(0, 0, 0, 0);
+        }
         {
             float dt = 0.f;
-            if (h2 == 0 && t < valid) {
-                const float raw = to_f32(static_cast<const bf16_t*>(a.dt)[(row0 + t0 + t) * a.dt_stride + h]);
-                dt = softplus_f32(raw + dt_bias);
-            }
+            if (h2 == 0 && t < valid) dt = softplus_f32(dt_raw_next + dt_bias);
+            // prefetch the next chunk's raw dt
+            if (h2 == 0 && c + 1 < nchunks && t < min(kQ, T - t0 - kQ))
+                dt_raw_next = to_f32(static_cast<const bf16_t*>(a.dt)[(row0 + t0 + kQ + t) * a.dt_stride + h]);
             float cum = dt * A;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
@@ -345,19 +357,36 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
         // W = w o B (row u = t of the B tile, scaled in place)
         {
             const float cum_t = s_cum[t];
+            const int wq = warp & 3;  // this warp's rows are t = 32*wq .. 32*wq+31
 #pragma unroll 1
-            for (int q = 2 * h2; q < 2 * h2 + 2; ++q) {  // columns u = 64*h2 .. 64*h2+63
+            for (int q = 2 * h2; q < 2 * h2 + 2; ++q) {  // columns u = 32q .. 32q+31
+                // 32 columns = 4 chunks of 8 in atom (q >> 1), chunks 4*(q&1) ..
+                uint8_t* dst = sm + kOffC + (q >> 1) * 16384;
+                if (q > wq) {  // every u > t: the causal mask zeroes the block (warp-uniform)
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj)
+                        *reinterpret_cast<uint4*>(dst + sw128(t, (q & 1) * 4 + jj)) = make_uint4(0, 0, 0, 0);
+                    continue;
+                }
                 float cb[32];
                 tmem_ld32(tmem + lane_base + kColCB + q * 32, cb);
                 float m[32];
+                const float4* cu4 = reinterpret_cast<const float4*>(s_cum + q * 32);
+                const float4* du4 = reinterpret_cast<const float4*>(s_dt + q * 32);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int u = q * 32 + i;
-                    m[i] = (u <= t) ? cb[i] * __expf(cum_t - s_cum[u]) * s_dt[u] : 0.f;
-                    range_max = fmaxf(range_max, fabsf(m[i]));
+                for (int i4 = 0; i4 < 8; ++i4) {
+                    const float4 cu = cu4[i4], du = du4[i4];
+                    const float cuv[4] = {cu.x, cu.y, cu.z, cu.w};
+                    const float duv[4] = {du.x, du.y, du.z, du.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int i = 4 * i4 + e;
+                        float v = cb[i] * __expf(cum_t - cuv[e]) * duv[e];
+                        if (q == wq && q * 32 + i > t) v = 0.f;  // diagonal block: mask u > t
+                        m[i] = v;
+                        range_max = fmaxf(range_max, fabsf(v));
+                    }
                 }
-                // 32 columns = 4 chunks of 8 in atom (q >> 1), chunks 4*(q&1) ..
-                uint8_t* dst = sm + kOffC + (q >> 1) * 16384;
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
                     const uint32_t j = (q & 1) * 4 + jj;
@@ -372,10 +401,13 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
                     uint4* p = reinterpret_cast<uint4*>(sm + kOffB + atom * 16384 + t * 128 + j * 16);
                     float v[8];
                     unpack16_f16(*p, v);
+                    const float2 w2 = make_float2(wu, wu);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        v[e] *= wu;
-                        range_max = fmaxf(range_max, fabsf(v[e]));
+                    for (int e = 0; e < 8; e += 2) {
+                        const float2 r2 = __fmul2_rn(make_float2(v[e], v[e + 1]), w2);
+                        v[e] = r2.x;
+                        v[e + 1] = r2.y;
+                        range_max = fmaxf(range_max, fmaxf(fabsf(r2.x), fabsf(r2.y)));
                     }
                     *p = pack16_f16(v);
                 }
@@ -409,7 +441,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
         {
             const float et = __expf(s_cum[t]);
             const bool row_ok = t < valid;
-            const bf16_t* zrow = a.z ? static_cast<const bf16_t*>(a.z) + (row0 + t0 + t) * a.z_stride + xcol : nullptr;
+            const bool gate = a.z != nullptr;
             bf16_t* yrow = y + (row0 + t0 + t) * a.y_stride + xcol;
             {
                 const int q = h2;  // columns p = 32*h2 .. 32*h2+31
@@ -422,12 +454,12 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
                     float xv[8], out[8];
                     unpack16_f16(*reinterpret_cast<const uint4*>(sm + kOffX + sw128(t, j)), xv);
                     float zv[8];
-                    if (zrow && row_ok) unpack16<bf16_t>(*reinterpret_cast<const uint4*>(zrow + 8 * j), zv);
+                    unpack16<bf16_t>(zpre[jj], zv);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         float v = fmaf(et, yo[8 * jj + e], yd[8 * jj + e]);
                         v = fmaf(Dh, xv[e], v);
-                        if (zrow) v *= silu_f32(zv[e]);
+                        if (gate) v *= silu_f32(zv[e]);
                         out[e] = v;
                     }
                     if (row_ok) *reinterpret_cast<uint4*>(yrow + 8 * j) = pack16<bf16_t>(out);
