@@ -12,12 +12,14 @@
 // with L[t,u] = exp(c_t - c_u) for u <= t, else 0. The four products run as
 // tcgen05 MMAs (M = 128, fp16 operands, fp32 accumulators in TMEM):
 //   MMA1  CB     [t,u] = C . B^T        A = C (K-major), B = B (K-major)
-//   MMA3  Yoff   [t,p] = C . S^T        A = C (K-major), B = S (K-major, bf16 copy)
-//   MMA2  Ydiag  [t,p] = M . X          A = M = CB o L o dt (K-major), B = X (MN-major)
+//   MMA3  Yoff   [t,p] = C . S^T        A = C (K-major), B = S (K-major, fp16 copy)
+//   MMA2  Ydiag  [t,p] = M . X          A = M = CB o L o dt + D I (K-major), B = X (MN-major)
 //   MMA4  dS^T   [n,p] = W^T . X        A = W = w o B (MN-major), B = X (MN-major)
 // The state itself is carried exactly in fp32 registers (thread n holds column
 // n of S) and rounded once when the sequence ends. Only the chunk-to-chunk carry
-// is sequential.
+// is sequential. D x rides on the diagonal of M, so once MMA2 and MMA4 are
+// done no operand tile is read again and the next chunk's TMA loads overlap
+// the output epilogue.
 //
 // Operand precision. The intra-chunk terms dt_u (C_t . B_u) x_u are often an
 // order of magnitude larger than y itself, so rounding M, W and the state copy
@@ -129,6 +131,30 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 16 consecutive fp32 columns of this thread's TMEM lane (load and wait as above).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+        "tcgen05.wait::ld.sync.aligned;\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 2^x with the hardware approximation (PTX ex2.approx, relative error about
+// 2^-22); the decay sums are kept in log2 units so exp(c) = 2^(c log2 e).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Generic-proxy shared-memory writes become visible to the async proxy
 // (tensor cores, TMA).
 __device__ __forceinline__ void fence_proxy_async() {
@@ -170,8 +196,11 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
     __shared__ __align__(8) uint64_t s_bar_ld;
     __shared__ __align__(8) uint64_t s_bar_mma;
     __shared__ uint32_t s_tmem;
-    __shared__ __align__(16) float s_cum[kQ];
+    __shared__ __align__(16) float s_cum[kQ];  // c_t in log2 units
     __shared__ __align__(16) float s_dt[kQ];
+    // g_u^(b) = exp(c_{32b} - c_u) dt_u for row blocks b = 1..3 and u < 32b,
+    // at offsets 0, 32, 96
+    __shared__ __align__(16) float s_gam[192];
     __shared__ float s_wsum[kQ / 32];
 
     const int tid = threadIdx.x;
@@ -228,6 +257,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;  // this warp's TMEM lanes
 
     const float A = -expf(a.A_log[h]);
+    const float A2 = A * 1.4426950408889634f;  // A log2(e)
     const float dt_bias = a.dt_bias[h];
     const float Dh = a.D[h];
     const int xcol = h * kP;
@@ -240,7 +270,8 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
     const int p0 = h2 * kPH;
     ST* state = static_cast<ST*>(a.ssm) + (static_cast<int64_t>(slot) * HP + static_cast<int64_t>(h) * kP) * kN;
     float S[kPH];
-    float range_max = 0.f;  // largest magnitude handed to an fp16 operand
+    float range_max = 0.f;  // largest magnitude handed to an fp16 operand (fp32 side)
+    __half2 hmax = __float2half2_rn(0.f);  // the same for values already rounded to fp16
     const bool init = a.has_init != nullptr && a.has_init[b] != 0;
 #pragma unroll
     for (int i = 0; i < kPH; ++i) S[i] = init ? to_f32(state[(p0 + i) * kN + n]) : 0.f;
@@ -298,7 +329,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
             // prefetch the next chunk's raw dt
             if (h2 == 0 && c + 1 < nchunks && t < min(kQ, T - t0 - kQ))
                 dt_raw_next = to_f32(static_cast<const bf16_t*>(a.dt)[(row0 + t0 + kQ + t) * a.dt_stride + h]);
-            float cum = dt * A;
+            float cum = dt * A2;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const float o = __shfl_up_sync(0xffffffffu, cum, off);
@@ -319,19 +350,26 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
         ++loads_done;
         if constexpr (std::is_same<XT, bf16_t>::value) {
             // bf16 -> fp16 in place (exact within range): row t of C and B
-            // (atom h2) and half of row t of X
+            // (atom h2) and half of row t of X. Chunks are visited in swizzled
+            // order (any order converts the whole row), so the eight rows a
+            // quarter-warp touches fall in different banks.
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                range_max = fmaxf(range_max, bf16_chunk_to_f16(sm + kOffC + h2 * 16384 + t * 128 + j * 16));
-                range_max = fmaxf(range_max, bf16_chunk_to_f16(sm + kOffB + h2 * 16384 + t * 128 + j * 16));
+                range_max = fmaxf(range_max, bf16_chunk_to_f16(sm + kOffC + h2 * 16384 + sw128(t, j)));
+                range_max = fmaxf(range_max, bf16_chunk_to_f16(sm + kOffB + h2 * 16384 + sw128(t, j)));
             }
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-                range_max = fmaxf(range_max, bf16_chunk_to_f16(sm + kOffX + t * 128 + (4 * h2 + j) * 16));
+                range_max = fmaxf(range_max, bf16_chunk_to_f16(sm + kOffX + sw128(t, 4 * h2 + j)));
             fence_proxy_async();
             __syncthreads();
         }
         const float cum_end = s_cum[kQ - 1];
+        if (tid < 192) {  // decay factors of the off-diagonal blocks of M (read after the MMA wait)
+            const int bq = tid < 32 ? 1 : (tid < 96 ? 2 : 3);
+            const int u = tid - (bq == 1 ? 0 : (bq == 2 ? 32 : 96));
+            s_gam[tid] = ex2(s_cum[32 * bq] - s_cum[u]) * s_dt[u];
+        }
         if (tid == 0) {
             tc_fence_after();
             for (int k = 0; k < kN / 16; ++k) {
@@ -353,64 +391,89 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
         ++mma_done;
         tc_fence_after();
 
-        // ---- epilogue 1: M = CB o L o dt (row t, bf16, into the C tile) and
-        // W = w o B (row u = t of the B tile, scaled in place)
+        // ---- epilogue 1: M = CB o L o dt + D I (row t, fp16, into the C tile)
+        // and W = w o B (row u = t of the B tile, scaled in place)
         {
             const float cum_t = s_cum[t];
             const int wq = warp & 3;  // this warp's rows are t = 32*wq .. 32*wq+31
+            // Off-diagonal blocks (u < 32 wq <= t) factor through the decay at
+            // the block start: L[t,u] = exp(c_t - c_{32wq}) exp(c_{32wq} - c_u),
+            // both factors <= 1 since c is non-increasing, so M = CB * alpha_t * g_u.
+            const float alpha = ex2(cum_t - s_cum[32 * wq]);
+            const float2 alpha2 = make_float2(alpha, alpha);
+            const float* gam = s_gam + (wq == 1 ? 0 : (wq == 2 ? 32 : 96));
 #pragma unroll 1
-            for (int q = 2 * h2; q < 2 * h2 + 2; ++q) {  // columns u = 32q .. 32q+31
-                // 32 columns = 4 chunks of 8 in atom (q >> 1), chunks 4*(q&1) ..
+            for (int q = 0; q < 4; ++q) {
+                // this thread's columns u = 32q + 16 h2 .. +15: chunks j0, j0+1 of atom q/2
                 uint8_t* dst = sm + kOffC + (q >> 1) * 16384;
+                const uint32_t j0 = (q & 1) * 4 + 2 * h2;
+                const int u0 = q * 32 + 16 * h2;
                 if (q > wq) {  // every u > t: the causal mask zeroes the block (warp-uniform)
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj)
-                        *reinterpret_cast<uint4*>(dst + sw128(t, (q & 1) * 4 + jj)) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4*>(dst + sw128(t, j0)) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4*>(dst + sw128(t, j0 + 1)) = make_uint4(0, 0, 0, 0);
                     continue;
                 }
-                float cb[32];
-                tmem_ld32(tmem + lane_base + kColCB + q * 32, cb);
-                float m[32];
-                const float4* cu4 = reinterpret_cast<const float4*>(s_cum + q * 32);
-                const float4* du4 = reinterpret_cast<const float4*>(s_dt + q * 32);
+                float m[16];
+                tmem_ld16(tmem + lane_base + kColCB + u0, m);
+                if (q < wq) {
+                    const float4* g4 = reinterpret_cast<const float4*>(gam + u0);
 #pragma unroll
-                for (int i4 = 0; i4 < 8; ++i4) {
-                    const float4 cu = cu4[i4], du = du4[i4];
-                    const float cuv[4] = {cu.x, cu.y, cu.z, cu.w};
-                    const float duv[4] = {du.x, du.y, du.z, du.w};
+                    for (int i4 = 0; i4 < 4; ++i4) {
+                        const float4 g = g4[i4];
+                        float2 lo = __fmul2_rn(make_float2(m[4 * i4], m[4 * i4 + 1]), make_float2(g.x, g.y));
+                        float2 hi = __fmul2_rn(make_float2(m[4 * i4 + 2], m[4 * i4 + 3]), make_float2(g.z, g.w));
+                        lo = __fmul2_rn(lo, alpha2);
+                        hi = __fmul2_rn(hi, alpha2);
+                        m[4 * i4] = lo.x;
+                        m[4 * i4 + 1] = lo.y;
+                        m[4 * i4 + 2] = hi.x;
+                        m[4 * i4 + 3] = hi.y;
+                    }
+                } else {  // diagonal block: exact per-element decay, mask u > t, D x_t rides on u = t
+                    const float4* cu4 = reinterpret_cast<const float4*>(s_cum + u0);
+                    const float4* du4 = reinterpret_cast<const float4*>(s_dt + u0);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int i = 4 * i4 + e;
-                        float v = cb[i] * __expf(cum_t - cuv[e]) * duv[e];
-                        if (q == wq && q * 32 + i > t) v = 0.f;  // diagonal block: mask u > t
-                        m[i] = v;
-                        range_max = fmaxf(range_max, fabsf(v));
+                    for (int i4 = 0; i4 < 4; ++i4) {
+                        const float4 cu = cu4[i4], du = du4[i4];
+                        const float cuv[4] = {cu.x, cu.y, cu.z, cu.w};
+                        const float duv[4] = {du.x, du.y, du.z, du.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int u = u0 + 4 * i4 + e;
+                            float v = m[4 * i4 + e] * ex2(cum_t - cuv[e]) * duv[e];
+                            if (u > t) v = 0.f;
+                            if (u == t) v += Dh;
+                            m[4 * i4 + e] = v;
+                        }
                     }
                 }
+                uint32_t hw[8];
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const uint32_t j = (q & 1) * 4 + jj;
-                    *reinterpret_cast<uint4*>(dst + sw128(t, j)) = pack16_f16(m + 8 * jj);
+                for (int i = 0; i < 8; ++i) {
+                    const __half2 hv = __floats2half2_rn(m[2 * i], m[2 * i + 1]);
+                    hmax = __hmax2(hmax, __habs2(hv));
+                    hw[i] = *reinterpret_cast<const uint32_t*>(&hv);
                 }
+                *reinterpret_cast<uint4*>(dst + sw128(t, j0)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4*>(dst + sw128(t, j0 + 1)) = make_uint4(hw[4], hw[5], hw[6], hw[7]);
             }
-            const float wu = (t < valid) ? __expf(cum_end - cum_t) * s_dt[t] : 0.f;
-            {
-                const int atom = h2;
+            // W row t = w_t * B row t, multiplied in fp16 pairs (w rounded once to fp16)
+            const float wu = (t < valid) ? ex2(cum_end - cum_t) * s_dt[t] : 0.f;
+            const __half2 w2 = __float2half2_rn(wu);
+            hmax = __hmax2(hmax, __habs2(w2));
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    uint4* p = reinterpret_cast<uint4*>(sm + kOffB + atom * 16384 + t * 128 + j * 16);
-                    float v[8];
-                    unpack16_f16(*p, v);
-                    const float2 w2 = make_float2(wu, wu);
+            for (int j = 0; j < 8; ++j) {
+                // swizzled chunk order: conflict-free across the quarter-warp's rows
+                uint4* p = reinterpret_cast<uint4*>(sm + kOffB + h2 * 16384 + sw128(t, j));
+                uint4 v = *p;
+                uint32_t* vw = reinterpret_cast<uint32_t*>(&v);
 #pragma unroll
-                    for (int e = 0; e < 8; e += 2) {
-                        const float2 r2 = __fmul2_rn(make_float2(v[e], v[e + 1]), w2);
-                        v[e] = r2.x;
-                        v[e + 1] = r2.y;
-                        range_max = fmaxf(range_max, fmaxf(fabsf(r2.x), fabsf(r2.y)));
-                    }
-                    *p = pack16_f16(v);
+                for (int e = 0; e < 4; ++e) {
+                    const __half2 r2 = __hmul2(*reinterpret_cast<const __half2*>(&vw[e]), w2);
+                    hmax = __hmax2(hmax, __habs2(r2));
+                    vw[e] = *reinterpret_cast<const uint32_t*>(&r2);
                 }
+                *p = v;
             }
         }
         fence_proxy_async();
@@ -436,10 +499,16 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
         if (!__syncthreads_and(got)) { ok = false; break; }
         ++mma_done;
         tc_fence_after();
+        // C, B and X are dead now (epilogue 2 reads TMEM and writes only the
+        // state copy): the next chunk's tiles stream in underneath it
+        if (tid == 0 && c + 1 < nchunks) {
+            issue_loads(c + 1);
+            ++loads_issued;
+        }
 
         // ---- epilogue 2: y row t, then the state carry (thread n = t)
         {
-            const float et = __expf(s_cum[t]);
+            const float et = ex2(s_cum[t]);
             const bool row_ok = t < valid;
             const bool gate = a.z != nullptr;
             bf16_t* yrow = y + (row0 + t0 + t) * a.y_stride + xcol;
@@ -451,21 +520,19 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
                     const uint32_t j = q * 4 + jj;  // chunk of 8 p values
-                    float xv[8], out[8];
-                    unpack16_f16(*reinterpret_cast<const uint4*>(sm + kOffX + sw128(t, j)), xv);
+                    float out[8];
                     float zv[8];
                     unpack16<bf16_t>(zpre[jj], zv);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        float v = fmaf(et, yo[8 * jj + e], yd[8 * jj + e]);
-                        v = fmaf(Dh, xv[e], v);
+                        float v = fmaf(et, yo[8 * jj + e], yd[8 * jj + e]);  // D x is in Ydiag
                         if (gate) v *= silu_f32(zv[e]);
                         out[e] = v;
                     }
                     if (row_ok) *reinterpret_cast<uint4*>(yrow + 8 * j) = pack16<bf16_t>(out);
                 }
             }
-            const float eend = __expf(cum_end);
+            const float eend = ex2(cum_end);
             {
                 float ds[32];
                 tmem_ld32(tmem + lane_base + kColDS + p0, ds);
@@ -477,14 +544,11 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
-        if (tid == 0 && c + 1 < nchunks) {
-            issue_loads(c + 1);
-            ++loads_issued;
-        }
     }
     if (ok) {
 #pragma unroll
         for (int i = 0; i < kPH; ++i) state[(p0 + i) * kN + n] = from_f32<ST>(S[i]);
+        range_max = fmaxf(range_max, fmaxf(__low2float(hmax), __high2float(hmax)));  // inf if rounded out of range
         if (range_max >= kF16Limit) record_error(a.error, M2_ERR_RANGE);
     } else {
         if (tid == 0) record_error(a.error, M2_ERR_TIMEOUT);
