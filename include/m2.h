@@ -107,7 +107,8 @@ typedef struct m2_cache {
 
 /* Depthwise causal conv parameters: weight [conv_dim, K] act_dtype (tap K-1
  * multiplies the newest input), bias [conv_dim] act_dtype or NULL,
- * activation 0 = none, 1 = SiLU. */
+ * activation 0 = none, 1 = SiLU. weight and bias are device pointers,
+ * 16-byte aligned (M2_ERR_INVALID_ARG otherwise). */
 typedef struct m2_conv_params {
     const void* weight;
     const void* bias;

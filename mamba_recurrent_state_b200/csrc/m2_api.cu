@@ -197,7 +197,8 @@ m2_status m2_conv1d_update(const m2_cache* c, const m2_conv_params* conv, int32_
     const int64_t cd = m2_conv_dim(&s);
     const int as = dsize(s.act_dtype);
     if (!aligned16(xBC) || !aligned16(xBC_out) || !stride_ok(xBC_row_stride, as, cd) ||
-        !stride_ok(out_row_stride, dsize(out_dtype), cd))
+        !stride_ok(out_row_stride, dsize(out_dtype), cd) || !aligned16(conv->weight) ||
+        (conv->bias && !aligned16(conv->bias)))
         return M2_ERR_INVALID_ARG;
     if (validate_mode()) {
         const m2_status v = validate_slots(slot_idx, batch, c->num_slots, reinterpret_cast<cudaStream_t>(stream));
@@ -240,6 +241,7 @@ m2_status m2_state_update(const m2_cache* c, const m2_ssm_params* ssm, const m2_
     const int64_t hp = static_cast<int64_t>(s.nheads) * s.head_dim;
     if (conv) {
         if (!conv->weight || (conv->activation != 0 && conv->activation != 1)) return M2_ERR_INVALID_ARG;
+        if (!aligned16(conv->weight) || (conv->bias && !aligned16(conv->bias))) return M2_ERR_INVALID_ARG;
         if (xBC_dtype != s.act_dtype) return M2_ERR_INVALID_ARG;
     }
     if (!aligned16(xBC) || !aligned16(y) || !stride_ok(xBC_row_stride, dsize(xBC_dtype), cd) ||

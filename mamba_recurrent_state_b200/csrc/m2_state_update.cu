@@ -99,26 +99,42 @@ __device__ __forceinline__ float reduce_rows(const float (&acc)[VPT], int lane, 
     }
 }
 
+// Slot-independent inputs of one conv vector (AV channels c0..): the raw
+// input, the bias and, for K = 4, the AV x K weight block, which is exactly
+// four 16-byte vectors with (e, k) at e*K + k. Loaded before the slot index
+// is known, so their latency overlaps the slot read and the bulk copies.
+struct ConvIn {
+    uint4 xin;
+    uint4 bias;
+    uint4 w[4];
+};
+
+template <typename AT>
+__device__ __forceinline__ ConvIn load_conv_in(const AT* xrow, const AT* w, const AT* bias, int64_t c0, int K) {
+    ConvIn in;
+    in.xin = *reinterpret_cast<const uint4*>(xrow + c0);
+    in.bias = bias ? __ldg(reinterpret_cast<const uint4*>(bias + c0)) : make_uint4(0, 0, 0, 0);
+    if (K == 4) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) in.w[q] = __ldg(reinterpret_cast<const uint4*>(w + c0 * 4) + q);
+    }
+    return in;
+}
+
 // Conv tap of AV consecutive channels c0.. for one row: the K-1 cached raw
 // inputs (staged in shared memory at `rows`, row pitch `pitch` elements,
-// oldest first) and the raw input `xin`; tap K-1 multiplies the newest input.
-// Weights and bias are loaded before waiting for the staged rows. Returns
-// false if the bounded wait for the rows ran out.
+// oldest first) and the raw input; tap K-1 multiplies the newest input.
+// Returns false if the bounded wait for the staged rows ran out.
 template <typename AT, int AV>
-__device__ __forceinline__ bool conv_vec_k4(const uint4& xin, const AT* w, const AT* bias, int64_t c0,
-                                            const AT* rows, int64_t pitch, int activation,
+__device__ __forceinline__ bool conv_vec_k4(const ConvIn& in, const AT* rows, int64_t pitch, int activation,
                                             uint64_t* bar, float (&out)[AV]) {
     constexpr int K = 4;
-    // the AV x K weight block is exactly K 16-byte vectors; (e, k) sits at e*K + k
-    uint4 wv[K];
-#pragma unroll
-    for (int q = 0; q < K; ++q) wv[q] = __ldg(reinterpret_cast<const uint4*>(w + c0 * K) + q);
     float wf[AV * K];
 #pragma unroll
-    for (int q = 0; q < K; ++q) unpack16<AT>(wv[q], wf + q * AV);
-#pragma unroll
-    for (int e = 0; e < AV; ++e) out[e] = bias ? to_f32(__ldg(bias + c0 + e)) : 0.f;
+    for (int q = 0; q < K; ++q) unpack16<AT>(in.w[q], wf + q * AV);
+    unpack16<AT>(in.bias, out);
     if (!mbar_wait_bounded(bar, 0, kWaitLimitNs)) return false;
+    const uint4& xin = in.xin;
     float xv[AV];
     unpack16<AT>(xin, xv);
 #pragma unroll
@@ -138,12 +154,12 @@ __device__ __forceinline__ bool conv_vec_k4(const uint4& xin, const AT* w, const
 
 // Same for any width K (2..8): weights read one by one (cached).
 template <typename AT, int AV>
-__device__ __forceinline__ bool conv_vec_any(const uint4& xin, const AT* w, const AT* bias, int64_t c0,
-                                             int K, const AT* rows, int64_t pitch, int activation,
+__device__ __forceinline__ bool conv_vec_any(const ConvIn& in, const AT* w, int64_t c0, int K,
+                                             const AT* rows, int64_t pitch, int activation,
                                              uint64_t* bar, float (&out)[AV]) {
-#pragma unroll
-    for (int e = 0; e < AV; ++e) out[e] = bias ? to_f32(__ldg(bias + c0 + e)) : 0.f;
+    unpack16<AT>(in.bias, out);
     if (!mbar_wait_bounded(bar, 0, kWaitLimitNs)) return false;
+    const uint4& xin = in.xin;
     float xv[AV];
     unpack16<AT>(xin, xv);
 #pragma unroll
@@ -207,9 +223,48 @@ state_update_kernel(const StateUpdateArgs a) {
     const int64_t cB = HP + static_cast<int64_t>(g) * N;                        // first B channel
     const int64_t cC = HP + static_cast<int64_t>(a.G) * N + static_cast<int64_t>(g) * N;
 
-    const int32_t slot = a.slot_idx[b];
     const AT* zrow = a.z ? static_cast<const AT*>(a.z) + b * a.z_stride : nullptr;
     AT* yrow = static_cast<AT*>(a.y) + b * a.y_stride;
+
+    // ---- slot-independent inputs first: under a saturated memory system every
+    // dependent round trip costs microseconds, so these loads are issued before
+    // the slot read and overlap it and the bulk copies.
+    // (a) this thread's first conv vector (fused) or x value and B/C column (unfused)
+    const bool first_half = tid < kHalf;
+    const int v_first = first_half ? tid : tid - kHalf;
+    ConvIn cin_first{};
+    float x_first = 0.f, b_first = 0.f, c_first = 0.f;
+    if constexpr (FUSED) {
+        const int nvec = first_half ? XV : 2 * BV;
+        if (v_first < nvec) {
+            const int64_t c0 = first_half ? r0 + static_cast<int64_t>(v_first) * AV
+                                          : ((v_first / BV) ? cC : cB) + (v_first % BV) * AV;
+            cin_first = load_conv_in<AT>(static_cast<const AT*>(a.xBC) + b * a.xBC_stride,
+                                         static_cast<const AT*>(a.conv_w), static_cast<const AT*>(a.conv_b),
+                                         c0, K);
+        }
+    } else {
+        const XT* xrow = static_cast<const XT*>(a.xBC) + b * a.xBC_stride;
+        if (tid < TILE) x_first = to_f32(xrow[r0 + tid]);
+        if (tid < N) {
+            b_first = to_f32(xrow[cB + tid]);
+            c_first = to_f32(xrow[cC + tid]);
+        }
+    }
+    // (b) the raw per-head scalars
+    float hs_dtr = 0.f, hs_bias = 0.f, hs_alog = 0.f, hs_D = 0.f;
+    if (tid < n_heads_tile) {
+        const int h = h_first + tid;
+        hs_dtr = to_f32(static_cast<const AT*>(a.dt)[b * a.dt_stride + h]);
+        hs_bias = a.dt_bias[h];
+        hs_alog = a.A_log[h];
+        hs_D = a.D[h];
+    }
+    // (c) z of this thread's first y row
+    float z_first = 0.f;
+    if (zrow && tid < TILE) z_first = to_f32(zrow[r0 + tid]);
+
+    const int32_t slot = a.slot_idx[b];
 
     if (slot < 0) {  // padding row: y = 0, caches untouched (uniform per cluster)
         for (int i = tid; i < TILE; i += kThreads) yrow[r0 + i] = from_f32<AT>(0.f);
@@ -247,15 +302,13 @@ state_update_kernel(const StateUpdateArgs a) {
                      CHUNK_BYTES, &s_bar[c]);
         }
     }
-    // per-head scalars
-    for (int i = tid; i < n_heads_tile; i += kThreads) {
-        const int h = h_first + i;
-        const float dtr = to_f32(static_cast<const AT*>(a.dt)[b * a.dt_stride + h]);
-        const float dt = softplus_f32(dtr + a.dt_bias[h]);
-        const float A = -expf(a.A_log[h]);
-        s_dt[i] = dt;
-        s_dA[i] = expf(dt * A);
-        s_D[i] = a.D[h];
+    // per-head scalars (n_heads_tile <= kMaxHeadsPerTile < kThreads: one per thread)
+    if (tid < n_heads_tile) {
+        const float dt = softplus_f32(hs_dtr + hs_bias);
+        const float A = -expf(hs_alog);
+        s_dt[tid] = dt;
+        s_dA[tid] = expf(dt * A);
+        s_D[tid] = hs_D;
     }
     __syncthreads();  // barrier initialisation and head scalars visible to all threads
 
@@ -264,9 +317,9 @@ state_update_kernel(const StateUpdateArgs a) {
         const AT* xrow = static_cast<const AT*>(a.xBC) + b * a.xBC_stride;
         const AT* w = static_cast<const AT*>(a.conv_w);
         const AT* bias = static_cast<const AT*>(a.conv_b);
-        const bool first_half = tid < kHalf;
         const int nvec = first_half ? XV : 2 * BV;
-        for (int v = first_half ? tid : tid - kHalf; v < nvec; v += kHalf) {
+        ConvIn cin = cin_first;  // the first vector's inputs were loaded up front
+        for (int v = v_first; v < nvec; v += kHalf) {
             // channel c0 .. c0+AV-1 and where its cached rows sit in shared memory
             int64_t c0;
             const AT* rows;
@@ -282,15 +335,14 @@ state_update_kernel(const StateUpdateArgs a) {
                 rows = s_cbc + seg * N + j0;
                 row_pitch = 2 * N;
             }
-            // inputs that do not depend on the slot (raw x, weights, bias) are
-            // loaded before waiting for the slot's staged conv rows
-            const uint4 xin = *reinterpret_cast<const uint4*>(xrow + c0);
+            if (v != v_first) cin = load_conv_in<AT>(xrow, w, bias, c0, K);
+            const uint4 xin = cin.xin;
             float out[AV];
             bool got;
             if (K == 4) {
-                got = conv_vec_k4<AT, AV>(xin, w, bias, c0, rows, row_pitch, a.activation, bar_conv, out);
+                got = conv_vec_k4<AT, AV>(cin, rows, row_pitch, a.activation, bar_conv, out);
             } else {
-                got = conv_vec_any<AT, AV>(xin, w, bias, c0, K, rows, row_pitch, a.activation, bar_conv, out);
+                got = conv_vec_any<AT, AV>(cin, w, c0, K, rows, row_pitch, a.activation, bar_conv, out);
             }
             if (!got) {
                 record_error(a.error, M2_ERR_TIMEOUT);
@@ -321,12 +373,12 @@ state_update_kernel(const StateUpdateArgs a) {
         const XT* xrow = static_cast<const XT*>(a.xBC) + b * a.xBC_stride;
         for (int i = tid; i < TILE; i += kThreads) {
             const int hl = static_cast<int>((r0 + i) / P) - h_first;
-            const float xv = to_f32(xrow[r0 + i]);
+            const float xv = (i == tid) ? x_first : to_f32(xrow[r0 + i]);
             s_rp[i] = make_float4(s_dt[hl] * xv, s_dA[hl], s_D[hl] * xv, 0.f);
         }
         for (int j = tid; j < N; j += kThreads) {
-            s_B[j] = to_f32(xrow[cB + j]);
-            s_C[j] = to_f32(xrow[cC + j]);
+            s_B[j] = (j == tid) ? b_first : to_f32(xrow[cB + j]);
+            s_C[j] = (j == tid) ? c_first : to_f32(xrow[cC + j]);
         }
     }
     __syncthreads();
@@ -389,7 +441,7 @@ state_update_kernel(const StateUpdateArgs a) {
     if (ok) {
         for (int i = tid; i < TILE; i += kThreads) {
             float yv = s_y[i];
-            if (zrow) yv *= silu_f32(to_f32(zrow[r0 + i]));
+            if (zrow) yv *= silu_f32(i == tid ? z_first : to_f32(zrow[r0 + i]));
             yrow[r0 + i] = from_f32<AT>(yv);
         }
     }
