@@ -42,9 +42,11 @@
  *    written for it, and M2_ERR_BAD_SLOT is recorded in the cache's error
  *    word. Slots must be unique within one call (checked on the host only when
  *    the environment variable M2_VALIDATE=1 is set, which synchronises).
- *  - All compute calls are asynchronous on `stream`, allocate nothing and never
- *    synchronise (outside M2_VALIDATE mode), so they can be captured in CUDA
- *    graphs. Argument errors are returned before anything is launched.
+ *  - All compute calls are asynchronous on `stream` and never synchronise
+ *    (outside M2_VALIDATE mode), so they can be captured in CUDA graphs. They
+ *    allocate nothing, except m2_chunk_scan_varlen when it splits sequences
+ *    (stream-ordered scratch, see there). Argument errors are returned before
+ *    anything is launched.
  *  - There is no CPU fallback: without a usable sm_100 device the compute
  *    calls fail with M2_ERR_CUDA.
  */
@@ -222,6 +224,43 @@ m2_status m2_chunk_scan(const m2_cache* cache, const m2_ssm_params* ssm, int32_t
                         const void* z, int64_t z_row_stride, void* y, int64_t y_row_stride,
                         const int32_t* slot_idx, const uint8_t* has_initial_state,
                         m2_stream stream);
+
+/*
+ * Variable-length prefill scan: the same recurrence as m2_chunk_scan over
+ * nseq sequences packed back to back (TensorRT-LLM issue #16976: mixed
+ * batches of long prompts, ~19K tokens). Sequence b is rows cu_seqlens[b] ..
+ * cu_seqlens[b+1]-1 of the packed arrays and runs from
+ * cache->ssm[slot_idx[b]] (or zero, as for m2_chunk_scan); its final state is
+ * stored back once. An empty sequence (cu_seqlens[b+1] == cu_seqlens[b])
+ * leaves its slot untouched.
+ *   cu_seqlens    [nseq+1] int32, device, non-decreasing, cu_seqlens[0] = 0,
+ *                 cu_seqlens[nseq] = total_tokens
+ *   total_tokens  rows of the packed arrays (host value, < 2^31)
+ *   max_seqlen    host upper bound on the sequence lengths, used only to plan
+ *                 the split below; a longer sequence is still computed
+ *                 correctly, with less parallelism
+ *   xBC           [total_tokens, conv_dim] xBC_dtype, POST-conv
+ *   dt            [total_tokens, H] act_dtype
+ *   z, y          [total_tokens, H*P] act_dtype (z may be NULL)
+ * Split sequences: on the tensor-core path (bf16 state and activations,
+ * P = 64, N = 128), when nseq * H (sequence, head) pairs are too few to fill
+ * the GPU (fewer than four per SM), each sequence is cut into segments of
+ * whole 128-token chunks that run in parallel: a first pass stores every
+ * segment's final state from a zero start and its total decay, a combine pass
+ * carries the states across segments in fp32 (the recurrence is linear in the
+ * state), and the scan pass runs each segment from its carried state. The
+ * scratch, nseq * segments * H * P * N * 4 bytes plus the decays, is taken with
+ * cudaMallocAsync and returned with cudaFreeAsync on `stream` (both
+ * stream-ordered and graph-capturable); M2_ERR_OOM if it cannot be had.
+ * Without a split the call allocates nothing.
+ */
+m2_status m2_chunk_scan_varlen(const m2_cache* cache, const m2_ssm_params* ssm, int32_t nseq,
+                               const int32_t* cu_seqlens, int64_t total_tokens, int32_t max_seqlen,
+                               int32_t chunk_size, const void* xBC, int32_t xBC_dtype,
+                               int64_t xBC_row_stride, const void* dt, int64_t dt_row_stride,
+                               const void* z, int64_t z_row_stride, void* y, int64_t y_row_stride,
+                               const int32_t* slot_idx, const uint8_t* has_initial_state,
+                               m2_stream stream);
 
 /* Debug/test path: synchronises `stream`, copies the cache's error word to
  * *out_code (0 or an m2_status value) and clears it. Not for hot loops. */

@@ -110,6 +110,14 @@ def slot_indices(w: Workload, layer: int = 0) -> np.ndarray:
     return perm[: w.batch].astype(np.int32)
 
 
+def slot_sets(w: Workload, layer: int = 0) -> list[np.ndarray]:
+    """The same permutation cut into num_slots // batch disjoint batches of
+    slots (set 0 is ``slot_indices``): a benchmark that rotates through them
+    touches each slot's state once per rotation."""
+    perm = permutation(stream_key(w.seed(layer), T_SLOTS), w.num_slots)
+    return [perm[i * w.batch:(i + 1) * w.batch].astype(np.int32) for i in range(w.num_slots // w.batch)]
+
+
 # --- initial caches: element index = flat index in the full cache tensor ----------
 
 def ssm_key(w: Workload, layer: int = 0) -> int:

@@ -5,6 +5,8 @@
 // on the host (the allocator and the error query are not hot-path calls).
 #include <cuda_runtime.h>
 
+#include <algorithm>
+
 #include <cstdlib>
 #include <cstring>
 #include <vector>
@@ -290,17 +292,20 @@ m2_status m2_state_update(const m2_cache* c, const m2_ssm_params* ssm, const m2_
     return from_cuda(m2::launch_state_update(a, plan, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-m2_status m2_chunk_scan(const m2_cache* c, const m2_ssm_params* ssm, int32_t batch, int32_t seqlen,
-                        int32_t chunk_size, const void* xBC, int32_t xBC_dtype, int64_t xBC_row_stride,
-                        const void* dt, int64_t dt_row_stride, const void* z, int64_t z_row_stride,
-                        void* y, int64_t y_row_stride, const int32_t* slot_idx,
-                        const uint8_t* has_initial_state, m2_stream stream) {
+namespace {
+
+// Shared by the fixed-length and the variable-length scan entry points:
+// validation and argument marshalling (cu_seqlens NULL: [batch, seqlen] rows).
+m2_status scan_args(const m2_cache* c, const m2_ssm_params* ssm, int32_t batch, int32_t chunk_size,
+                    const void* xBC, int32_t xBC_dtype, int64_t xBC_row_stride, const void* dt,
+                    int64_t dt_row_stride, const void* z, int64_t z_row_stride, void* y, int64_t y_row_stride,
+                    const int32_t* slot_idx, const uint8_t* has_initial_state, m2_stream stream,
+                    m2::ScanArgs* out) {
     const m2_status st = cache_status(c);
     if (st != M2_OK) return st;
-    if (!ssm || !ssm->A_log || !ssm->dt_bias || !ssm->D || batch < 0 || seqlen < 0 ||
-        chunk_size <= 0 || !valid_buffer_dtype(xBC_dtype))
+    if (!ssm || !ssm->A_log || !ssm->dt_bias || !ssm->D || batch < 0 || chunk_size <= 0 ||
+        !valid_buffer_dtype(xBC_dtype))
         return M2_ERR_INVALID_ARG;
-    if (batch == 0 || seqlen == 0) return M2_OK;
     if (!xBC || !dt || !y || !slot_idx) return M2_ERR_INVALID_ARG;
     const m2_shape& s = c->shape;
     const int as = dsize(s.act_dtype);
@@ -331,7 +336,6 @@ m2_status m2_chunk_scan(const m2_cache* c, const m2_ssm_params* ssm, int32_t bat
     a.dt_bias = ssm->dt_bias;
     a.D = ssm->D;
     a.batch = batch;
-    a.seqlen = seqlen;
     a.chunk = chunk_size;
     a.xBC = xBC;
     a.xBC_stride = xBC_row_stride;
@@ -343,7 +347,89 @@ m2_status m2_chunk_scan(const m2_cache* c, const m2_ssm_params* ssm, int32_t bat
     a.y_stride = y_row_stride;
     a.slot_idx = slot_idx;
     a.has_init = has_initial_state;
+    a.nseg = 1;
+    *out = a;
+    return M2_OK;
+}
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        n = 148;
+    return n > 0 ? n : 148;
+}
+
+}  // namespace
+
+m2_status m2_chunk_scan(const m2_cache* c, const m2_ssm_params* ssm, int32_t batch, int32_t seqlen,
+                        int32_t chunk_size, const void* xBC, int32_t xBC_dtype, int64_t xBC_row_stride,
+                        const void* dt, int64_t dt_row_stride, const void* z, int64_t z_row_stride,
+                        void* y, int64_t y_row_stride, const int32_t* slot_idx,
+                        const uint8_t* has_initial_state, m2_stream stream) {
+    if (seqlen < 0 || batch < 0) return M2_ERR_INVALID_ARG;
+    if (batch == 0 || seqlen == 0) {
+        const m2_status st = cache_status(c);
+        return st != M2_OK ? st : (ssm && chunk_size > 0 ? M2_OK : M2_ERR_INVALID_ARG);
+    }
+    if (static_cast<int64_t>(batch) * seqlen > INT32_MAX) return M2_ERR_UNSUPPORTED;
+    m2::ScanArgs a{};
+    const m2_status st = scan_args(c, ssm, batch, chunk_size, xBC, xBC_dtype, xBC_row_stride, dt, dt_row_stride,
+                                   z, z_row_stride, y, y_row_stride, slot_idx, has_initial_state, stream, &a);
+    if (st != M2_OK) return st;
+    a.seqlen = seqlen;
+    a.total_tokens = static_cast<int64_t>(batch) * seqlen;
     return from_cuda(m2::launch_chunk_scan(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+m2_status m2_chunk_scan_varlen(const m2_cache* c, const m2_ssm_params* ssm, int32_t nseq,
+                               const int32_t* cu_seqlens, int64_t total_tokens, int32_t max_seqlen,
+                               int32_t chunk_size, const void* xBC, int32_t xBC_dtype, int64_t xBC_row_stride,
+                               const void* dt, int64_t dt_row_stride, const void* z, int64_t z_row_stride,
+                               void* y, int64_t y_row_stride, const int32_t* slot_idx,
+                               const uint8_t* has_initial_state, m2_stream stream) {
+    if (nseq < 0 || total_tokens < 0 || max_seqlen < 0) return M2_ERR_INVALID_ARG;
+    if (total_tokens > INT32_MAX) return M2_ERR_UNSUPPORTED;
+    if (nseq == 0 || total_tokens == 0) {
+        const m2_status st = cache_status(c);
+        return st != M2_OK ? st : (ssm && chunk_size > 0 ? M2_OK : M2_ERR_INVALID_ARG);
+    }
+    if (!cu_seqlens) return M2_ERR_INVALID_ARG;
+    m2::ScanArgs a{};
+    const m2_status st = scan_args(c, ssm, nseq, chunk_size, xBC, xBC_dtype, xBC_row_stride, dt, dt_row_stride,
+                                   z, z_row_stride, y, y_row_stride, slot_idx, has_initial_state, stream, &a);
+    if (st != M2_OK) return st;
+    a.cu_seqlens = cu_seqlens;
+    a.seqlen = max_seqlen;
+    a.total_tokens = total_tokens;
+    const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    // Split long sequences across CTAs when there are too few (sequence, head)
+    // pairs to fill the GPU: two waves of two CTAs per SM.
+    const int64_t pairs = static_cast<int64_t>(nseq) * a.H;
+    const int64_t target = 4LL * sm_count();
+    const int max_chunks = (max_seqlen + 127) / 128;
+    if (m2::chunk_scan_tc_supported(a) && pairs < target && max_chunks >= 2) {
+        int nseg = static_cast<int>(std::min<int64_t>({(target + pairs - 1) / pairs, max_chunks, 32}));
+        const int seg_chunks = (max_chunks + nseg - 1) / nseg;
+        nseg = (max_chunks + seg_chunks - 1) / seg_chunks;
+        if (nseg > 1) {
+            const size_t state_bytes = static_cast<size_t>(nseq) * nseg * a.H * a.P * a.N * sizeof(float);
+            const size_t decay_bytes = static_cast<size_t>(nseq) * nseg * a.H * sizeof(float);
+            void* scratch = nullptr;
+            if (cudaMallocAsync(&scratch, state_bytes + decay_bytes, cs) != cudaSuccess) {
+                cudaGetLastError();
+                return M2_ERR_OOM;
+            }
+            a.nseg = nseg;
+            a.seg_chunks = seg_chunks;
+            a.seg_state = static_cast<float*>(scratch);
+            a.seg_decay = reinterpret_cast<float*>(static_cast<char*>(scratch) + state_bytes);
+            const cudaError_t e = m2::launch_chunk_scan(a, cs);
+            const cudaError_t f = cudaFreeAsync(scratch, cs);
+            return from_cuda(e != cudaSuccess ? e : f);
+        }
+    }
+    return from_cuda(m2::launch_chunk_scan(a, cs));
 }
 
 m2_status m2_get_device_error(const m2_cache* c, m2_stream stream, int32_t* out_code) {

@@ -47,10 +47,11 @@ __global__ void __launch_bounds__(kScanThreads) scan_seq_kernel(const ScanArgs a
     const int H = a.H;
     const int g = h / (H / a.G);
     const int64_t HP = static_cast<int64_t>(H) * P;
-    const int T = a.seqlen;
+    // this sequence's rows of the packed token arrays
+    const int64_t row0 = a.cu_seqlens ? static_cast<int64_t>(a.cu_seqlens[b]) : static_cast<int64_t>(b) * a.seqlen;
+    const int T = a.cu_seqlens ? a.cu_seqlens[b + 1] - a.cu_seqlens[b] : a.seqlen;
+    if (T <= 0) return;  // an empty sequence leaves its cache slot untouched
     const int32_t slot = a.slot_idx[b];
-
-    const int64_t row0 = static_cast<int64_t>(b) * T;  // first token row of this sequence
     AT* y = static_cast<AT*>(a.y);
     if (slot < 0) {
         for (int64_t i = tid; i < static_cast<int64_t>(T) * P; i += kScanThreads) {
@@ -164,7 +165,7 @@ m2_status plan_chunk_scan(int H, int P, int N, int G, int chunk) {
 }
 
 cudaError_t launch_chunk_scan(const ScanArgs& a, cudaStream_t s) {
-    if (a.batch == 0 || a.seqlen == 0) return cudaSuccess;
+    if (a.batch == 0 || a.total_tokens == 0) return cudaSuccess;
     if (chunk_scan_tc_supported(a)) return launch_chunk_scan_tc(a, s);
     if (a.state_bf16) return a.act_bf16 ? scan_by_x<bf16_t, bf16_t>(a, s) : scan_by_x<bf16_t, float>(a, s);
     return a.act_bf16 ? scan_by_x<float, bf16_t>(a, s) : scan_by_x<float, float>(a, s);

@@ -172,12 +172,11 @@ __device__ __forceinline__ void fence_proxy_async() {
     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
 }
 
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
-                                            uint64_t* bar) {
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
     asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5}], [%2];\n" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y), "r"(z)
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];\n" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y)
         : "memory");
 }
 
@@ -198,9 +197,21 @@ __device__ __forceinline__ float bf16_chunk_to_f16(uint8_t* p) {
     return mx;
 }
 
+// Segments a sequence of nchunks chunks is cut into: seg_chunks chunks each,
+// at most nseg (the grid's segments per sequence), 1 when unsplit.
+__device__ __forceinline__ int segments_of(int nchunks, int nseg, int seg_chunks) {
+    if (nseg <= 1 || nchunks <= seg_chunks) return 1;
+    return min(nseg, (nchunks + seg_chunks - 1) / seg_chunks);
+}
+
 // XT: element type of the post-conv xBC tiles (bf16_t: converted to fp16 in
 // shared memory after each load; f16_t: used as loaded).
-template <typename ST, typename XT>
+// STATE_ONLY: the first pass of a split sequence. The CTA runs one segment of
+// chunks from a zero state and stores only its final state (fp32, scratch)
+// and the segment's total decay: no C tile, no y, only the dS^T MMA.
+// Otherwise the CTA scans its segment (the whole sequence when unsplit) from
+// its initial state and writes y; the last segment stores the state.
+template <typename ST, typename XT, bool STATE_ONLY>
 __global__ void __launch_bounds__(kTC, 2)
 chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs a) {
     extern __shared__ uint8_t s_raw[];
@@ -222,26 +233,43 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
     const int r = tid & (kQ - 1);   // TMEM lane / tile row of this thread
     const int h2 = tid >> 7;        // column half of this thread
     const int h = blockIdx.x;
-    const int b = blockIdx.y;
+    const int nseg = a.nseg;  // segments per sequence in the grid (1: unsplit)
+    const int b = blockIdx.y / nseg;
+    const int seg = blockIdx.y - b * nseg;
     const int H = a.H;
     const int G = a.G;
     const int g = h / (H / G);
-    const int T = a.seqlen;
     const int64_t HP = static_cast<int64_t>(H) * kP;
+    // this sequence's rows of the packed token arrays, and its chunk range
+    const int64_t row0 = a.cu_seqlens ? static_cast<int64_t>(a.cu_seqlens[b]) : static_cast<int64_t>(b) * a.seqlen;
+    const int T = a.cu_seqlens ? a.cu_seqlens[b + 1] - a.cu_seqlens[b] : a.seqlen;
+    if (T <= 0) return;  // an empty sequence leaves its cache slot untouched
+    const int nchunks_seq = (T + kQ - 1) / kQ;
+    const int nseg_s = segments_of(nchunks_seq, nseg, a.seg_chunks);
+    const bool split = nseg_s > 1;
+    if (seg >= nseg_s) return;                                  // empty segment
+    if (STATE_ONLY && (!split || seg == nseg_s - 1)) return;   // nothing to summarise
+    // the last segment runs to the end of the sequence (also when the sequence
+    // is longer than the grid was planned for)
+    const int c_begin = split ? seg * a.seg_chunks : 0;
+    const int c_end = (split && seg < nseg_s - 1) ? c_begin + a.seg_chunks : nchunks_seq;
     const int32_t slot = a.slot_idx[b];
     bf16_t* y = static_cast<bf16_t*>(a.y);
-    const int64_t row0 = static_cast<int64_t>(b) * T;
 
-    if (slot < 0) {  // padding row: y = 0, cache untouched
-        for (int64_t i = tid; i < static_cast<int64_t>(T) * (kP / 8); i += kTC) {
-            const int64_t t = i / (kP / 8);
-            *reinterpret_cast<uint4*>(y + (row0 + t) * a.y_stride + h * kP + (i % (kP / 8)) * 8) =
-                make_uint4(0, 0, 0, 0);
+    if (slot < 0) {  // padding row: y = 0 over this segment's tokens, cache untouched
+        if constexpr (!STATE_ONLY) {
+            const int64_t tb = static_cast<int64_t>(c_begin) * kQ;
+            const int64_t te = min(static_cast<int64_t>(c_end) * kQ, static_cast<int64_t>(T));
+            for (int64_t i = tb * (kP / 8) + tid; i < te * (kP / 8); i += kTC) {
+                const int64_t t = i / (kP / 8);
+                *reinterpret_cast<uint4*>(y + (row0 + t) * a.y_stride + h * kP + (i % (kP / 8)) * 8) =
+                    make_uint4(0, 0, 0, 0);
+            }
         }
         return;
     }
     if (slot >= a.num_slots) {
-        if (tid == 0) record_error(a.error, M2_ERR_BAD_SLOT);
+        if (tid == 0 && !STATE_ONLY) record_error(a.error, M2_ERR_BAD_SLOT);
         return;
     }
 
@@ -285,9 +313,22 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
     float S[kPH];
     float range_max = 0.f;  // largest magnitude handed to an fp16 operand (fp32 side)
     __half2 hmax = __float2half2_rn(0.f);  // the same for values already rounded to fp16
-    const bool init = a.has_init != nullptr && a.has_init[b] != 0;
+    // scratch slot j of (sequence b, head h): [batch][nseg][H][P][N] fp32
+    auto seg_slot = [&](int j) {
+        return a.seg_state + ((static_cast<int64_t>(b) * nseg + j) * H + h) * (kP * kN);
+    };
+    if (STATE_ONLY) {
 #pragma unroll
-    for (int i = 0; i < kPH; ++i) S[i] = init ? to_f32(state[(p0 + i) * kN + n]) : 0.f;
+        for (int i = 0; i < kPH; ++i) S[i] = 0.f;
+    } else if (split) {  // initial state of this segment, from the combine pass
+        const float* src = seg_slot(seg);
+#pragma unroll
+        for (int i = 0; i < kPH; ++i) S[i] = src[(p0 + i) * kN + n];
+    } else {
+        const bool init = a.has_init != nullptr && a.has_init[b] != 0;
+#pragma unroll
+        for (int i = 0; i < kPH; ++i) S[i] = init ? to_f32(state[(p0 + i) * kN + n]) : 0.f;
+    }
     // fp16 copy for MMA3: element (p, n) of the K-major [2 atoms][64 p][64 n] tile
     auto write_state_copy = [&]() {
         uint8_t* sS = sm + kOffS + (n >> 6) * 8192;
@@ -300,36 +341,41 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
             *reinterpret_cast<__half*>(sS + sw128(p0 + i + 1, j) + (n & 7) * 2) = __high2half(hv);
         }
     };
-    write_state_copy();
+    if (!STATE_ONLY) write_state_copy();
 
-    const int nchunks = (T + kQ - 1) / kQ;
     const uint32_t id_cb = idesc_f16(128, 128, false, false);
     const uint32_t id_yoff = idesc_f16(128, 64, false, false);
     const uint32_t id_ydiag = idesc_f16(128, 64, false, true);
     const uint32_t id_ds = idesc_f16(128, 64, true, true);
+    // chunk c of the sequence = packed rows row0 + 128c ..; rows past the end
+    // of the buffer arrive as zeros, rows of the next sequence get dt = 0
     auto issue_loads = [&](int c) {
-        const int t0 = c * kQ;
-        mbar_arrive_expect_tx(&s_bar_ld, 5u * 16384u);
-        tma_load_3d(base + kOffX, &tmap_x, xcol, t0, b, &s_bar_ld);
-        tma_load_3d(base + kOffB, &tmap_x, bcol, t0, b, &s_bar_ld);
-        tma_load_3d(base + kOffB + 16384, &tmap_x, bcol + 64, t0, b, &s_bar_ld);
-        tma_load_3d(base + kOffC, &tmap_x, ccol, t0, b, &s_bar_ld);
-        tma_load_3d(base + kOffC + 16384, &tmap_x, ccol + 64, t0, b, &s_bar_ld);
+        const int ty = static_cast<int>(row0 + static_cast<int64_t>(c) * kQ);
+        mbar_arrive_expect_tx(&s_bar_ld, (STATE_ONLY ? 3u : 5u) * 16384u);
+        tma_load_2d(base + kOffX, &tmap_x, xcol, ty, &s_bar_ld);
+        tma_load_2d(base + kOffB, &tmap_x, bcol, ty, &s_bar_ld);
+        tma_load_2d(base + kOffB + 16384, &tmap_x, bcol + 64, ty, &s_bar_ld);
+        if (!STATE_ONLY) {
+            tma_load_2d(base + kOffC, &tmap_x, ccol, ty, &s_bar_ld);
+            tma_load_2d(base + kOffC + 16384, &tmap_x, ccol + 64, ty, &s_bar_ld);
+        }
     };
-    if (tid == 0) issue_loads(0);
+    if (tid == 0 && c_begin < c_end) issue_loads(c_begin);
 
     bool ok = true;
-    int loads_issued = 1, loads_done = 0, mma_issued = 0, mma_done = 0;
+    int loads_issued = c_begin < c_end ? 1 : 0, loads_done = 0, mma_issued = 0, mma_done = 0;
     const int t = r;  // token (row) of this thread within a chunk
     float dt_raw_next = 0.f;  // raw dt of this thread's token in the chunk to be prepared next
-    if (tid < kQ && tid < T) dt_raw_next = to_f32(static_cast<const bf16_t*>(a.dt)[(row0 + tid) * a.dt_stride + h]);
+    if (tid < kQ && c_begin * kQ + tid < T)
+        dt_raw_next = to_f32(static_cast<const bf16_t*>(a.dt)[(row0 + c_begin * kQ + tid) * a.dt_stride + h]);
+    float seg_log2 = 0.f;  // total decay of the chunks done so far, log2 units
     // dt and the cumulative decay c_t of chunk cn, in two parts around a block
     // barrier (warps 0..3, thread = token): the in-warp scan, then the
     // cross-warp prefix and the store into buffer cn & 1.
     auto cum_scan = [&](int cn, float& dt, float& cum) {
         const int vn = min(kQ, T - cn * kQ);
         dt = (t < vn) ? softplus_f32(dt_raw_next + dt_bias) : 0.f;
-        if (cn + 1 < nchunks && t < min(kQ, T - (cn + 1) * kQ))  // prefetch the following chunk's raw dt
+        if (cn + 1 < c_end && t < min(kQ, T - (cn + 1) * kQ))  // prefetch the following chunk's raw dt
             dt_raw_next = to_f32(static_cast<const bf16_t*>(a.dt)[(row0 + (cn + 1) * kQ + t) * a.dt_stride + h]);
         cum = dt * A2;
 #pragma unroll
@@ -346,11 +392,11 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
     };
     {
         float dt0 = 0.f, cum0 = 0.f;
-        if (h2 == 0) cum_scan(0, dt0, cum0);
+        if (h2 == 0 && c_begin < c_end) cum_scan(c_begin, dt0, cum0);
         __syncthreads();
-        if (h2 == 0) cum_store(0, dt0, cum0);
+        if (h2 == 0 && c_begin < c_end) cum_store(c_begin, dt0, cum0);
     }
-    for (int c = 0; c < nchunks; ++c) {
+    for (int c = c_begin; c < c_end; ++c) {
         const int t0 = c * kQ;
         const int valid = min(kQ, T - t0);
         const float* cum_c = s_cum[c & 1];
@@ -367,7 +413,8 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
             // quarter-warp touches fall in different banks.
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                range_max = fmaxf(range_max, bf16_chunk_to_f16(sm + kOffC + h2 * 16384 + sw128(t, j)));
+                if (!STATE_ONLY)
+                    range_max = fmaxf(range_max, bf16_chunk_to_f16(sm + kOffC + h2 * 16384 + sw128(t, j)));
                 range_max = fmaxf(range_max, bf16_chunk_to_f16(sm + kOffB + h2 * 16384 + sw128(t, j)));
             }
 #pragma unroll
@@ -377,6 +424,8 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
             __syncthreads();
         }
         const float cum_end = cum_c[kQ - 1];
+        seg_log2 += cum_end;
+        if constexpr (!STATE_ONLY) {
         if (tid < 192) {  // decay factors of the off-diagonal blocks of M (read after the MMA wait)
             const int bq = tid < 32 ? 1 : (tid < 96 ? 2 : 3);
             const int u = tid - (bq == 1 ? 0 : (bq == 2 ? 32 : 96));
@@ -402,11 +451,13 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
         if (!__syncthreads_and(got)) { ok = false; break; }
         ++mma_done;
         tc_fence_after();
+        }  // !STATE_ONLY
 
         // ---- epilogue 1: M = CB o L o dt + D I (row t, fp16, into the C tile)
         // and W = w o B (row u = t of the B tile, scaled in place)
         {
             const float cum_t = cum_c[t];
+            if constexpr (!STATE_ONLY) {
             const int wq = warp & 3;  // this warp's rows are t = 32*wq .. 32*wq+31
             // Off-diagonal blocks (u < 32 wq <= t) factor through the decay at
             // the block start: L[t,u] = exp(c_t - c_{32wq}) exp(c_{32wq} - c_u),
@@ -469,6 +520,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
                 *reinterpret_cast<uint4*>(dst + sw128(t, j0)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
                 *reinterpret_cast<uint4*>(dst + sw128(t, j0 + 1)) = make_uint4(hw[4], hw[5], hw[6], hw[7]);
             }
+            }  // !STATE_ONLY
             // W row t = w_t * B row t, multiplied in fp16 pairs (w rounded once to fp16)
             const float wu = (t < valid) ? ex2(cum_end - cum_t) * dt_c[t] : 0.f;
             const __half2 w2 = __float2half2_rn(wu);
@@ -495,10 +547,12 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
         // ---- MMA2 (Ydiag = M X) and MMA4 (dS^T = W^T X)
         if (tid == 0) {
             tc_fence_after();
-            for (int k = 0; k < kQ / 16; ++k) {
-                const uint32_t koff = (k >> 2) * 16384u + (k & 3) * 32u;
-                mma_f16(tmem + kColYdiag, sw128_desc(base + kOffC + koff, 16, 1024),
-                         sw128_desc(base + kOffX + k * 2048u, 16384, 1024), id_ydiag, k > 0);
+            if (!STATE_ONLY) {
+                for (int k = 0; k < kQ / 16; ++k) {
+                    const uint32_t koff = (k >> 2) * 16384u + (k & 3) * 32u;
+                    mma_f16(tmem + kColYdiag, sw128_desc(base + kOffC + koff, 16, 1024),
+                             sw128_desc(base + kOffX + k * 2048u, 16384, 1024), id_ydiag, k > 0);
+                }
             }
             for (int k = 0; k < kQ / 16; ++k) {
                 mma_f16(tmem + kColDS, sw128_desc(base + kOffB + k * 2048u, 16384, 1024),
@@ -511,7 +565,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
         // overlaps the MMAs
         uint4 zpre[4];
         {
-            const bool zok = a.z != nullptr && t < valid;
+            const bool zok = !STATE_ONLY && a.z != nullptr && t < valid;
             const bf16_t* zr = zok ? static_cast<const bf16_t*>(a.z) + (row0 + t0 + t) * a.z_stride + xcol + 32 * h2
                                    : nullptr;
 #pragma unroll
@@ -519,15 +573,15 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
         }
         // the next chunk's dt and decay sums, while the MMAs run
         float dt_n = 0.f, cum_n = 0.f;
-        if (h2 == 0 && c + 1 < nchunks) cum_scan(c + 1, dt_n, cum_n);
+        if (h2 == 0 && c + 1 < c_end) cum_scan(c + 1, dt_n, cum_n);
         got = mbar_wait_bounded(&s_bar_mma, mma_done & 1, kLimitNs);
         if (!__syncthreads_and(got)) { ok = false; break; }
         ++mma_done;
         tc_fence_after();
-        if (h2 == 0 && c + 1 < nchunks) cum_store(c + 1, dt_n, cum_n);
+        if (h2 == 0 && c + 1 < c_end) cum_store(c + 1, dt_n, cum_n);
         // C, B and X are dead now (epilogue 2 reads TMEM and writes only the
         // state copy): the next chunk's tiles stream in underneath it
-        if (tid == 0 && c + 1 < nchunks) {
+        if (tid == 0 && c + 1 < c_end) {
             issue_loads(c + 1);
             ++loads_issued;
         }
@@ -539,7 +593,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
             const bool row_ok = t < valid;
             const bool gate = a.z != nullptr;
             bf16_t* yrow = y + (row0 + t0 + t) * a.y_stride + xcol;
-            {
+            if constexpr (!STATE_ONLY) {
                 const int q = h2;  // columns p = 32*h2 .. 32*h2+31, in two passes of 16
                 const float2 et2 = make_float2(et, et);
 #pragma unroll
@@ -574,15 +628,22 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
 #pragma unroll
                 for (int i = 0; i < kPH; ++i) S[i] = fmaf(eend, S[i], ds[i]);
             }
-            write_state_copy();
+            if (!STATE_ONLY) write_state_copy();
         }
         fence_proxy_async();
         tc_fence_before();
         __syncthreads();
     }
     if (ok) {
+        if constexpr (STATE_ONLY) {  // segment summary for the combine pass
+            float* dst = seg_slot(seg + 1);
 #pragma unroll
-        for (int i = 0; i < kPH; ++i) state[(p0 + i) * kN + n] = from_f32<ST>(S[i]);
+            for (int i = 0; i < kPH; ++i) dst[(p0 + i) * kN + n] = S[i];
+            if (tid == 0) a.seg_decay[(static_cast<int64_t>(b) * nseg + seg) * H + h] = ex2(seg_log2);
+        } else if (!split || seg == nseg_s - 1) {  // the sequence's final state, in place
+#pragma unroll
+            for (int i = 0; i < kPH; ++i) state[(p0 + i) * kN + n] = from_f32<ST>(S[i]);
+        }
         range_max = fmaxf(range_max, fmaxf(__low2float(hmax), __high2float(hmax)));  // inf if rounded out of range
         if (range_max >= kF16Limit) record_error(a.error, M2_ERR_RANGE);
     } else {
@@ -626,37 +687,83 @@ bool chunk_scan_tc_supported(const ScanArgs& a) {
            (a.x_dtype == M2_BF16 || a.x_dtype == M2_F16) && (a.xBC_stride * 2) % 16 == 0;
 }
 
+// Combine pass of a split sequence (CUDA cores, fp32): scratch slot 0 <- the
+// initial state (the cache's, or zero), then slot j+1 <- decay_j * slot j +
+// slot j+1, where slot j+1 held segment j's summary (its final state from a
+// zero start). Afterwards slot j is the state entering segment j.
+template <typename ST>
+__global__ void __launch_bounds__(256) seg_combine_kernel(const ScanArgs a) {
+    constexpr int kPN = kP * kN;
+    const int h = blockIdx.x;
+    const int b = blockIdx.y;
+    const int H = a.H;
+    const int T = a.cu_seqlens ? a.cu_seqlens[b + 1] - a.cu_seqlens[b] : a.seqlen;
+    const int nseg_s = segments_of((T + kQ - 1) / kQ, a.nseg, a.seg_chunks);
+    if (nseg_s <= 1) return;
+    const int32_t slot = a.slot_idx[b];
+    if (slot < 0 || slot >= a.num_slots) return;  // the scan pass handles both
+    const bool init = a.has_init != nullptr && a.has_init[b] != 0;
+    const ST* st = static_cast<const ST*>(a.ssm) +
+                   (static_cast<int64_t>(slot) * H + h) * static_cast<int64_t>(kPN);
+    float* slot0 = a.seg_state + (static_cast<int64_t>(b) * a.nseg * H + h) * kPN;
+    const int64_t slot_stride = static_cast<int64_t>(H) * kPN;
+    const float* decay = a.seg_decay + static_cast<int64_t>(b) * a.nseg * H + h;
+    for (int e = threadIdx.x; e < kPN; e += blockDim.x) {
+        float v = init ? to_f32(st[e]) : 0.f;
+        slot0[e] = v;
+        for (int j = 0; j + 1 < nseg_s; ++j) {
+            float* nxt = slot0 + (j + 1) * slot_stride + e;
+            v = fmaf(decay[static_cast<int64_t>(j) * H], v, *nxt);
+            *nxt = v;
+        }
+    }
+}
+
 cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t stream) {
     EncodeFn enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
-    // xBC as a 3-D tensor (channel, token, sequence), 64 x 128 x 1 boxes of bf16,
-    // 128-byte swizzle; out-of-range tokens read as zeros
+    // xBC as a 2-D tensor (channel, packed token row), 64 x 128 boxes of 16-bit
+    // elements, 128-byte swizzle; rows past the end of the buffer read as zeros
     CUtensorMap map;
     const int64_t cd = static_cast<int64_t>(a.H) * a.P + 2LL * a.G * a.N;
-    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(cd), static_cast<cuuint64_t>(a.seqlen),
-                                static_cast<cuuint64_t>(a.batch)};
-    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(a.xBC_stride) * 2,
-                                   static_cast<cuuint64_t>(a.xBC_stride) * 2 * a.seqlen};
-    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kQ), 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cd), static_cast<cuuint64_t>(a.total_tokens)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.xBC_stride) * 2};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(kQ)};
+    const cuuint32_t estr[2] = {1, 1};
     const bool f16_in = a.x_dtype == M2_F16;
-    if (enc(&map, f16_in ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+    if (enc(&map, f16_in ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
             const_cast<void*>(a.xBC), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    auto kern = f16_in ? chunk_scan_tc_kernel<bf16_t, f16_t> : chunk_scan_tc_kernel<bf16_t, bf16_t>;
-    static const cudaError_t attr_err = [] {
-        cudaError_t e = cudaFuncSetAttribute(chunk_scan_tc_kernel<bf16_t, f16_t>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(kSmemBytes));
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(chunk_scan_tc_kernel<bf16_t, bf16_t>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
-        return e;
-    }();
+    static AttrOnce attrs;
+    const cudaError_t attr_err = attrs.ensure([] {
+        const void* kerns[4] = {
+            reinterpret_cast<const void*>(chunk_scan_tc_kernel<bf16_t, f16_t, false>),
+            reinterpret_cast<const void*>(chunk_scan_tc_kernel<bf16_t, bf16_t, false>),
+            reinterpret_cast<const void*>(chunk_scan_tc_kernel<bf16_t, f16_t, true>),
+            reinterpret_cast<const void*>(chunk_scan_tc_kernel<bf16_t, bf16_t, true>)};
+        for (const void* k : kerns) {
+            const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                       static_cast<int>(kSmemBytes));
+            if (e != cudaSuccess) return e;
+        }
+        return cudaSuccess;
+    });
     if (attr_err != cudaSuccess) return attr_err;
-    const dim3 grid(static_cast<unsigned>(a.H), static_cast<unsigned>(a.batch));
+    const int nseg = a.nseg > 1 ? a.nseg : 1;
+    const dim3 grid(static_cast<unsigned>(a.H), static_cast<unsigned>(a.batch) * static_cast<unsigned>(nseg));
+    if (nseg > 1) {  // pass 1: segment summaries; pass 2: carry them across segments
+        auto summ = f16_in ? chunk_scan_tc_kernel<bf16_t, f16_t, true> : chunk_scan_tc_kernel<bf16_t, bf16_t, true>;
+        summ<<<grid, kTC, kSmemBytes, stream>>>(map, a);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        seg_combine_kernel<bf16_t><<<dim3(static_cast<unsigned>(a.H), static_cast<unsigned>(a.batch)), 256, 0,
+                                     stream>>>(a);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    auto kern = f16_in ? chunk_scan_tc_kernel<bf16_t, f16_t, false> : chunk_scan_tc_kernel<bf16_t, bf16_t, false>;
     kern<<<grid, kTC, kSmemBytes, stream>>>(map, a);
     return cudaGetLastError();
 }

@@ -5,9 +5,29 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "m2.h"
 
 namespace m2 {
+
+// Runs a kernel's one-time function-attribute setup once per device (the
+// attributes belong to the device's context). Concurrent first calls may both
+// run the setup, which is harmless; a failure is returned and retried.
+struct AttrOnce {
+    static constexpr int kMaxDevices = 64;
+    std::atomic<int> done[kMaxDevices] = {};
+    template <typename F>
+    cudaError_t ensure(F&& setup) {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < kMaxDevices && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+        e = setup();
+        if (e == cudaSuccess && dev >= 0 && dev < kMaxDevices) done[dev].store(1, std::memory_order_release);
+        return e;
+    }
+};
 
 // Everything a decode-step launch needs (host-validated).
 struct StateUpdateArgs {
@@ -89,6 +109,15 @@ struct ScanArgs {
     int64_t y_stride;
     const int32_t* slot_idx;
     const uint8_t* has_init;
+    // variable-length batches: sequence b is packed rows cu_seqlens[b] ..
+    // cu_seqlens[b+1]-1 (NULL: rows b*seqlen .. of a [batch, seqlen] layout)
+    const int32_t* cu_seqlens;
+    int64_t total_tokens;  // rows of the packed xBC / dt / z / y
+    // split sequences (tensor-core path): nseg segments of seg_chunks chunks
+    // per sequence in the grid; nseg = 1 runs every sequence in one CTA per head
+    int nseg, seg_chunks;
+    float* seg_state;  // [batch][nseg][H][P][N] fp32 scratch (nseg > 1)
+    float* seg_decay;  // [batch][nseg][H] fp32 scratch (nseg > 1)
 };
 
 // Launch-shape query for the decode kernels: M2_OK and the shape, or

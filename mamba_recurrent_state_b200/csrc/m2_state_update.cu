@@ -476,13 +476,19 @@ cudaError_t launch_one(const StateUpdateArgs& a, const DecodePlan& plan, cudaStr
     constexpr int TILE = CHUNKS * (kThreads / LPR) * VPT;
     size_t smem = static_cast<size_t>(TILE) * N * sizeof(ST);
     if (FUSED) smem += static_cast<size_t>(a.K - 1) * (TILE + 2 * N) * sizeof(AT);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    if (FUSED && plan.cluster > 8) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (e != cudaSuccess) return e;
-    }
+    // function attributes once per instantiation and device, sized for the
+    // widest conv (K = 8), so the launch path makes no extra driver calls
+    static AttrOnce attrs;
+    const cudaError_t attr_err = attrs.ensure([&] {
+        size_t smem_max = static_cast<size_t>(TILE) * N * sizeof(ST);
+        if (FUSED) smem_max += static_cast<size_t>(7) * (TILE + 2 * N) * sizeof(AT);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem_max));
+        if (e == cudaSuccess && FUSED)
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        return e;
+    });
+    if (attr_err != cudaSuccess) return attr_err;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(plan.ctas_per_seq, a.batch, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
