@@ -360,6 +360,29 @@ int sm_count() {
     return n > 0 ? n : 148;
 }
 
+// Split plan of a variable-length scan: when the (sequence, head) pairs are
+// too few to fill the GPU (two waves of two CTAs per SM) and the tensor-core
+// path applies, sequences are cut into segments of seg_chunks 128-token
+// chunks, nseg per sequence in the grid. Returns the scratch bytes (state
+// slots, then decays; 0 without a split) and sets a->nseg / a->seg_chunks.
+size_t plan_split(m2::ScanArgs* a, int32_t nseq, int32_t max_seqlen, size_t* state_bytes) {
+    a->nseg = 1;
+    a->seg_chunks = 0;
+    *state_bytes = 0;
+    const int64_t pairs = static_cast<int64_t>(nseq) * a->H;
+    const int64_t target = 4LL * sm_count();
+    const int max_chunks = (max_seqlen + 127) / 128;
+    if (!m2::chunk_scan_tc_supported(*a) || pairs >= target || max_chunks < 2) return 0;
+    int nseg = static_cast<int>(std::min<int64_t>({(target + pairs - 1) / pairs, max_chunks, 32}));
+    const int seg_chunks = (max_chunks + nseg - 1) / nseg;
+    nseg = (max_chunks + seg_chunks - 1) / seg_chunks;
+    if (nseg <= 1) return 0;
+    a->nseg = nseg;
+    a->seg_chunks = seg_chunks;
+    *state_bytes = static_cast<size_t>(nseq) * nseg * a->H * a->P * a->N * sizeof(float);
+    return *state_bytes + static_cast<size_t>(nseq) * nseg * a->H * sizeof(float);
+}
+
 }  // namespace
 
 m2_status m2_chunk_scan(const m2_cache* c, const m2_ssm_params* ssm, int32_t batch, int32_t seqlen,
@@ -403,31 +426,19 @@ m2_status m2_chunk_scan_varlen(const m2_cache* c, const m2_ssm_params* ssm, int3
     a.seqlen = max_seqlen;
     a.total_tokens = total_tokens;
     const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-    // Split long sequences across CTAs when there are too few (sequence, head)
-    // pairs to fill the GPU: two waves of two CTAs per SM.
-    const int64_t pairs = static_cast<int64_t>(nseq) * a.H;
-    const int64_t target = 4LL * sm_count();
-    const int max_chunks = (max_seqlen + 127) / 128;
-    if (m2::chunk_scan_tc_supported(a) && pairs < target && max_chunks >= 2) {
-        int nseg = static_cast<int>(std::min<int64_t>({(target + pairs - 1) / pairs, max_chunks, 32}));
-        const int seg_chunks = (max_chunks + nseg - 1) / nseg;
-        nseg = (max_chunks + seg_chunks - 1) / seg_chunks;
-        if (nseg > 1) {
-            const size_t state_bytes = static_cast<size_t>(nseq) * nseg * a.H * a.P * a.N * sizeof(float);
-            const size_t decay_bytes = static_cast<size_t>(nseq) * nseg * a.H * sizeof(float);
-            void* scratch = nullptr;
-            if (cudaMallocAsync(&scratch, state_bytes + decay_bytes, cs) != cudaSuccess) {
-                cudaGetLastError();
-                return M2_ERR_OOM;
-            }
-            a.nseg = nseg;
-            a.seg_chunks = seg_chunks;
-            a.seg_state = static_cast<float*>(scratch);
-            a.seg_decay = reinterpret_cast<float*>(static_cast<char*>(scratch) + state_bytes);
-            const cudaError_t e = m2::launch_chunk_scan(a, cs);
-            const cudaError_t f = cudaFreeAsync(scratch, cs);
-            return from_cuda(e != cudaSuccess ? e : f);
+    size_t state_bytes = 0;
+    const size_t scratch_bytes = plan_split(&a, nseq, max_seqlen, &state_bytes);
+    if (scratch_bytes > 0) {
+        void* scratch = nullptr;
+        if (cudaMallocAsync(&scratch, scratch_bytes, cs) != cudaSuccess) {
+            cudaGetLastError();
+            return M2_ERR_OOM;
         }
+        a.seg_state = static_cast<float*>(scratch);
+        a.seg_decay = reinterpret_cast<float*>(static_cast<char*>(scratch) + state_bytes);
+        const cudaError_t e = m2::launch_chunk_scan(a, cs);
+        const cudaError_t f = cudaFreeAsync(scratch, cs);
+        return from_cuda(e != cudaSuccess ? e : f);
     }
     return from_cuda(m2::launch_chunk_scan(a, cs));
 }
