@@ -262,6 +262,34 @@ m2_status m2_chunk_scan_varlen(const m2_cache* cache, const m2_ssm_params* ssm, 
                                const int32_t* slot_idx, const uint8_t* has_initial_state,
                                m2_stream stream);
 
+/*
+ * m2_chunk_scan_varlen without any allocation, for callers that must not
+ * allocate device memory once they are running: a serving runtime that fixes
+ * its device memory budget at start-up (the fixed-size state allocator of the
+ * Nemotron-H-8B-Base-8K record) and must not fail a step on an allocation, or
+ * a process whose stream-ordered memory pool is unavailable. Same arguments,
+ * results and split plan as m2_chunk_scan_varlen (bit for bit); the scratch of
+ * a split is a file-scope device array of 40 MiB, enough for every split plan
+ * on a 148-SM B200 (P = 64, N = 128). A plan that needs more returns
+ * M2_ERR_UNSUPPORTED before launching. Nothing in the array needs clearing:
+ * every slot the scan pass reads is written earlier in the same call.
+ *   - The first call on a device looks up the array's address with
+ *     cudaGetSymbolAddress (once per device; its error is returned as
+ *     M2_ERR_CUDA) and may load the module that holds it: make that first call
+ *     before any stream capture begins on that device.
+ *   - All calls on a device share the one array: two calls whose executions
+ *     overlap (other streams, other host threads) race on it and corrupt each
+ *     other's results. Serialise them, e.g. on one stream.
+ * Without a split the call uses no scratch at all.
+ */
+m2_status m2_chunk_scan_varlen_static(const m2_cache* cache, const m2_ssm_params* ssm, int32_t nseq,
+                                      const int32_t* cu_seqlens, int64_t total_tokens,
+                                      int32_t max_seqlen, int32_t chunk_size, const void* xBC,
+                                      int32_t xBC_dtype, int64_t xBC_row_stride, const void* dt,
+                                      int64_t dt_row_stride, const void* z, int64_t z_row_stride,
+                                      void* y, int64_t y_row_stride, const int32_t* slot_idx,
+                                      const uint8_t* has_initial_state, m2_stream stream);
+
 /* Debug/test path: synchronises `stream`, copies the cache's error word to
  * *out_code (0 or an m2_status value) and clears it. Not for hot loops. */
 m2_status m2_get_device_error(const m2_cache* cache, m2_stream stream, int32_t* out_code);

@@ -106,6 +106,9 @@ SIGNATURES = {
     "m2_chunk_scan_varlen": (_I32, [ctypes.POINTER(m2_cache), ctypes.POINTER(m2_ssm_params), _I32, _P,
                                     _I64, _I32, _I32, _P, _I32, _I64, _P, _I64, _P, _I64, _P, _I64,
                                     _P, _P, _P]),
+    "m2_chunk_scan_varlen_static": (_I32, [ctypes.POINTER(m2_cache), ctypes.POINTER(m2_ssm_params), _I32,
+                                           _P, _I64, _I32, _I32, _P, _I32, _I64, _P, _I64, _P, _I64,
+                                           _P, _I64, _P, _P, _P]),
     "m2_get_device_error": (_I32, [ctypes.POINTER(m2_cache), _P, ctypes.POINTER(_I32)]),
     "m2_status_string": (ctypes.c_char_p, [_I32]),
     "m2_version": (ctypes.c_char_p, []),
@@ -354,11 +357,12 @@ def chunk_scan_varlen(cache: Cache, ssm: SSMParams, xBC: torch.Tensor, dt: torch
                       cu_seqlens: torch.Tensor, slot_idx: torch.Tensor, max_seqlen: Optional[int] = None,
                       z: Optional[torch.Tensor] = None, chunk_size: int = 128,
                       has_initial_state: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
-                      stream: Optional[int] = None) -> torch.Tensor:
+                      stream: Optional[int] = None, static_scratch: bool = False) -> torch.Tensor:
     """Prefill scan over sequences packed back to back: xBC [total_tokens, conv_dim]
     (post-conv), dt [total_tokens, H], cu_seqlens [nseq+1] int32 on the device.
     ``max_seqlen`` plans the split of long sequences; when None it is read from
-    cu_seqlens (a device-to-host copy: pass it explicitly under graph capture)."""
+    cu_seqlens (a device-to-host copy). ``static_scratch`` calls
+    m2_chunk_scan_varlen_static (no allocation; calls must not overlap)."""
     sh = cache.shape
     total = xBC.shape[0]
     nseq = cu_seqlens.numel() - 1
@@ -369,10 +373,11 @@ def chunk_scan_varlen(cache: Cache, ssm: SSMParams, xBC: torch.Tensor, dt: torch
     if y is None:
         y = torch.empty((total, sh.H * sh.P), dtype=torch_dtype(sh.act_dtype), device=xBC.device)
     sp = ssm.c()
-    st = lib().m2_chunk_scan_varlen(
+    fn = lib().m2_chunk_scan_varlen_static if static_scratch else lib().m2_chunk_scan_varlen
+    st = fn(
         ctypes.byref(cache.c), ctypes.byref(sp), nseq, cu_seqlens.data_ptr(), total, max_seqlen,
         chunk_size, xBC.data_ptr(), _dtype_code(xBC.dtype), xBC.stride(0), dt.data_ptr(), dt.stride(0),
         _ptr(z), z.stride(0) if z is not None else 0, y.data_ptr(), y.stride(0), slot_idx.data_ptr(),
         _ptr(has_initial_state), _stream_ptr() if stream is None else stream)
-    _check(st, "m2_chunk_scan_varlen")
+    _check(st, "m2_chunk_scan_varlen_static" if static_scratch else "m2_chunk_scan_varlen")
     return y

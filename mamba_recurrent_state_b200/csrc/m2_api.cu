@@ -443,6 +443,41 @@ m2_status m2_chunk_scan_varlen(const m2_cache* c, const m2_ssm_params* ssm, int3
     return from_cuda(m2::launch_chunk_scan(a, cs));
 }
 
+m2_status m2_chunk_scan_varlen_static(const m2_cache* c, const m2_ssm_params* ssm, int32_t nseq,
+                                      const int32_t* cu_seqlens, int64_t total_tokens, int32_t max_seqlen,
+                                      int32_t chunk_size, const void* xBC, int32_t xBC_dtype,
+                                      int64_t xBC_row_stride, const void* dt, int64_t dt_row_stride,
+                                      const void* z, int64_t z_row_stride, void* y, int64_t y_row_stride,
+                                      const int32_t* slot_idx, const uint8_t* has_initial_state,
+                                      m2_stream stream) {
+    if (nseq < 0 || total_tokens < 0 || max_seqlen < 0) return M2_ERR_INVALID_ARG;
+    if (total_tokens > INT32_MAX) return M2_ERR_UNSUPPORTED;
+    if (nseq == 0 || total_tokens == 0) {
+        const m2_status st = cache_status(c);
+        return st != M2_OK ? st : (ssm && chunk_size > 0 ? M2_OK : M2_ERR_INVALID_ARG);
+    }
+    if (!cu_seqlens) return M2_ERR_INVALID_ARG;
+    m2::ScanArgs a{};
+    const m2_status st = scan_args(c, ssm, nseq, chunk_size, xBC, xBC_dtype, xBC_row_stride, dt, dt_row_stride,
+                                   z, z_row_stride, y, y_row_stride, slot_idx, has_initial_state, stream, &a);
+    if (st != M2_OK) return st;
+    a.cu_seqlens = cu_seqlens;
+    a.seqlen = max_seqlen;
+    a.total_tokens = total_tokens;
+    size_t state_bytes = 0;
+    const size_t need = plan_split(&a, nseq, max_seqlen, &state_bytes);
+    if (need > 0) {  // the same plan as m2_chunk_scan_varlen, on the fixed array
+        void* scratch = nullptr;
+        size_t capacity = 0;
+        const cudaError_t e = m2::static_scan_scratch(&scratch, &capacity);
+        if (e != cudaSuccess) return from_cuda(e);
+        if (need > capacity) return M2_ERR_UNSUPPORTED;
+        a.seg_state = static_cast<float*>(scratch);
+        a.seg_decay = reinterpret_cast<float*>(static_cast<char*>(scratch) + state_bytes);
+    }
+    return from_cuda(m2::launch_chunk_scan(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 m2_status m2_get_device_error(const m2_cache* c, m2_stream stream, int32_t* out_code) {
     if (!c || !out_code) return M2_ERR_INVALID_ARG;
     *out_code = 0;

@@ -136,6 +136,9 @@ cudaError_t launch_state_update(const StateUpdateArgs& a, const DecodePlan& plan
 cudaError_t launch_conv1d_update(const ConvArgs& a, cudaStream_t stream);
 cudaError_t launch_zero_slots(const ZeroArgs& a, cudaStream_t stream);
 m2_status plan_chunk_scan(int H, int P, int N, int G, int chunk);
+// Address and size of the fixed scratch array of m2_chunk_scan_varlen_static
+// on the current device (looked up once per device with cudaGetSymbolAddress).
+cudaError_t static_scan_scratch(void** ptr, size_t* bytes);
 cudaError_t launch_chunk_scan(const ScanArgs& a, cudaStream_t stream);
 // Tensor-core (tcgen05) scan: bf16 state, activations and xBC, P = 64, N = 128.
 bool chunk_scan_tc_supported(const ScanArgs& a);

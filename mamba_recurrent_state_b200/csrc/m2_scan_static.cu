@@ -1,0 +1,47 @@
+// m2_scan_static.cu -- the fixed device scratch of m2_chunk_scan_varlen_static.
+//
+// A split variable-length scan (vllm.cpp issue #1311 "NemotronH runs the
+// PREFILL mamba kernels at decode", section "The divergence": the chunk scan
+// at prefill) keeps one fp32 P x N state per (sequence, segment, head) plus one
+// decay each between its passes. This translation unit holds that scratch as
+// a file-scope device array, so the entry point that uses it allocates
+// nothing. The array lives in its own module: it is only loaded (and its
+// device memory only reserved) on a device where the static entry point runs.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "m2_internal.cuh"
+
+namespace m2 {
+namespace {
+
+// The largest split plan on a 148-SM B200 keeps fewer than 2 x 4 x 148
+// (sequence, segment, head) states of 32 KB (P = 64, N = 128): under 37 MiB.
+constexpr size_t kStaticScanScratchBytes = size_t{40} << 20;
+
+__device__ __align__(256) unsigned char g_static_scan_scratch[kStaticScanScratchBytes];
+
+}  // namespace
+
+cudaError_t static_scan_scratch(void** ptr, size_t* bytes) {
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static void* addr[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_static_scan_scratch);
+        if (e != cudaSuccess) return e;
+        addr[dev] = p;
+    }
+    *ptr = addr[dev];
+    *bytes = kStaticScanScratchBytes;
+    return cudaSuccess;
+}
+
+}  // namespace m2
