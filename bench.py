@@ -57,9 +57,10 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--l2", choices=["rotate", "flush"], default="rotate",
                     help="rotate: disjoint slot sets, back to back; flush: 512 MiB write before each step")
-    ap.add_argument("--sections", default="decode,prefill,stack48",
+    ap.add_argument("--sections", default="decode,prefill,longprompt,stack48",
                     help="comma list: decode (the headline, always run), prefill (workload 4: "
-                         "prefill conv and tensor-core scan), stack48 (workload 2: 48-layer token)")
+                         "prefill conv and tensor-core scan), longprompt (one 16K-token prompt: "
+                         "conv and varlen scan), stack48 (workload 2: 48-layer token)")
     return ap.parse_args()
 
 
@@ -357,6 +358,52 @@ def measure_prefill(flush, peak_gbs: float, peak_tflops: float, reps: int = 10) 
     }
 
 
+def measure_longprompt(flush, peak_gbs: float, reps: int = 10, T: int = 16384) -> dict:
+    """One long prompt (16384 tokens, the long-prompt regime of mixed serving)
+    through the Nemotron-H layer: the prefill conv (fp16 post-conv buffer),
+    then the variable-length scan. Its 128 (sequence, head) pairs run one CTA
+    per head: a split into segments does not pay at this head count."""
+    import torch
+    import mamba_recurrent_state_b200 as m2
+    import m2synth as S
+    from m2synth import torch_inputs as TI
+    from m2synth import workloads as W
+    w = W.Workload(405, "longprompt", 128, 64, 128, 8, 4, S.BF16, S.BF16, 4, 1, seqlen=T, chunk=128)
+    shape = m2.Shape(w.H, w.P, w.N, w.G, w.K, w.state_dtype, w.act_dtype)
+    cache = m2.Cache(shape, w.num_slots)
+    t = TI.layer_tensors(w)
+    ssm = m2.SSMParams(t["A_log"], t["dt_bias"], t["D"])
+    conv = m2.ConvParams(t["conv_w"], t["conv_b"], 1)
+    d = TI.step_tensors(w, 0, rows=T)
+    xr = d["xBC"].view(1, T, -1)
+    xp = torch.empty(xr.shape, dtype=torch.float16, device="cuda")
+    y = torch.empty((T, w.H * w.P), dtype=torch.bfloat16, device="cuda")
+    cu = torch.tensor([0, T], dtype=torch.int32, device="cuda")
+    slots = t["slots"][:1]
+
+    def conv_step():
+        m2.conv1d_update(cache, conv, xr, slots, out=xp)
+
+    def scan_step():
+        m2.chunk_scan_varlen(cache, ssm, xp.view(T, -1), d["dt"], cu, slots, max_seqlen=T, z=d["z"], y=y)
+
+    for _ in range(3):
+        conv_step()
+        scan_step()
+    conv_us = statistics.median(_time_us(conv_step, flush, reps))
+    scan_us = statistics.median(_time_us(scan_step, flush, reps))
+    if cache.device_error() != 0:
+        raise RuntimeError("device error word set during the long-prompt benchmark")
+    hp, cd = w.H * w.P, w.conv_dim
+    scan_bytes = T * (cd + w.H + hp + hp) * 2 + w.H * w.P * w.N * 2
+    return {
+        "workload": f"one {T}-token prompt, Nemotron-H layer, bf16, fp16 post-conv buffer",
+        "conv_us": conv_us, "scan_us": scan_us, "scan_bytes": scan_bytes,
+        "scan_GBs": scan_bytes / scan_us / 1e3, "scan_frac_hbm": scan_bytes / scan_us / 1e3 / peak_gbs,
+        "tokens_per_s": T / (conv_us + scan_us) * 1e6,
+    }
+
+
 def measure_stack48(flush, reps: int = 10) -> dict:
     """Workload 2: one decode token for 384 sequences through 48 layers
     (36 GiB of bf16 state), one CUDA graph of 48 fused launches per token."""
@@ -543,6 +590,8 @@ def run_ours(args, world, rank, local):
         tpeak, tkind = measured_tensor_peak()
         line["prefill"] = measure_prefill(flush, peak, tpeak)
         line["prefill"]["tensor_peak"] = f"{tpeak} TFLOP/s ({tkind} bf16_tflops)"
+    if "longprompt" in sections:
+        line["longprompt"] = measure_longprompt(flush, peak)
     if "stack48" in sections:
         line["stack48"] = measure_stack48(flush)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

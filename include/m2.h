@@ -243,16 +243,17 @@ m2_status m2_chunk_scan(const m2_cache* cache, const m2_ssm_params* ssm, int32_t
  *   dt            [total_tokens, H] act_dtype
  *   z, y          [total_tokens, H*P] act_dtype (z may be NULL)
  * Split sequences: on the tensor-core path (bf16 state and activations,
- * P = 64, N = 128), when nseq * H (sequence, head) pairs are too few to fill
- * the GPU (fewer than four per SM), each sequence is cut into segments of
- * whole 128-token chunks that run in parallel: a first pass stores every
- * segment's final state from a zero start and its total decay, a combine pass
- * carries the states across segments in fp32 (the recurrence is linear in the
- * state), and the scan pass runs each segment from its carried state. The
- * scratch, nseq * segments * H * P * N * 4 bytes plus the decays, is taken with
- * cudaMallocAsync and returned with cudaFreeAsync on `stream` (both
- * stream-ordered and graph-capturable); M2_ERR_OOM if it cannot be had.
- * Without a split the call allocates nothing.
+ * P = 64, N = 128), when the nseq * H (sequence, head) pairs leave room for at
+ * least three segments per pair at one CTA per SM (nseq * H * 3 <= SMs), each
+ * sequence is cut into segments of whole 128-token chunks that run in
+ * parallel: a first pass stores every segment's final state from a zero start
+ * and its total decay, a combine pass carries the states across segments in
+ * fp32 (the recurrence is linear in the state), and the scan pass runs each
+ * segment from its carried state. The scratch (at most one 32 KB state and
+ * one decay per SM) is allocated stream-ordered on `stream` from a memory pool
+ * the library creates once per device and that keeps its memory for reuse,
+ * then freed stream-ordered; M2_ERR_OOM if it cannot be had. Without a split
+ * the call allocates nothing.
  */
 m2_status m2_chunk_scan_varlen(const m2_cache* cache, const m2_ssm_params* ssm, int32_t nseq,
                                const int32_t* cu_seqlens, int64_t total_tokens, int32_t max_seqlen,
@@ -269,9 +270,9 @@ m2_status m2_chunk_scan_varlen(const m2_cache* cache, const m2_ssm_params* ssm, 
  * Nemotron-H-8B-Base-8K record) and must not fail a step on an allocation, or
  * a process whose stream-ordered memory pool is unavailable. Same arguments,
  * results and split plan as m2_chunk_scan_varlen (bit for bit); the scratch of
- * a split is a file-scope device array of 40 MiB, enough for every split plan
- * on a 148-SM B200 (P = 64, N = 128). A plan that needs more returns
- * M2_ERR_UNSUPPORTED before launching. Nothing in the array needs clearing:
+ * a split is a file-scope device array of 16 MiB, enough for every split plan
+ * on GPUs of up to 511 SMs (one 32 KB state and one decay per SM at most). A
+ * plan that needs more returns M2_ERR_UNSUPPORTED before launching. Nothing in the array needs clearing:
  * every slot the scan pass reads is written earlier in the same call.
  *   - The first call on a device looks up the array's address with
  *     cudaGetSymbolAddress (once per device; its error is returned as

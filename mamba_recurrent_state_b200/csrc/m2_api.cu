@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include <cstdlib>
 #include <cstring>
@@ -352,6 +353,40 @@ m2_status scan_args(const m2_cache* c, const m2_ssm_params* ssm, int32_t batch, 
     return M2_OK;
 }
 
+// The split scan's stream-ordered memory pool on the current device, created
+// once per device. It keeps freed memory (release threshold: never), so after
+// the first split call on a device the scratch costs no driver allocation;
+// the device's default pool, whose memory goes back to the driver at every
+// synchronisation, cost up to milliseconds per call.
+cudaError_t scratch_pool(cudaMemPool_t* out) {
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static cudaMemPool_t pools[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (pools[dev] == nullptr) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t p = nullptr;
+        e = cudaMemPoolCreate(&p, &props);
+        if (e != cudaSuccess) return e;
+        uint64_t keep = UINT64_MAX;
+        e = cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep);
+        if (e != cudaSuccess) {
+            cudaMemPoolDestroy(p);
+            return e;
+        }
+        pools[dev] = p;
+    }
+    *out = pools[dev];
+    return cudaSuccess;
+}
+
 int sm_count() {
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -360,20 +395,24 @@ int sm_count() {
     return n > 0 ? n : 148;
 }
 
-// Split plan of a variable-length scan: when the (sequence, head) pairs are
-// too few to fill the GPU (two waves of two CTAs per SM) and the tensor-core
-// path applies, sequences are cut into segments of seg_chunks 128-token
-// chunks, nseg per sequence in the grid. Returns the scratch bytes (state
-// slots, then decays; 0 without a split) and sets a->nseg / a->seg_chunks.
+// Split plan of a variable-length scan (tensor-core path). The scan of a
+// chunk is latency-bound inside its CTA: on B200 a CTA alone on its SM takes
+// about 5.6 us per 128-token chunk, two CTAs sharing an SM about 8.7 us each,
+// and the summary pass of a split about 4.9 us per chunk. Splitting therefore
+// only pays when whole extra SMs can be put to work: sequences are cut into
+// nseg segments so that the (sequence, segment, head) CTAs of the scan pass
+// are at most one per SM, and only when at least three segments fit. Returns
+// the scratch bytes (state slots, then decays; 0 without a split) and sets
+// a->nseg / a->seg_chunks.
 size_t plan_split(m2::ScanArgs* a, int32_t nseq, int32_t max_seqlen, size_t* state_bytes) {
     a->nseg = 1;
     a->seg_chunks = 0;
     *state_bytes = 0;
     const int64_t pairs = static_cast<int64_t>(nseq) * a->H;
-    const int64_t target = 4LL * sm_count();
     const int max_chunks = (max_seqlen + 127) / 128;
-    if (!m2::chunk_scan_tc_supported(*a) || pairs >= target || max_chunks < 2) return 0;
-    int nseg = static_cast<int>(std::min<int64_t>({(target + pairs - 1) / pairs, max_chunks, 32}));
+    if (!m2::chunk_scan_tc_supported(*a) || pairs <= 0 || max_chunks < 3) return 0;
+    int nseg = static_cast<int>(std::min<int64_t>({sm_count() / pairs, max_chunks, 64}));
+    if (nseg < 3) return 0;
     const int seg_chunks = (max_chunks + nseg - 1) / nseg;
     nseg = (max_chunks + seg_chunks - 1) / seg_chunks;
     if (nseg <= 1) return 0;
@@ -429,8 +468,11 @@ m2_status m2_chunk_scan_varlen(const m2_cache* c, const m2_ssm_params* ssm, int3
     size_t state_bytes = 0;
     const size_t scratch_bytes = plan_split(&a, nseq, max_seqlen, &state_bytes);
     if (scratch_bytes > 0) {
+        cudaMemPool_t pool = nullptr;
+        const cudaError_t pe = scratch_pool(&pool);
+        if (pe != cudaSuccess) return from_cuda(pe);
         void* scratch = nullptr;
-        if (cudaMallocAsync(&scratch, scratch_bytes, cs) != cudaSuccess) {
+        if (cudaMallocFromPoolAsync(&scratch, scratch_bytes, pool, cs) != cudaSuccess) {
             cudaGetLastError();
             return M2_ERR_OOM;
         }

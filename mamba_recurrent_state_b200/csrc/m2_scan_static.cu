@@ -16,9 +16,10 @@
 namespace m2 {
 namespace {
 
-// The largest split plan on a 148-SM B200 keeps fewer than 2 x 4 x 148
-// (sequence, segment, head) states of 32 KB (P = 64, N = 128): under 37 MiB.
-constexpr size_t kStaticScanScratchBytes = size_t{40} << 20;
+// A split plan keeps at most one (sequence, segment, head) state of 32 KB
+// (P = 64, N = 128) and one decay per SM: 4.6 MiB on a 148-SM B200; 16 MiB
+// covers GPUs of up to 511 SMs.
+constexpr size_t kStaticScanScratchBytes = size_t{16} << 20;
 
 __device__ __align__(256) unsigned char g_static_scan_scratch[kStaticScanScratchBytes];
 

@@ -4,10 +4,11 @@ sequence is its own run of T sequential updates from its slot's state (or
 zero), the working state unrounded until the end.
 
 Cases: ragged lengths with a padding row, an empty sequence and mixed initial
-states; few long sequences, which the call splits into segments (first pass,
-fp32 combine, scan pass); the Nemotron-H layer with one 4096-token prompt,
-checked on sampled heads; a sequence longer than the max_seqlen hint; and the
-split result against the unsplit fixed-length scan of the same input.
+states (6 x 8 pairs: split into 3 segments); few long sequences, which the call
+splits into segments (first pass, fp32 combine, scan pass); the Nemotron-H
+layer with one 4096-token prompt, checked on sampled heads; a sequence longer
+than the max_seqlen hint; and the split result against the unsplit
+fixed-length scan of the same input.
 """
 
 import numpy as np
@@ -118,8 +119,8 @@ def test_varlen_ragged_mixed():
 
 def test_varlen_split_long_sequences():
     """Two long sequences over 8 heads: 16 (sequence, head) pairs, so the call
-    splits each sequence into one-chunk segments (summary pass, fp32 combine,
-    scan pass), with and without an initial state."""
+    splits each sequence into segments of three chunks (summary pass, fp32
+    combine, scan pass), with and without an initial state."""
     w = wl(401, batch=2)
     run_case(w, lengths=[1000, 2500], slot_list=[6, 1], init_list=[1, 0])
 
@@ -133,8 +134,9 @@ def test_varlen_split_longer_than_hint():
 
 def test_nemotron_h_one_long_prompt_sampled_heads():
     """Nemotron-H layer (H = 128, G = 8), one 4096-token prompt from the slot's
-    state: 128 (sequence, head) pairs, split into segments; heads 0, 77 and 127
-    are followed by the oracle."""
+    state through the variable-length call (128 (sequence, head) pairs: one
+    CTA per head, no split on a 148-SM GPU); heads 0, 77 and 127 are followed
+    by the oracle."""
     w = W.Workload(403, "varlen_nemotron", 128, 64, 128, 8, 4, S.BF16, S.BF16, 4, 1, seqlen=4096,
                    chunk=128)
     run_case(w, lengths=[4096], slot_list=[2], init_list=[1], heads=[0, 77, 127])
