@@ -72,6 +72,8 @@ class Oracle:
         L.m2o_ssm_step.argtypes = [ctypes.c_int] * 4 + [_dp, ctypes.c_int] + [_dp] * 7
         L.m2o_ssm_scan.restype = None
         L.m2o_ssm_scan.argtypes = [ctypes.c_int] * 5 + [_dp, ctypes.c_int] + [_dp] * 7
+        L.m2o_group_rmsnorm.restype = None
+        L.m2o_group_rmsnorm.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_double, _dp, _dp, _dp]
 
     @property
     def tag(self) -> str:
@@ -162,6 +164,15 @@ class Oracle:
                               self._p(self._f64(A_log)), self._p(self._f64(D)), self._p(zz),
                               self._p(y))
         return y
+
+    def group_rmsnorm(self, v, G: int, eps: float, w) -> np.ndarray:
+        """Gated RMSNorm of one row: v [H*P] is the gated y; groups of H*P/G
+        consecutive channels; w [H*P] the norm weight. Returns out [H*P]."""
+        v = self._f64(v).reshape(-1)
+        w = self._f64(w).reshape(-1)
+        out = np.empty_like(v)
+        self.lib.m2o_group_rmsnorm(int(v.size), int(G), float(eps), self._p(v), self._p(w), self._p(out))
+        return out
 
 
 _DEFAULT: Oracle | None = None

@@ -29,6 +29,10 @@
  *   chunked prefill scan -- must land on the same state as T sequential
  *     selective_state_update steps; the definition used here is exactly that
  *     loop, with the working state kept unrounded across the T tokens.
+ *   gated RMSNorm -- the mixer's `norm` tensor (Nemotron-H-8B-Base-8K model
+ *     record, the tensor list of the Mamba-2 mixer layers): the gated y is
+ *     normalised by its root mean square over groups of H*P/G consecutive
+ *     channels and scaled by the norm weight.
  *
  * Shapes follow the Nemotron-H-8B-Base-8K model record (ssm_state_size N,
  * mamba_head_dim P, mamba_num_heads H, n_groups G): the state of one sequence
@@ -271,6 +275,39 @@ void m2o_ssm_scan(int H, int P, int N, int G, int T, double* state, int round_mo
     for (size_t i = 0; i < n; ++i) state[i] = m2o_round(state[i], round_mode);
 }
 
+/*
+ * Gated RMSNorm of one row of mixer output. v is the gated y (y * silu(z), as
+ * m2o_ssm_step returns it: the gate comes before the norm); the HP channels
+ * split into G groups of L = HP/G consecutive channels, and in each group
+ *     ms     = (1/L) * sum_c v[c]^2
+ *     out[c] = v[c] / sqrt(ms + eps) * w[c]
+ */
+void m2o_group_rmsnorm(int HP, int G, double eps, const double* v, const double* w, double* out) {
+#ifdef M2O_MUTANT_NORM_WHOLE_ROW
+    G = 1;
+#endif
+    const int L = HP / G;
+    for (int gi = 0; gi < G; ++gi) {
+        const double* vg = v + (size_t)gi * L;
+        double ss = 0.0;
+        for (int c = 0; c < L; ++c) ss += vg[c] * vg[c];
+        const double ms = ss / L;
+#ifdef M2O_MUTANT_NORM_EPS_OUTSIDE
+        const double denom = sqrt(ms) + eps;
+#else
+        const double denom = sqrt(ms + eps);
+#endif
+        for (int c = 0; c < L; ++c) {
+            const size_t i = (size_t)gi * L + c;
+#ifdef M2O_MUTANT_NORM_NO_WEIGHT
+            out[i] = v[i] / denom;
+#else
+            out[i] = v[i] / denom * w[i];
+#endif
+        }
+    }
+}
+
 /* Version tag so the Python side can tell a mutant build from the default. */
 const char* m2o_build_tag(void) {
 #if defined(M2O_MUTANT_CONV_FLIP)
@@ -297,6 +334,12 @@ const char* m2o_build_tag(void) {
     return "mutant:swap_bc";
 #elif defined(M2O_MUTANT_DT_NO_BIAS)
     return "mutant:dt_no_bias";
+#elif defined(M2O_MUTANT_NORM_WHOLE_ROW)
+    return "mutant:norm_whole_row";
+#elif defined(M2O_MUTANT_NORM_EPS_OUTSIDE)
+    return "mutant:norm_eps_outside";
+#elif defined(M2O_MUTANT_NORM_NO_WEIGHT)
+    return "mutant:norm_no_weight";
 #else
     return "oracle";
 #endif

@@ -443,6 +443,66 @@ def pin_state_rounding_on_store(orc: O.Oracle) -> None:
             assert np.array_equal(S_r.ravel(), [_nearest_bf16_brute(v) for v in S_exact.ravel()])
 
 
+# ------------------------------------------------------------ gated RMSNorm
+
+def pin_rmsnorm_hand(orc: O.Oracle) -> None:
+    """Hand-worked example, tests/golden/group_rmsnorm_hand.txt (two groups,
+    eps = 0 and eps = 1, non-unit weights)."""
+    g = read_golden("group_rmsnorm_hand.txt")
+    for eps, tag in ((0.0, "eps0"), (1.0, "eps1")):
+        out = orc.group_rmsnorm(g["v"], int(g["G"]), eps, g["w"])
+        want = g[f"{tag}_coef"] * np.sqrt(g[f"{tag}_root"])
+        assert np.allclose(out, want, rtol=1e-14, atol=0), (tag, out, want)
+
+
+def pin_rmsnorm_unit_rms(orc: O.Oracle) -> None:
+    """With unit weights and eps = 0 every group of the output has root mean
+    square exactly 1 and is a positive multiple of the input group."""
+    rng = _rng(71)
+    G, L = 4, 16
+    v = rng.normal(size=G * L) * rng.uniform(0.1, 10.0, size=G).repeat(L)
+    out = orc.group_rmsnorm(v, G, 0.0, np.ones(G * L))
+    for gi in range(G):
+        o, x = out[gi * L:(gi + 1) * L], v[gi * L:(gi + 1) * L]
+        assert abs(np.mean(o * o) - 1.0) < 1e-12
+        ratio = o / x
+        assert np.all(ratio > 0) and np.ptp(ratio) < 1e-12 * np.max(ratio)
+
+
+def pin_rmsnorm_scale_sign(orc: O.Oracle) -> None:
+    """eps = 0: the output does not change when a row is scaled by a positive
+    factor, and changes sign with the row."""
+    rng = _rng(72)
+    G, L = 2, 8
+    v = rng.normal(size=G * L)
+    w = rng.normal(size=G * L)
+    base = orc.group_rmsnorm(v, G, 0.0, w)
+    assert np.allclose(orc.group_rmsnorm(2.5 * v, G, 0.0, w), base, rtol=1e-13, atol=0)
+    assert np.array_equal(orc.group_rmsnorm(-v, G, 0.0, w), -base)
+
+
+def pin_rmsnorm_group_partition(orc: O.Oracle) -> None:
+    """A G-group row is G independent one-group rows, bit for bit."""
+    rng = _rng(73)
+    G, L = 4, 8
+    v = rng.normal(size=G * L)
+    w = rng.normal(size=G * L)
+    full = orc.group_rmsnorm(v, G, 1e-5, w)
+    for gi in range(G):
+        sl = slice(gi * L, (gi + 1) * L)
+        assert np.array_equal(full[sl], orc.group_rmsnorm(v[sl], 1, 1e-5, w[sl]))
+
+
+def pin_rmsnorm_eps_dominates(orc: O.Oracle) -> None:
+    """When eps is far above the mean square, out = v * w / sqrt(eps)."""
+    rng = _rng(74)
+    G, L = 2, 8
+    v = 1e-9 * rng.normal(size=G * L)
+    w = rng.normal(size=G * L)
+    out = orc.group_rmsnorm(v, G, 4.0, w)
+    assert np.allclose(out, v * w / 2.0, rtol=1e-9, atol=0)
+
+
 ALL_PINS = [
     pin_round_bf16_brute,
     pin_round_f16_brute,
@@ -461,4 +521,9 @@ ALL_PINS = [
     pin_group_partition,
     pin_scan_is_steps,
     pin_state_rounding_on_store,
+    pin_rmsnorm_hand,
+    pin_rmsnorm_unit_rms,
+    pin_rmsnorm_scale_sign,
+    pin_rmsnorm_group_partition,
+    pin_rmsnorm_eps_dominates,
 ]

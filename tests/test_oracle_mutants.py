@@ -4,7 +4,9 @@ The oracle source carries compile-time switches that each plant one plausible
 mistake (a flipped conv kernel, a wrong head->group map, a wrong sign of A, a
 dropped dt on the input term, y read from the old state, y read with B instead
 of C, a dropped D skip, truncating bf16 rounding, a sigmoid gate, no conv
-roll, swapped B/C halves, dt without its bias). Each mutant is built on the
+roll, swapped B/C halves, dt without its bias; for the gated RMSNorm: one
+group over the whole row, eps outside the square root, no weight). Each
+mutant is built on the
 CPU into a temporary directory and run against the same pins as the default
 build; the test asserts that some pin rejects it.
 """
@@ -29,6 +31,9 @@ MUTANTS = [
     "M2O_MUTANT_NO_ROLL",
     "M2O_MUTANT_SWAP_BC",
     "M2O_MUTANT_DT_NO_BIAS",
+    "M2O_MUTANT_NORM_WHOLE_ROW",
+    "M2O_MUTANT_NORM_EPS_OUTSIDE",
+    "M2O_MUTANT_NORM_NO_WEIGHT",
 ]
 
 
