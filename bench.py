@@ -57,8 +57,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--l2", choices=["rotate", "flush"], default="rotate",
                     help="rotate: disjoint slot sets, back to back; flush: 512 MiB write before each step")
-    ap.add_argument("--sections", default="decode,prefill,longprompt,stack48",
-                    help="comma list: decode (the headline, always run), prefill (workload 4: "
+    ap.add_argument("--sections", default="decode,norm,prefill,longprompt,stack48",
+                    help="comma list: decode (the headline, always run), norm (decode with the "
+                         "fused gated RMSNorm), prefill (workload 4: "
                          "prefill conv and tensor-core scan), longprompt (one 16K-token prompt: "
                          "conv and varlen scan), stack48 (workload 2: 48-layer token)")
     return ap.parse_args()
@@ -404,6 +405,52 @@ def measure_longprompt(flush, peak_gbs: float, reps: int = 10, T: int = 16384) -
     }
 
 
+def measure_decode_norm(peak_gbs: float, reps: int = 200) -> dict:
+    """The workload-1 decode step with the gated RMSNorm fused
+    (m2_state_update_norm), rotating the four disjoint slot sets back to back
+    like the headline loop, against the same loop without the norm."""
+    import torch
+    import mamba_recurrent_state_b200 as m2
+    from m2synth import torch_inputs as TI
+    from m2synth import workloads as W
+    w = W.WORKLOADS[1]
+    shape = m2.Shape(w.H, w.P, w.N, w.G, w.K, w.state_dtype, w.act_dtype)
+    cache = m2.Cache(shape, w.num_slots)
+    TI.fill_caches(w, cache.ssm, cache.conv)
+    t = TI.layer_tensors(w)
+    ssm = m2.SSMParams(t["A_log"], t["dt_bias"], t["D"])
+    conv = m2.ConvParams(t["conv_w"], t["conv_b"], 1)
+    norm = m2.NormParams(TI.to_torch(W.norm_weight(w), w.act_dtype), 1e-5)
+    sets = [torch.from_numpy(x).to("cuda") for x in W.slot_sets(w)]
+    inputs = [TI.step_tensors(w, s) for s in range(len(sets))]
+    y = torch.empty((w.batch, w.H * w.P), dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream()
+    out = {}
+    for tag, nrm in (("plain", None), ("norm", norm)):
+        def step(i):
+            inp = inputs[i % len(sets)]
+            m2.state_update(cache, ssm, inp["xBC"], inp["dt"], sets[i % len(sets)], z=inp["z"], conv=conv,
+                            y=y, norm=nrm)
+        for i in range(8):
+            step(i)
+        a = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+        b = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+        torch.cuda.synchronize()
+        for i in range(reps):
+            a[i].record(stream)
+            step(i)
+            b[i].record(stream)
+        torch.cuda.synchronize()
+        out[f"{tag}_us"] = statistics.median(x.elapsed_time(e) * 1e3 for x, e in zip(a, b))
+    if cache.device_error() != 0:
+        raise RuntimeError("device error word set during the norm benchmark")
+    bytes_ = W.bytes_per_unit(w) * w.batch + W.param_bytes_per_launch(w) + w.H * w.P * 2
+    out["norm_GBs"] = bytes_ / out["norm_us"] / 1e3
+    out["norm_frac_hbm"] = out["norm_GBs"] / peak_gbs
+    out["workload"] = "workload-1 decode step + fused gated RMSNorm (1024-channel groups, eps 1e-5)"
+    return out
+
+
 def measure_stack48(flush, reps: int = 10) -> dict:
     """Workload 2: one decode token for 384 sequences through 48 layers
     (36 GiB of bf16 state), one CUDA graph of 48 fused launches per token."""
@@ -590,6 +637,8 @@ def run_ours(args, world, rank, local):
         tpeak, tkind = measured_tensor_peak()
         line["prefill"] = measure_prefill(flush, peak, tpeak)
         line["prefill"]["tensor_peak"] = f"{tpeak} TFLOP/s ({tkind} bf16_tflops)"
+    if "norm" in sections:
+        line["decode_norm"] = measure_decode_norm(peak)
     if "longprompt" in sections:
         line["longprompt"] = measure_longprompt(flush, peak)
     if "stack48" in sections:

@@ -197,6 +197,32 @@ m2_status m2_state_update(const m2_cache* cache, const m2_ssm_params* ssm,
                           int64_t dt_row_stride, const void* z, int64_t z_row_stride, void* y,
                           int64_t y_row_stride, const int32_t* slot_idx, m2_stream stream);
 
+/* Gated RMSNorm applied to the decode output (the `norm` tensor of the
+ * Mamba-2 mixer in the Nemotron-H-8B-Base-8K record): weight [H*P] act_dtype
+ * (device, 16-byte aligned), eps >= 0. */
+typedef struct m2_norm_params {
+    const void* weight;
+    float eps;
+} m2_norm_params;
+
+/*
+ * m2_state_update with the gated RMSNorm fused into the same launch. The
+ * gated y, v = y * silu(z) (v = y when z is NULL), is normalised over each
+ * group of H*P/G consecutive channels (the heads of one SSM group):
+ *     out[c] = v[c] / sqrt(mean over the group of v^2 + eps) * weight[c]
+ * and out is written to y. The conv is always fused here (conv must be
+ * non-NULL; xBC is the raw row in act_dtype): the group's CTAs are the
+ * launch's thread-block cluster and exchange their partial sums of squares
+ * through distributed shared memory, so y makes no extra round trip. Other
+ * arguments, the state update and the conv cache as for m2_state_update.
+ * One launch, no scratch memory.
+ */
+m2_status m2_state_update_norm(const m2_cache* cache, const m2_ssm_params* ssm,
+                               const m2_conv_params* conv, const m2_norm_params* norm, int32_t batch,
+                               const void* xBC, int64_t xBC_row_stride, const void* dt,
+                               int64_t dt_row_stride, const void* z, int64_t z_row_stride, void* y,
+                               int64_t y_row_stride, const int32_t* slot_idx, m2_stream stream);
+
 /*
  * Chunked prefill scan (vllm.cpp issue, "The divergence": the chunk scan that
  * follows CausalConv1dFwd at prefill). For each row, runs `seqlen` tokens of

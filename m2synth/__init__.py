@@ -48,6 +48,7 @@ T_A_LOG = 5
 T_DT_BIAS = 6
 T_D = 7
 T_SLOTS = 8
+T_NORM_W = 9
 T_XBC = 10
 T_Z = 11
 T_DT = 12

@@ -30,7 +30,7 @@ from __future__ import annotations
 import dataclasses
 import numpy as np
 
-from . import (BF16, F32, T_A_LOG, T_CONV, T_CONV_B, T_CONV_W, T_D, T_DT, T_DT_BIAS,
+from . import (BF16, F32, T_A_LOG, T_CONV, T_CONV_B, T_CONV_W, T_D, T_DT, T_DT_BIAS, T_NORM_W,
                T_SLOTS, T_SSM, T_XBC, T_Z, config_seed, normal, normal_storage, permutation,
                stream_key, to_storage, uniform)
 
@@ -102,6 +102,11 @@ def layer_params(w: Workload, layer: int = 0) -> LayerParams:
     dt_bias = np.log(np.expm1(u)).astype(np.float32)
     D = normal(stream_key(s, T_D), 0, w.H, 0.0, 1.0).astype(np.float32)
     return LayerParams(conv_w, conv_b, A_log, dt_bias, D)
+
+
+def norm_weight(w: Workload, layer: int = 0) -> np.ndarray:
+    """Gated RMSNorm weight [H*P] in act storage form, ~N(1, 0.1)."""
+    return normal_storage(stream_key(w.seed(layer), T_NORM_W), 0, w.H * w.P, 1.0, 0.1, w.act_dtype)
 
 
 def slot_indices(w: Workload, layer: int = 0) -> np.ndarray:

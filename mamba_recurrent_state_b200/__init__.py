@@ -82,6 +82,10 @@ class m2_ssm_params(ctypes.Structure):
     _fields_ = [("A_log", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p), ("D", ctypes.c_void_p)]
 
 
+class m2_norm_params(ctypes.Structure):
+    _fields_ = [("weight", ctypes.c_void_p), ("eps", ctypes.c_float)]
+
+
 # exported symbols and their signatures (mirrors include/m2.h)
 _P = ctypes.c_void_p
 _I32 = ctypes.c_int32
@@ -101,6 +105,9 @@ SIGNATURES = {
     "m2_state_update": (_I32, [ctypes.POINTER(m2_cache), ctypes.POINTER(m2_ssm_params),
                                ctypes.POINTER(m2_conv_params), _I32, _P, _I32, _I64, _P, _I64,
                                _P, _I64, _P, _I64, _P, _P]),
+    "m2_state_update_norm": (_I32, [ctypes.POINTER(m2_cache), ctypes.POINTER(m2_ssm_params),
+                                    ctypes.POINTER(m2_conv_params), ctypes.POINTER(m2_norm_params), _I32,
+                                    _P, _I64, _P, _I64, _P, _I64, _P, _I64, _P, _P]),
     "m2_chunk_scan": (_I32, [ctypes.POINTER(m2_cache), ctypes.POINTER(m2_ssm_params), _I32, _I32,
                              _I32, _P, _I32, _I64, _P, _I64, _P, _I64, _P, _I64, _P, _P, _P]),
     "m2_chunk_scan_varlen": (_I32, [ctypes.POINTER(m2_cache), ctypes.POINTER(m2_ssm_params), _I32, _P,
@@ -287,15 +294,28 @@ class ConvParams:
         return m2_conv_params(self.weight.data_ptr(), _ptr(self.bias), self.activation)
 
 
+@dataclasses.dataclass
+class NormParams:
+    """Gated RMSNorm after the decode step: weight [H*P] (activation dtype), eps."""
+    weight: torch.Tensor
+    eps: float = 1e-5
+
+    def c(self) -> m2_norm_params:
+        if not self.weight.is_contiguous():
+            raise ValueError("norm weight must be contiguous [H*P]")
+        return m2_norm_params(self.weight.data_ptr(), float(self.eps))
+
+
 def state_update(cache: Cache, ssm: SSMParams, xBC: torch.Tensor, dt: torch.Tensor,
                  slot_idx: torch.Tensor, z: Optional[torch.Tensor] = None,
                  conv: Optional[ConvParams] = None, y: Optional[torch.Tensor] = None,
-                 stream: Optional[int] = None) -> torch.Tensor:
+                 stream: Optional[int] = None, norm: Optional[NormParams] = None) -> torch.Tensor:
     """One decode step for ``xBC.shape[0]`` rows, in place on ``cache``.
 
     With ``conv`` given, ``xBC`` is the raw row and the conv tap is fused;
-    otherwise ``xBC`` is post-conv (float32 or bfloat16). Returns y
-    [batch, H*P] in the activation dtype.
+    otherwise ``xBC`` is post-conv (float32 or bfloat16). With ``norm`` given
+    (requires ``conv``) the gated RMSNorm is fused too (m2_state_update_norm).
+    Returns y [batch, H*P] in the activation dtype.
     """
     sh = cache.shape
     batch = xBC.shape[0]
@@ -303,6 +323,17 @@ def state_update(cache: Cache, ssm: SSMParams, xBC: torch.Tensor, dt: torch.Tens
         y = torch.empty((batch, sh.H * sh.P), dtype=torch_dtype(sh.act_dtype), device=xBC.device)
     sp = ssm.c()
     cp = conv.c() if conv is not None else None
+    if norm is not None:
+        if cp is None:
+            raise ValueError("the fused gated RMSNorm needs the fused conv (conv=...)")
+        npar = norm.c()
+        st = lib().m2_state_update_norm(
+            ctypes.byref(cache.c), ctypes.byref(sp), ctypes.byref(cp), ctypes.byref(npar), batch,
+            xBC.data_ptr(), _row_stride(xBC), dt.data_ptr(), _row_stride(dt), _ptr(z),
+            _row_stride(z) if z is not None else 0, y.data_ptr(), _row_stride(y), slot_idx.data_ptr(),
+            _stream_ptr() if stream is None else stream)
+        _check(st, "m2_state_update_norm")
+        return y
     st = lib().m2_state_update(
         ctypes.byref(cache.c), ctypes.byref(sp), ctypes.byref(cp) if cp is not None else None,
         batch, xBC.data_ptr(), _dtype_code(xBC.dtype), _row_stride(xBC), dt.data_ptr(),

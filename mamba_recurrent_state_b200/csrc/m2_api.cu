@@ -228,10 +228,13 @@ m2_status m2_conv1d_update(const m2_cache* c, const m2_conv_params* conv, int32_
     return from_cuda(m2::launch_conv1d_update(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-m2_status m2_state_update(const m2_cache* c, const m2_ssm_params* ssm, const m2_conv_params* conv,
-                          int32_t batch, const void* xBC, int32_t xBC_dtype, int64_t xBC_row_stride,
-                          const void* dt, int64_t dt_row_stride, const void* z, int64_t z_row_stride,
-                          void* y, int64_t y_row_stride, const int32_t* slot_idx, m2_stream stream) {
+namespace {
+
+m2_status state_update_impl(const m2_cache* c, const m2_ssm_params* ssm, const m2_conv_params* conv,
+                            const m2_norm_params* norm, int32_t batch, const void* xBC, int32_t xBC_dtype,
+                            int64_t xBC_row_stride, const void* dt, int64_t dt_row_stride, const void* z,
+                            int64_t z_row_stride, void* y, int64_t y_row_stride, const int32_t* slot_idx,
+                            m2_stream stream) {
     const m2_status st = cache_status(c);
     if (st != M2_OK) return st;
     if (!ssm || !ssm->A_log || !ssm->dt_bias || !ssm->D || batch < 0 || !valid_buffer_dtype(xBC_dtype))
@@ -251,6 +254,10 @@ m2_status m2_state_update(const m2_cache* c, const m2_ssm_params* ssm, const m2_
         !stride_ok(y_row_stride, as, hp) || dt_row_stride < s.nheads)
         return M2_ERR_INVALID_ARG;
     if (z && (!aligned16(z) || !stride_ok(z_row_stride, as, hp))) return M2_ERR_INVALID_ARG;
+    if (norm) {  // the fused launch's group cluster carries the norm's reduction
+        if (!conv) return M2_ERR_UNSUPPORTED;
+        if (!norm->weight || !aligned16(norm->weight) || !(norm->eps >= 0.f)) return M2_ERR_INVALID_ARG;
+    }
     m2::DecodePlan plan;
     const m2_status ps = m2::plan_state_update(s.nheads, s.head_dim, s.d_state, s.ngroups,
                                                s.state_dtype == M2_BF16, conv != nullptr, &plan);
@@ -290,7 +297,31 @@ m2_status m2_state_update(const m2_cache* c, const m2_ssm_params* ssm, const m2_
     a.y = y;
     a.y_stride = y_row_stride;
     a.slot_idx = slot_idx;
+    a.norm_w = norm ? norm->weight : nullptr;
+    a.norm_eps = norm ? norm->eps : 0.f;
     return from_cuda(m2::launch_state_update(a, plan, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
+m2_status m2_state_update(const m2_cache* c, const m2_ssm_params* ssm, const m2_conv_params* conv,
+                          int32_t batch, const void* xBC, int32_t xBC_dtype, int64_t xBC_row_stride,
+                          const void* dt, int64_t dt_row_stride, const void* z, int64_t z_row_stride,
+                          void* y, int64_t y_row_stride, const int32_t* slot_idx, m2_stream stream) {
+    return state_update_impl(c, ssm, conv, nullptr, batch, xBC, xBC_dtype, xBC_row_stride, dt, dt_row_stride, z,
+                             z_row_stride, y, y_row_stride, slot_idx, stream);
+}
+
+m2_status m2_state_update_norm(const m2_cache* c, const m2_ssm_params* ssm, const m2_conv_params* conv,
+                               const m2_norm_params* norm, int32_t batch, const void* xBC,
+                               int64_t xBC_row_stride, const void* dt, int64_t dt_row_stride, const void* z,
+                               int64_t z_row_stride, void* y, int64_t y_row_stride, const int32_t* slot_idx,
+                               m2_stream stream) {
+    if (!norm || !conv) return M2_ERR_INVALID_ARG;
+    const m2_status st = cache_status(c);
+    if (st != M2_OK) return st;
+    return state_update_impl(c, ssm, conv, norm, batch, xBC, c->shape.act_dtype, xBC_row_stride, dt,
+                             dt_row_stride, z, z_row_stride, y, y_row_stride, slot_idx, stream);
 }
 
 namespace {

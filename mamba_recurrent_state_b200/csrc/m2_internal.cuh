@@ -56,6 +56,8 @@ struct StateUpdateArgs {
     void* y;
     int64_t y_stride;
     const int32_t* slot_idx;
+    const void* norm_w;  // gated RMSNorm weight [H*P] act dtype, or NULL (fused launches only)
+    float norm_eps;
 };
 
 struct ConvArgs {

@@ -67,6 +67,24 @@ __device__ __forceinline__ uint32_t cluster_rank() {
     asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
     return r;
 }
+__device__ __forceinline__ uint32_t cluster_size() {
+    uint32_t n;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;\n" : "=r"(n));
+    return n;
+}
+// Release arrive: this CTA's shared-memory writes before it become visible to
+// the cluster threads that complete the matching wait.
+__device__ __forceinline__ void cluster_arrive_release() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
+}
+// A float in the shared memory of cluster CTA `rank`, at the offset of `local`.
+__device__ __forceinline__ float ld_cluster_f32(const float* local, uint32_t rank) {
+    uint32_t remote;
+    float v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
+    asm volatile("ld.shared::cluster.f32 %0, [%1];\n" : "=f"(v) : "r"(remote) : "memory");
+    return v;
+}
 
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // bounded waits: one second
 
@@ -173,9 +191,14 @@ __device__ __forceinline__ bool conv_vec_any(const ConvIn& in, const AT* w, int6
     return true;
 }
 
-template <typename ST, typename AT, typename XT, int N, int CHUNKS, int VPT, bool FUSED>
+// NORM (fused only): the gated y goes through the gated RMSNorm before it is
+// stored. The norm's channel group (the hpg*P rows of an SSM group) is exactly
+// the CTA cluster, so the group's sum of squares is exchanged through
+// distributed shared memory.
+template <typename ST, typename AT, typename XT, int N, int CHUNKS, int VPT, bool FUSED, bool NORM>
 __global__ void __launch_bounds__(kThreads, M2_DECODE_MIN_BLOCKS)
 state_update_kernel(const StateUpdateArgs a) {
+    static_assert(FUSED || !NORM, "the norm exchange needs the group cluster of the fused launch");
     constexpr int EPV = Vec16<ST>::n;       // state elements per 16-byte vector
     constexpr int LPR = N / EPV;            // lanes per state row
     static_assert(LPR >= 1 && LPR <= 32 && (32 % LPR) == 0, "row must fit a warp");
@@ -207,6 +230,9 @@ state_update_kernel(const StateUpdateArgs a) {
     __shared__ float s_dA[kMaxHeadsPerTile];
     __shared__ float s_D[kMaxHeadsPerTile];
     __shared__ int s_fail;
+    __shared__ float s_red[kWarps];  // (NORM) per-warp sums of squares
+    __shared__ float s_part;         // (NORM) this CTA's sum of squares, read by the cluster
+    __shared__ float s_rstd;         // (NORM) 1 / sqrt(mean square + eps) of the group
 
     const int tid = threadIdx.x;
     const int b = blockIdx.y;
@@ -438,12 +464,53 @@ state_update_kernel(const StateUpdateArgs a) {
     __syncthreads();
 
     // ---- y (gated), contiguous over the tile's rows
-    if (ok) {
+    if constexpr (!NORM) {
+        if (ok) {
+            for (int i = tid; i < TILE; i += kThreads) {
+                float yv = s_y[i];
+                if (zrow) yv *= silu_f32(i == tid ? z_first : to_f32(zrow[r0 + i]));
+                yrow[r0 + i] = from_f32<AT>(yv);
+            }
+        }
+    } else {
+        // gated RMSNorm: v = y silu(z) over the group's hpg*P channels (this
+        // cluster), out = v / sqrt(mean(v^2) + eps) * w
+        float ss = 0.f;
         for (int i = tid; i < TILE; i += kThreads) {
             float yv = s_y[i];
             if (zrow) yv *= silu_f32(i == tid ? z_first : to_f32(zrow[r0 + i]));
-            yrow[r0 + i] = from_f32<AT>(yv);
+            s_y[i] = yv;
+            ss = fmaf(yv, yv, ss);
         }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        if ((tid & 31) == 0) s_red[tid >> 5] = ss;
+        __syncthreads();
+        if (tid == 0) {
+            float part = 0.f;
+            for (int w = 0; w < kWarps; ++w) part += s_red[w];
+            s_part = part;
+        }
+        // barrier phases (every thread, in order): the wait of the phase-1
+        // arrive, then publish s_part and wait for every CTA's, then read them
+        cluster_wait();
+        cluster_arrive_release();
+        cluster_wait();
+        if (tid == 0) {
+            float total = 0.f;
+            const uint32_t cs = cluster_size();
+            for (uint32_t q = 0; q < cs; ++q) total += ld_cluster_f32(&s_part, q);
+            s_rstd = rsqrtf(total / static_cast<float>(hpg * P) + a.norm_eps);
+        }
+        __syncthreads();
+        if (ok) {
+            const AT* nw = static_cast<const AT*>(a.norm_w);
+            const float rstd = s_rstd;
+            for (int i = tid; i < TILE; i += kThreads)
+                yrow[r0 + i] = from_f32<AT>(s_y[i] * rstd * to_f32(nw[r0 + i]));
+        }
+        // done with the other CTAs' s_part; the matching wait comes last
+        cluster_arrive();
     }
 
     if constexpr (FUSED) {
@@ -451,7 +518,7 @@ state_update_kernel(const StateUpdateArgs a) {
         // staged copy of the old rows and the raw inputs). Only rank 0 writes
         // after the barrier, so only rank 0 waits; the other CTAs have arrived
         // and may exit (exited threads never hold up a cluster wait).
-        if (cluster_rank() == 0) cluster_wait();
+        if (!NORM && cluster_rank() == 0) cluster_wait();  // NORM: that phase completed above
         if (ok && cluster_rank() == 0) {
             const AT* xrow = static_cast<const AT*>(a.xBC) + b * a.xBC_stride;
             for (int v = tid; v < 2 * BV; v += kThreads) {
@@ -466,12 +533,14 @@ state_update_kernel(const StateUpdateArgs a) {
                 }
             }
         }
+        // NORM: no CTA leaves while another may still read its s_part
+        if constexpr (NORM) cluster_wait();
     }
 }
 
-template <typename ST, typename AT, typename XT, int N, int CHUNKS, int VPT, bool FUSED>
+template <typename ST, typename AT, typename XT, int N, int CHUNKS, int VPT, bool FUSED, bool NORM>
 cudaError_t launch_one(const StateUpdateArgs& a, const DecodePlan& plan, cudaStream_t stream) {
-    auto kern = state_update_kernel<ST, AT, XT, N, CHUNKS, VPT, FUSED>;
+    auto kern = state_update_kernel<ST, AT, XT, N, CHUNKS, VPT, FUSED, NORM>;
     constexpr int LPR = N / Vec16<ST>::n;
     constexpr int TILE = CHUNKS * (kThreads / LPR) * VPT;
     size_t smem = static_cast<size_t>(TILE) * N * sizeof(ST);
@@ -504,15 +573,24 @@ cudaError_t launch_one(const StateUpdateArgs& a, const DecodePlan& plan, cudaStr
     return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-template <typename ST, typename AT, typename XT, int N, bool FUSED>
-cudaError_t by_loads(const StateUpdateArgs& a, const DecodePlan& p, cudaStream_t s) {
+template <typename ST, typename AT, typename XT, int N, bool FUSED, bool NORM>
+cudaError_t by_loads_norm(const StateUpdateArgs& a, const DecodePlan& p, cudaStream_t s) {
     // loads = 16-byte vectors per thread per tile = CHUNKS * VPT
     switch (p.loads) {
-        case 4 * M2_DECODE_MAIN_CHUNKS: return launch_one<ST, AT, XT, N, M2_DECODE_MAIN_CHUNKS, 4, FUSED>(a, p, s);
-        case 4: return launch_one<ST, AT, XT, N, 1, 4, FUSED>(a, p, s);
-        case 1: return launch_one<ST, AT, XT, N, 1, 1, FUSED>(a, p, s);
+        case 4 * M2_DECODE_MAIN_CHUNKS:
+            return launch_one<ST, AT, XT, N, M2_DECODE_MAIN_CHUNKS, 4, FUSED, NORM>(a, p, s);
+        case 4: return launch_one<ST, AT, XT, N, 1, 4, FUSED, NORM>(a, p, s);
+        case 1: return launch_one<ST, AT, XT, N, 1, 1, FUSED, NORM>(a, p, s);
         default: return cudaErrorInvalidValue;
     }
+}
+
+template <typename ST, typename AT, typename XT, int N, bool FUSED>
+cudaError_t by_loads(const StateUpdateArgs& a, const DecodePlan& p, cudaStream_t s) {
+    if constexpr (FUSED) {
+        if (a.norm_w) return by_loads_norm<ST, AT, XT, N, true, true>(a, p, s);
+    }
+    return by_loads_norm<ST, AT, XT, N, FUSED, false>(a, p, s);
 }
 
 template <typename ST, typename AT, typename XT, bool FUSED>
