@@ -177,6 +177,20 @@ m2_status m2_conv1d_update(const m2_cache* cache, const m2_conv_params* conv, in
                            const int32_t* slot_idx, m2_stream stream);
 
 /*
+ * m2_conv1d_update over nseq sequences packed back to back: sequence b is
+ * rows cu_seqlens[b] .. cu_seqlens[b+1]-1 of xBC / xBC_out (cu_seqlens
+ * [nseq+1] int32 on the device, cu_seqlens[nseq] = total_tokens) and rolls
+ * cache->conv[slot_idx[b]]. max_seqlen (host) sizes the grid; a longer
+ * sequence is still covered. An empty sequence leaves its slot untouched.
+ * Otherwise as m2_conv1d_update. One launch.
+ */
+m2_status m2_conv1d_update_varlen(const m2_cache* cache, const m2_conv_params* conv, int32_t nseq,
+                                  const int32_t* cu_seqlens, int64_t total_tokens, int32_t max_seqlen,
+                                  const void* xBC, int64_t xBC_row_stride, void* xBC_out,
+                                  int32_t out_dtype, int64_t out_row_stride, const int32_t* slot_idx,
+                                  m2_stream stream);
+
+/*
  * selective_state_update for one token per row (vllm.cpp issue, "The
  * divergence"), in place on cache->ssm at slot_idx[b].
  *   conv     non-NULL: xBC is the RAW row and the conv tap + roll of
@@ -316,6 +330,58 @@ m2_status m2_chunk_scan_varlen_static(const m2_cache* cache, const m2_ssm_params
                                       int64_t dt_row_stride, const void* z, int64_t z_row_stride,
                                       void* y, int64_t y_row_stride, const int32_t* slot_idx,
                                       const uint8_t* has_initial_state, m2_stream stream);
+
+/* The decode rows of a mixed step: one token each, raw xBC (the conv is
+ * fused), as for m2_state_update with conv != NULL. */
+typedef struct m2_decode_rows {
+    int32_t batch;
+    const void* xBC;  /* [batch, conv_dim] act_dtype, raw */
+    int64_t xBC_row_stride;
+    const void* dt;   /* [batch, H] act_dtype */
+    int64_t dt_row_stride;
+    const void* z;    /* [batch, H*P] act_dtype or NULL */
+    int64_t z_row_stride;
+    void* y;          /* [batch, H*P] act_dtype, out */
+    int64_t y_row_stride;
+    const int32_t* slot_idx;
+} m2_decode_rows;
+
+/* The prefill sequences of a mixed step, packed back to back (as for
+ * m2_chunk_scan_varlen), with the caller's buffer for the post-conv xBC. */
+typedef struct m2_prefill_rows {
+    int32_t nseq;
+    const int32_t* cu_seqlens;  /* [nseq+1] int32, device */
+    int64_t total_tokens;
+    int32_t max_seqlen;         /* host bound, sizes the grids */
+    const void* xBC;            /* [total_tokens, conv_dim] act_dtype, raw */
+    int64_t xBC_row_stride;
+    void* xBC_post;             /* [total_tokens, conv_dim] xBC_post_dtype, written */
+    int32_t xBC_post_dtype;     /* M2_F32, M2_BF16 or M2_F16 */
+    int64_t xBC_post_row_stride;
+    const void* dt;             /* [total_tokens, H] act_dtype */
+    int64_t dt_row_stride;
+    const void* z;              /* [total_tokens, H*P] act_dtype or NULL */
+    int64_t z_row_stride;
+    void* y;                    /* [total_tokens, H*P] act_dtype, out */
+    int64_t y_row_stride;
+    const int32_t* slot_idx;    /* [nseq] */
+    const uint8_t* has_initial_state;  /* [nseq] or NULL (all start from zero) */
+} m2_prefill_rows;
+
+/*
+ * One mixed serving step on one slot-indexed cache (TensorRT-LLM issue #16976:
+ * iterations that mix prefill chunks and decode tokens, where the decode part
+ * should stay graphed): the prefill sequences run the prefill conv
+ * (m2_conv1d_update_varlen into xBC_post) and the variable-length chunk scan,
+ * and the decode rows run the fused decode step, all enqueued on `stream` in
+ * one call (three launches: conv, scan, decode) with no allocation and no
+ * synchronisation. The scan does not split sequences here (no scratch). The
+ * decode slots and the prefill slots must be disjoint. Either part may be
+ * NULL or empty. Results are those of the separate calls, bit for bit.
+ */
+m2_status m2_mixed_step(const m2_cache* cache, const m2_ssm_params* ssm, const m2_conv_params* conv,
+                        const m2_decode_rows* decode, const m2_prefill_rows* prefill,
+                        m2_stream stream);
 
 /* Debug/test path: synchronises `stream`, copies the cache's error word to
  * *out_code (0 or an m2_status value) and clears it. Not for hot loops. */

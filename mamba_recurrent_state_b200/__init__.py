@@ -86,6 +86,23 @@ class m2_norm_params(ctypes.Structure):
     _fields_ = [("weight", ctypes.c_void_p), ("eps", ctypes.c_float)]
 
 
+class m2_decode_rows(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("xBC", ctypes.c_void_p), ("xBC_row_stride", ctypes.c_int64),
+                ("dt", ctypes.c_void_p), ("dt_row_stride", ctypes.c_int64), ("z", ctypes.c_void_p),
+                ("z_row_stride", ctypes.c_int64), ("y", ctypes.c_void_p), ("y_row_stride", ctypes.c_int64),
+                ("slot_idx", ctypes.c_void_p)]
+
+
+class m2_prefill_rows(ctypes.Structure):
+    _fields_ = [("nseq", ctypes.c_int32), ("cu_seqlens", ctypes.c_void_p), ("total_tokens", ctypes.c_int64),
+                ("max_seqlen", ctypes.c_int32), ("xBC", ctypes.c_void_p), ("xBC_row_stride", ctypes.c_int64),
+                ("xBC_post", ctypes.c_void_p), ("xBC_post_dtype", ctypes.c_int32),
+                ("xBC_post_row_stride", ctypes.c_int64), ("dt", ctypes.c_void_p),
+                ("dt_row_stride", ctypes.c_int64), ("z", ctypes.c_void_p), ("z_row_stride", ctypes.c_int64),
+                ("y", ctypes.c_void_p), ("y_row_stride", ctypes.c_int64), ("slot_idx", ctypes.c_void_p),
+                ("has_initial_state", ctypes.c_void_p)]
+
+
 # exported symbols and their signatures (mirrors include/m2.h)
 _P = ctypes.c_void_p
 _I32 = ctypes.c_int32
@@ -116,6 +133,11 @@ SIGNATURES = {
     "m2_chunk_scan_varlen_static": (_I32, [ctypes.POINTER(m2_cache), ctypes.POINTER(m2_ssm_params), _I32,
                                            _P, _I64, _I32, _I32, _P, _I32, _I64, _P, _I64, _P, _I64,
                                            _P, _I64, _P, _P, _P]),
+    "m2_conv1d_update_varlen": (_I32, [ctypes.POINTER(m2_cache), ctypes.POINTER(m2_conv_params), _I32, _P,
+                                       _I64, _I32, _P, _I64, _P, _I32, _I64, _P, _P]),
+    "m2_mixed_step": (_I32, [ctypes.POINTER(m2_cache), ctypes.POINTER(m2_ssm_params),
+                             ctypes.POINTER(m2_conv_params), ctypes.POINTER(m2_decode_rows),
+                             ctypes.POINTER(m2_prefill_rows), _P]),
     "m2_get_device_error": (_I32, [ctypes.POINTER(m2_cache), _P, ctypes.POINTER(_I32)]),
     "m2_status_string": (ctypes.c_char_p, [_I32]),
     "m2_version": (ctypes.c_char_p, []),
@@ -359,6 +381,51 @@ def conv1d_update(cache: Cache, conv: ConvParams, xBC: torch.Tensor, slot_idx: t
                                 _stream_ptr() if stream is None else stream)
     _check(st, "m2_conv1d_update")
     return out
+
+
+def conv1d_update_varlen(cache: Cache, conv: ConvParams, xBC: torch.Tensor, cu_seqlens: torch.Tensor,
+                         slot_idx: torch.Tensor, max_seqlen: int, out: Optional[torch.Tensor] = None,
+                         out_dtype: Optional[torch.dtype] = None, stream: Optional[int] = None) -> torch.Tensor:
+    """causal_conv1d_update over sequences packed back to back: xBC [total_tokens, conv_dim]."""
+    total, cd = xBC.shape
+    if out is None:
+        out = torch.empty((total, cd), dtype=out_dtype or xBC.dtype, device=xBC.device)
+    cp = conv.c()
+    st = lib().m2_conv1d_update_varlen(ctypes.byref(cache.c), ctypes.byref(cp), cu_seqlens.numel() - 1,
+                                       cu_seqlens.data_ptr(), total, max_seqlen, xBC.data_ptr(), xBC.stride(0),
+                                       out.data_ptr(), _dtype_code(out.dtype), out.stride(0),
+                                       slot_idx.data_ptr(), _stream_ptr() if stream is None else stream)
+    _check(st, "m2_conv1d_update_varlen")
+    return out
+
+
+def mixed_step(cache: Cache, ssm: SSMParams, conv: ConvParams, decode: Optional[dict] = None,
+               prefill: Optional[dict] = None, stream: Optional[int] = None) -> None:
+    """One mixed step (m2_mixed_step). ``decode``: dict(xBC, dt, z, y, slot_idx) with
+    one raw row per sequence; ``prefill``: dict(xBC, xBC_post, dt, z, y, cu_seqlens,
+    slot_idx, max_seqlen, has_initial_state) over packed tokens. Outputs are written
+    into the given y tensors."""
+    d = p = None
+    if decode is not None:
+        z = decode.get("z")
+        d = m2_decode_rows(decode["xBC"].shape[0], decode["xBC"].data_ptr(), decode["xBC"].stride(0),
+                           decode["dt"].data_ptr(), decode["dt"].stride(0), _ptr(z),
+                           z.stride(0) if z is not None else 0, decode["y"].data_ptr(), decode["y"].stride(0),
+                           decode["slot_idx"].data_ptr())
+    if prefill is not None:
+        z = prefill.get("z")
+        xp = prefill["xBC_post"]
+        cu = prefill["cu_seqlens"]
+        p = m2_prefill_rows(cu.numel() - 1, cu.data_ptr(), prefill["xBC"].shape[0], prefill["max_seqlen"],
+                            prefill["xBC"].data_ptr(), prefill["xBC"].stride(0), xp.data_ptr(),
+                            _dtype_code(xp.dtype), xp.stride(0), prefill["dt"].data_ptr(),
+                            prefill["dt"].stride(0), _ptr(z), z.stride(0) if z is not None else 0,
+                            prefill["y"].data_ptr(), prefill["y"].stride(0), prefill["slot_idx"].data_ptr(),
+                            _ptr(prefill.get("has_initial_state")))
+    st = lib().m2_mixed_step(ctypes.byref(cache.c), ctypes.byref(ssm.c()), ctypes.byref(conv.c()),
+                             ctypes.byref(d) if d is not None else None, ctypes.byref(p) if p is not None else None,
+                             _stream_ptr() if stream is None else stream)
+    _check(st, "m2_mixed_step")
 
 
 def chunk_scan(cache: Cache, ssm: SSMParams, xBC: torch.Tensor, dt: torch.Tensor,

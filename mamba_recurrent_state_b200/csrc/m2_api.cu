@@ -185,10 +185,11 @@ m2_status m2_cache_zero_slots(const m2_cache* c, int32_t n, const int32_t* slot_
     return from_cuda(m2::launch_zero_slots(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-m2_status m2_conv1d_update(const m2_cache* c, const m2_conv_params* conv, int32_t batch,
-                           int32_t seqlen, const void* xBC, int64_t xBC_row_stride, void* xBC_out,
-                           int32_t out_dtype, int64_t out_row_stride, const int32_t* slot_idx,
-                           m2_stream stream) {
+namespace {
+
+m2_status conv1d_impl(const m2_cache* c, const m2_conv_params* conv, int32_t batch, int32_t seqlen,
+                      const int32_t* cu_seqlens, const void* xBC, int64_t xBC_row_stride, void* xBC_out,
+                      int32_t out_dtype, int64_t out_row_stride, const int32_t* slot_idx, m2_stream stream) {
     const m2_status st = cache_status(c);
     if (st != M2_OK) return st;
     if (!conv || !conv->weight || batch < 0 || seqlen < 0 || !valid_buffer_dtype(out_dtype))
@@ -225,7 +226,30 @@ m2_status m2_conv1d_update(const m2_cache* c, const m2_conv_params* conv, int32_
     a.out = xBC_out;
     a.out_stride = out_row_stride;
     a.slot_idx = slot_idx;
+    a.cu_seqlens = cu_seqlens;
     return from_cuda(m2::launch_conv1d_update(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
+m2_status m2_conv1d_update(const m2_cache* c, const m2_conv_params* conv, int32_t batch, int32_t seqlen,
+                           const void* xBC, int64_t xBC_row_stride, void* xBC_out, int32_t out_dtype,
+                           int64_t out_row_stride, const int32_t* slot_idx, m2_stream stream) {
+    return conv1d_impl(c, conv, batch, seqlen, nullptr, xBC, xBC_row_stride, xBC_out, out_dtype, out_row_stride,
+                       slot_idx, stream);
+}
+
+m2_status m2_conv1d_update_varlen(const m2_cache* c, const m2_conv_params* conv, int32_t nseq,
+                                  const int32_t* cu_seqlens, int64_t total_tokens, int32_t max_seqlen,
+                                  const void* xBC, int64_t xBC_row_stride, void* xBC_out, int32_t out_dtype,
+                                  int64_t out_row_stride, const int32_t* slot_idx, m2_stream stream) {
+    if (nseq < 0 || total_tokens < 0 || max_seqlen < 0) return M2_ERR_INVALID_ARG;
+    if (total_tokens > INT32_MAX) return M2_ERR_UNSUPPORTED;
+    if (nseq > 0 && total_tokens > 0 && !cu_seqlens) return M2_ERR_INVALID_ARG;
+    // no tokens: validate and return, as a zero-length fixed call does
+    const int32_t len = (nseq == 0 || total_tokens == 0) ? 0 : std::max(max_seqlen, 1);
+    return conv1d_impl(c, conv, nseq, len, cu_seqlens, xBC, xBC_row_stride, xBC_out, out_dtype, out_row_stride,
+                       slot_idx, stream);
 }
 
 namespace {
@@ -549,6 +573,43 @@ m2_status m2_chunk_scan_varlen_static(const m2_cache* c, const m2_ssm_params* ss
         a.seg_decay = reinterpret_cast<float*>(static_cast<char*>(scratch) + state_bytes);
     }
     return from_cuda(m2::launch_chunk_scan(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+m2_status m2_mixed_step(const m2_cache* c, const m2_ssm_params* ssm, const m2_conv_params* conv,
+                        const m2_decode_rows* decode, const m2_prefill_rows* prefill, m2_stream stream) {
+    const m2_status st = cache_status(c);
+    if (st != M2_OK) return st;
+    if (!ssm || !conv) return M2_ERR_INVALID_ARG;
+    const bool has_pre = prefill && prefill->nseq > 0 && prefill->total_tokens > 0;
+    const bool has_dec = decode && decode->batch > 0;
+    if ((prefill && (prefill->nseq < 0 || prefill->total_tokens < 0)) || (decode && decode->batch < 0))
+        return M2_ERR_INVALID_ARG;
+    if (has_pre) {
+        const m2_prefill_rows& p = *prefill;
+        if (p.total_tokens > INT32_MAX) return M2_ERR_UNSUPPORTED;
+        if (!p.cu_seqlens || !p.xBC_post) return M2_ERR_INVALID_ARG;
+        m2_status r = conv1d_impl(c, conv, p.nseq, std::max(p.max_seqlen, 1), p.cu_seqlens, p.xBC,
+                                  p.xBC_row_stride, p.xBC_post, p.xBC_post_dtype, p.xBC_post_row_stride,
+                                  p.slot_idx, stream);
+        if (r != M2_OK) return r;
+        m2::ScanArgs a{};
+        r = scan_args(c, ssm, p.nseq, 128, p.xBC_post, p.xBC_post_dtype, p.xBC_post_row_stride, p.dt,
+                      p.dt_row_stride, p.z, p.z_row_stride, p.y, p.y_row_stride, p.slot_idx, p.has_initial_state,
+                      stream, &a);
+        if (r != M2_OK) return r;
+        a.cu_seqlens = p.cu_seqlens;
+        a.seqlen = p.max_seqlen;
+        a.total_tokens = p.total_tokens;  // nseg = 1: no split, no scratch
+        const cudaError_t e = m2::launch_chunk_scan(a, reinterpret_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return from_cuda(e);
+    }
+    if (has_dec) {
+        const m2_decode_rows& d = *decode;
+        return state_update_impl(c, ssm, conv, nullptr, d.batch, d.xBC, c->shape.act_dtype, d.xBC_row_stride,
+                                 d.dt, d.dt_row_stride, d.z, d.z_row_stride, d.y, d.y_row_stride, d.slot_idx,
+                                 stream);
+    }
+    return M2_OK;
 }
 
 m2_status m2_get_device_error(const m2_cache* c, m2_stream stream, int32_t* out_code) {

@@ -16,6 +16,7 @@
 // new cache rows afterwards, so no other CTA can observe a half-rolled cache.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <type_traits>
 
 #include "m2_device.cuh"
@@ -43,24 +44,30 @@ __device__ __forceinline__ void store_vec(OT* p, const float* o) {
     }
 }
 
+// Variable-length batches (cu_seqlens): sequence b is packed rows
+// cu_seqlens[b] .. cu_seqlens[b+1]-1 and the CTA walks the sequence's token
+// tiles blockIdx.y, blockIdx.y + gridDim.y, ..., so a sequence longer than
+// the grid was planned for is still covered; tile 0 (the only one that reads
+// the cache) is always its blockIdx.y == 0 CTA's first.
 template <typename AT, typename OT, int K>
 __global__ void __launch_bounds__(kConvThreads) conv1d_kernel(const ConvArgs a) {
     constexpr int VEC = Vec16<AT>::n;
     const int b = blockIdx.z;
-    const int t0 = blockIdx.y * kTT;
     const int64_t c0 = (static_cast<int64_t>(blockIdx.x) * kConvThreads + threadIdx.x) * VEC;
     if (c0 >= a.conv_dim) return;
-    const int T = a.seqlen;
-    const int t_end = min(t0 + kTT, T);
+    const int64_t row0 = a.cu_seqlens ? static_cast<int64_t>(a.cu_seqlens[b]) : static_cast<int64_t>(b) * a.seqlen;
+    const int T = a.cu_seqlens ? a.cu_seqlens[b + 1] - a.cu_seqlens[b] : a.seqlen;
+    if (T <= 0) return;  // an empty sequence leaves its cache slot untouched
 
     const int32_t slot = a.slot_idx[b];
-    const AT* xb = static_cast<const AT*>(a.x) + static_cast<int64_t>(b) * T * a.x_stride;
-    OT* ob = static_cast<OT*>(a.out) + static_cast<int64_t>(b) * T * a.out_stride;
+    const AT* xb = static_cast<const AT*>(a.x) + row0 * a.x_stride;
+    OT* ob = static_cast<OT*>(a.out) + row0 * a.out_stride;
     if (slot < 0) {  // padding row: zero output, cache untouched
         float zeros[VEC];
 #pragma unroll
         for (int v = 0; v < VEC; ++v) zeros[v] = 0.f;
-        for (int t = t0; t < t_end; ++t) store_vec<OT, VEC>(ob + t * a.out_stride + c0, zeros);
+        for (int t0 = blockIdx.y * kTT; t0 < T; t0 += gridDim.y * kTT)
+            for (int t = t0; t < min(t0 + kTT, T); ++t) store_vec<OT, VEC>(ob + t * a.out_stride + c0, zeros);
         return;
     }
     if (slot >= a.num_slots) {
@@ -82,8 +89,13 @@ __global__ void __launch_bounds__(kConvThreads) conv1d_kernel(const ConvArgs a) 
         }
     }
 
-    // history: raw vectors of tokens t0-K+1 .. t0-1 (oldest first)
+    float out_max = 0.f;  // largest post-conv magnitude (checked for fp16 outputs)
+    // the raw history of the CTA's latest tile; the cache roll below needs the
+    // old cache rows only when T < K-1, when tile 0 is the only tile
     uint4 hist_raw[K - 1];
+    for (int t0 = blockIdx.y * kTT; t0 < T; t0 += gridDim.y * kTT) {
+    const int t_end = min(t0 + kTT, T);
+    // history: raw vectors of tokens t0-K+1 .. t0-1 (oldest first)
 #pragma unroll
     for (int j = 0; j < K - 1; ++j) {
         const int t = t0 - (K - 1) + j;
@@ -94,7 +106,6 @@ __global__ void __launch_bounds__(kConvThreads) conv1d_kernel(const ConvArgs a) 
 #pragma unroll
     for (int j = 0; j < K - 1; ++j) unpack16<AT>(hist_raw[j], hist[j]);
 
-    float out_max = 0.f;  // largest post-conv magnitude (checked for fp16 outputs)
     // all of the tile's raw inputs are loaded before any output is stored, so
     // the loads are in flight together (the output may alias nothing, but the
     // compiler cannot know that)
@@ -133,6 +144,7 @@ __global__ void __launch_bounds__(kConvThreads) conv1d_kernel(const ConvArgs a) 
             for (int v = 0; v < VEC; ++v) hist[K - 2][v] = cur[v];
         }
     }
+    }
 
     if (out_max >= 65520.f) record_error(a.error, M2_ERR_RANGE);  // beyond fp16 (rounds to inf)
     if (blockIdx.y == 0) {
@@ -159,8 +171,10 @@ __global__ void __launch_bounds__(kConvThreads) conv1d_kernel(const ConvArgs a) 
 template <typename AT, typename OT>
 cudaError_t conv_by_k(const ConvArgs& a, cudaStream_t s) {
     constexpr int VEC = Vec16<AT>::n;
+    // token tiles per sequence: at least one, at most 65535 (the CTAs loop)
+    const int64_t tiles = std::min<int64_t>(std::max<int64_t>((a.seqlen + kTT - 1) / kTT, 1), 65535);
     const dim3 grid(static_cast<unsigned>((a.conv_dim / VEC + kConvThreads - 1) / kConvThreads),
-                    static_cast<unsigned>((a.seqlen + kTT - 1) / kTT), static_cast<unsigned>(a.batch));
+                    static_cast<unsigned>(tiles), static_cast<unsigned>(a.batch));
     switch (a.K) {
         case 2: conv1d_kernel<AT, OT, 2><<<grid, kConvThreads, 0, s>>>(a); break;
         case 3: conv1d_kernel<AT, OT, 3><<<grid, kConvThreads, 0, s>>>(a); break;

@@ -77,6 +77,9 @@ struct ConvArgs {
     void* out;
     int64_t out_stride;
     const int32_t* slot_idx;
+    // variable-length batches: sequence b is packed rows cu_seqlens[b] ..
+    // cu_seqlens[b+1]-1 (NULL: rows b*seqlen ..); seqlen then bounds the grid
+    const int32_t* cu_seqlens;
 };
 
 struct ZeroArgs {
