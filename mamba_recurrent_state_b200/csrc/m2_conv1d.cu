@@ -49,8 +49,11 @@ __device__ __forceinline__ void store_vec(OT* p, const float* o) {
 // tiles blockIdx.y, blockIdx.y + gridDim.y, ..., so a sequence longer than
 // the grid was planned for is still covered; tile 0 (the only one that reads
 // the cache) is always its blockIdx.y == 0 CTA's first.
+// The prefill path (K <= 4, 16-bit post-conv output) is held to three CTAs
+// per SM (168 registers, no spills); the tile loop would otherwise take ~200.
 template <typename AT, typename OT, int K>
-__global__ void __launch_bounds__(kConvThreads) conv1d_kernel(const ConvArgs a) {
+__global__ void __launch_bounds__(kConvThreads, (sizeof(OT) == 2 && K <= 4) ? 3 : 1)
+conv1d_kernel(const ConvArgs a) {
     constexpr int VEC = Vec16<AT>::n;
     const int b = blockIdx.z;
     const int64_t c0 = (static_cast<int64_t>(blockIdx.x) * kConvThreads + threadIdx.x) * VEC;
@@ -90,12 +93,11 @@ __global__ void __launch_bounds__(kConvThreads) conv1d_kernel(const ConvArgs a) 
     }
 
     float out_max = 0.f;  // largest post-conv magnitude (checked for fp16 outputs)
-    // the raw history of the CTA's latest tile; the cache roll below needs the
-    // old cache rows only when T < K-1, when tile 0 is the only tile
-    uint4 hist_raw[K - 1];
+#pragma unroll 1
     for (int t0 = blockIdx.y * kTT; t0 < T; t0 += gridDim.y * kTT) {
     const int t_end = min(t0 + kTT, T);
     // history: raw vectors of tokens t0-K+1 .. t0-1 (oldest first)
+    uint4 hist_raw[K - 1];
 #pragma unroll
     for (int j = 0; j < K - 1; ++j) {
         const int t = t0 - (K - 1) + j;
@@ -149,20 +151,14 @@ __global__ void __launch_bounds__(kConvThreads) conv1d_kernel(const ConvArgs a) 
     if (out_max >= 65520.f) record_error(a.error, M2_ERR_RANGE);  // beyond fp16 (rounds to inf)
     if (blockIdx.y == 0) {
         // new cache row k holds the raw input of token T-(K-1)+k: from the input
-        // when that token exists, else from the old cache rows read above
-        // (only possible when T < K-1, in which case this tile saw every token)
+        // when that token exists, else old cache row k + T (only when
+        // T < K-1; rows are written in increasing k and row k + T > k is read
+        // before row k + T is written, so every read sees an old row)
 #pragma unroll
         for (int k = 0; k < K - 1; ++k) {
             const int t = T - (K - 1) + k;
-            uint4 v;
-            if (t >= 0) {
-                v = *reinterpret_cast<const uint4*>(xb + t * a.x_stride + c0);
-            } else {
-#pragma unroll
-                for (int j = 0; j < K - 1; ++j) {
-                    if (j == k + T) v = hist_raw[j];  // old cache row k + T
-                }
-            }
+            const uint4 v = t >= 0 ? *reinterpret_cast<const uint4*>(xb + t * a.x_stride + c0)
+                                   : *reinterpret_cast<const uint4*>(cache + (k + T) * a.conv_dim + c0);
             *reinterpret_cast<uint4*>(cache + k * a.conv_dim + c0) = v;
         }
     }

@@ -77,13 +77,11 @@ __device__ __forceinline__ uint32_t cluster_size() {
 __device__ __forceinline__ void cluster_arrive_release() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
 }
-// A float in the shared memory of cluster CTA `rank`, at the offset of `local`.
-__device__ __forceinline__ float ld_cluster_f32(const float* local, uint32_t rank) {
+// Stores v into the shared memory of cluster CTA `rank`, at the offset of `local`.
+__device__ __forceinline__ void st_cluster_f32(float* local, uint32_t rank, float v) {
     uint32_t remote;
-    float v;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
-    asm volatile("ld.shared::cluster.f32 %0, [%1];\n" : "=f"(v) : "r"(remote) : "memory");
-    return v;
+    asm volatile("st.shared::cluster.f32 [%0], %1;\n" ::"r"(remote), "f"(v) : "memory");
 }
 
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // bounded waits: one second
@@ -231,7 +229,7 @@ state_update_kernel(const StateUpdateArgs a) {
     __shared__ float s_D[kMaxHeadsPerTile];
     __shared__ int s_fail;
     __shared__ float s_red[kWarps];  // (NORM) per-warp sums of squares
-    __shared__ float s_part;         // (NORM) this CTA's sum of squares, read by the cluster
+    __shared__ float s_parts[16];    // (NORM) every cluster CTA's sum of squares, pushed by each
     __shared__ float s_rstd;         // (NORM) 1 / sqrt(mean square + eps) of the group
 
     const int tid = threadIdx.x;
@@ -486,20 +484,23 @@ state_update_kernel(const StateUpdateArgs a) {
         for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
         if ((tid & 31) == 0) s_red[tid >> 5] = ss;
         __syncthreads();
-        if (tid == 0) {
+        // barrier phases (every thread, in order): the wait of the phase-1
+        // arrive (after it every cluster CTA is past its conv reads), then each
+        // CTA pushes its partial into every CTA's s_parts[own rank] and the
+        // release/acquire phase makes them visible. Nothing reads another CTA's
+        // shared memory afterwards, so a CTA may exit as soon as it is done.
+        cluster_wait();
+        const uint32_t cs = cluster_size();
+        if (tid < static_cast<int>(cs)) {
             float part = 0.f;
             for (int w = 0; w < kWarps; ++w) part += s_red[w];
-            s_part = part;
+            st_cluster_f32(&s_parts[cluster_rank()], static_cast<uint32_t>(tid), part);
         }
-        // barrier phases (every thread, in order): the wait of the phase-1
-        // arrive, then publish s_part and wait for every CTA's, then read them
-        cluster_wait();
         cluster_arrive_release();
         cluster_wait();
         if (tid == 0) {
             float total = 0.f;
-            const uint32_t cs = cluster_size();
-            for (uint32_t q = 0; q < cs; ++q) total += ld_cluster_f32(&s_part, q);
+            for (uint32_t q = 0; q < cs; ++q) total += s_parts[q];
             s_rstd = rsqrtf(total / static_cast<float>(hpg * P) + a.norm_eps);
         }
         __syncthreads();
@@ -509,8 +510,6 @@ state_update_kernel(const StateUpdateArgs a) {
             for (int i = tid; i < TILE; i += kThreads)
                 yrow[r0 + i] = from_f32<AT>(s_y[i] * rstd * to_f32(nw[r0 + i]));
         }
-        // done with the other CTAs' s_part; the matching wait comes last
-        cluster_arrive();
     }
 
     if constexpr (FUSED) {
@@ -533,8 +532,6 @@ state_update_kernel(const StateUpdateArgs a) {
                 }
             }
         }
-        // NORM: no CTA leaves while another may still read its s_part
-        if constexpr (NORM) cluster_wait();
     }
 }
 
