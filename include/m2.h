@@ -331,7 +331,34 @@ m2_status m2_chunk_scan_varlen_static(const m2_cache* cache, const m2_ssm_params
                                       void* y, int64_t y_row_stride, const int32_t* slot_idx,
                                       const uint8_t* has_initial_state, m2_stream stream);
 
-/* The decode rows of a mixed step: one token each, raw xBC (the conv is
+/*
+ * Multi-token decode for speculative decoding: T draft tokens per sequence in
+ * one launch (1 <= T <= 16), each token a decode step with the conv tap fused,
+ * starting from the state and conv window of cache slot slot_idx[b]. The
+ * state and the conv window after token t are stored into cache slot
+ * token_slots[b*T + t] (negative: not stored); the input slot is only read, so
+ * after verifying the drafts the caller adopts the slot of the last accepted
+ * token and the rejected ones are simply dropped. Every state is rounded to the
+ * storage dtype after its token, exactly as T separate m2_state_update calls
+ * would store it; y of token t comes from the unrounded state.
+ *   xBC          [batch, T, conv_dim] act_dtype, raw; token rows
+ *                xBC_row_stride apart, row b*T + t
+ *   dt           [batch, T, H] act_dtype;  z [batch, T, H*P] act_dtype or NULL
+ *   y            [batch, T, H*P] act_dtype, out
+ *   slot_idx     [batch] int32 (negative: padding row, y = 0, nothing stored)
+ *   token_slots  [batch, T] int32; every non-negative entry, and every input
+ *                slot, must be distinct (checked on the host under
+ *                M2_VALIDATE=1); an entry >= num_slots is a device error
+ * Supported: H*P/G a multiple of 64, P a multiple of 8, N in {64, 128, 256}
+ * (256 only with a bf16 state). One launch, no scratch memory.
+ */
+m2_status m2_state_update_multi(const m2_cache* cache, const m2_ssm_params* ssm,
+                                const m2_conv_params* conv, int32_t batch, int32_t T, const void* xBC,
+                                int64_t xBC_row_stride, const void* dt, int64_t dt_row_stride,
+                                const void* z, int64_t z_row_stride, void* y, int64_t y_row_stride,
+                                const int32_t* slot_idx, const int32_t* token_slots, m2_stream stream);
+
+/* The decode rows of a mixed step: one token each, raw xBC (the conv is/* The decode rows of a mixed step: one token each, raw xBC (the conv is
  * fused), as for m2_state_update with conv != NULL. */
 typedef struct m2_decode_rows {
     int32_t batch;

@@ -138,6 +138,9 @@ SIGNATURES = {
     "m2_mixed_step": (_I32, [ctypes.POINTER(m2_cache), ctypes.POINTER(m2_ssm_params),
                              ctypes.POINTER(m2_conv_params), ctypes.POINTER(m2_decode_rows),
                              ctypes.POINTER(m2_prefill_rows), _P]),
+    "m2_state_update_multi": (_I32, [ctypes.POINTER(m2_cache), ctypes.POINTER(m2_ssm_params),
+                                     ctypes.POINTER(m2_conv_params), _I32, _I32, _P, _I64, _P, _I64, _P, _I64,
+                                     _P, _I64, _P, _P, _P]),
     "m2_get_device_error": (_I32, [ctypes.POINTER(m2_cache), _P, ctypes.POINTER(_I32)]),
     "m2_status_string": (ctypes.c_char_p, [_I32]),
     "m2_version": (ctypes.c_char_p, []),
@@ -397,6 +400,27 @@ def conv1d_update_varlen(cache: Cache, conv: ConvParams, xBC: torch.Tensor, cu_s
                                        slot_idx.data_ptr(), _stream_ptr() if stream is None else stream)
     _check(st, "m2_conv1d_update_varlen")
     return out
+
+
+def state_update_multi(cache: Cache, ssm: SSMParams, conv: ConvParams, xBC: torch.Tensor, dt: torch.Tensor,
+                       slot_idx: torch.Tensor, token_slots: torch.Tensor, z: Optional[torch.Tensor] = None,
+                       y: Optional[torch.Tensor] = None, stream: Optional[int] = None) -> torch.Tensor:
+    """T draft tokens per row (m2_state_update_multi): xBC [batch, T, conv_dim] raw,
+    dt [batch, T, H]; the state after token t goes to slot token_slots[b, t].
+    Returns y [batch, T, H*P]."""
+    sh = cache.shape
+    batch, T, _ = xBC.shape
+    for t in (xBC, dt) + ((z,) if z is not None else ()):
+        if t.stride(0) != t.shape[1] * t.stride(1):
+            raise ValueError("token rows of a sequence must be consecutive")
+    if y is None:
+        y = torch.empty((batch, T, sh.H * sh.P), dtype=torch_dtype(sh.act_dtype), device=xBC.device)
+    st = lib().m2_state_update_multi(
+        ctypes.byref(cache.c), ctypes.byref(ssm.c()), ctypes.byref(conv.c()), batch, T, xBC.data_ptr(),
+        xBC.stride(1), dt.data_ptr(), dt.stride(1), _ptr(z), z.stride(1) if z is not None else 0, y.data_ptr(),
+        y.stride(1), slot_idx.data_ptr(), token_slots.data_ptr(), _stream_ptr() if stream is None else stream)
+    _check(st, "m2_state_update_multi")
+    return y
 
 
 def mixed_step(cache: Cache, ssm: SSMParams, conv: ConvParams, decode: Optional[dict] = None,

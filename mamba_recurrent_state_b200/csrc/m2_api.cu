@@ -575,6 +575,79 @@ m2_status m2_chunk_scan_varlen_static(const m2_cache* c, const m2_ssm_params* ss
     return from_cuda(m2::launch_chunk_scan(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+m2_status m2_state_update_multi(const m2_cache* c, const m2_ssm_params* ssm, const m2_conv_params* conv,
+                                int32_t batch, int32_t T, const void* xBC, int64_t xBC_row_stride, const void* dt,
+                                int64_t dt_row_stride, const void* z, int64_t z_row_stride, void* y,
+                                int64_t y_row_stride, const int32_t* slot_idx, const int32_t* token_slots,
+                                m2_stream stream) {
+    const m2_status st = cache_status(c);
+    if (st != M2_OK) return st;
+    if (!ssm || !ssm->A_log || !ssm->dt_bias || !ssm->D || !conv || !conv->weight || batch < 0 || T < 0)
+        return M2_ERR_INVALID_ARG;
+    if (conv->activation != 0 && conv->activation != 1) return M2_ERR_INVALID_ARG;
+    if (batch == 0 || T == 0) return M2_OK;
+    if (!xBC || !dt || !y || !slot_idx || !token_slots) return M2_ERR_INVALID_ARG;
+    const m2_shape& s = c->shape;
+    const int as = dsize(s.act_dtype);
+    const int64_t cd = m2_conv_dim(&s);
+    const int64_t hp = static_cast<int64_t>(s.nheads) * s.head_dim;
+    if (!aligned16(xBC) || !aligned16(y) || !stride_ok(xBC_row_stride, as, cd) || !stride_ok(y_row_stride, as, hp) ||
+        dt_row_stride < s.nheads || !aligned16(conv->weight) || (conv->bias && !aligned16(conv->bias)))
+        return M2_ERR_INVALID_ARG;
+    if (z && (!aligned16(z) || !stride_ok(z_row_stride, as, hp))) return M2_ERR_INVALID_ARG;
+    const m2_status ps = m2::plan_multi_token(s.nheads, s.head_dim, s.d_state, s.ngroups, s.d_conv, T);
+    if (ps != M2_OK) return ps;
+    if (s.state_dtype != M2_BF16 && s.d_state == 256) return M2_ERR_UNSUPPORTED;
+    if (validate_mode()) {
+        // input slots and every token's destination slot: all distinct
+        const int64_t n = static_cast<int64_t>(batch) * (T + 1);
+        std::vector<int32_t> all(static_cast<size_t>(n));
+        const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+        if (cudaMemcpyAsync(all.data(), slot_idx, batch * sizeof(int32_t), cudaMemcpyDeviceToHost, cs) != cudaSuccess ||
+            cudaMemcpyAsync(all.data() + batch, token_slots, static_cast<size_t>(batch) * T * sizeof(int32_t),
+                            cudaMemcpyDeviceToHost, cs) != cudaSuccess ||
+            cudaStreamSynchronize(cs) != cudaSuccess)
+            return M2_ERR_CUDA;
+        std::vector<int32_t> used;
+        for (int32_t v : all)
+            if (v >= 0) used.push_back(v);
+        std::sort(used.begin(), used.end());
+        if (std::adjacent_find(used.begin(), used.end()) != used.end()) return M2_ERR_INVALID_ARG;
+    }
+    m2::MtArgs a{};
+    a.ssm = c->ssm;
+    a.conv = c->conv;
+    a.error = c->error;
+    a.num_slots = c->num_slots;
+    a.H = s.nheads;
+    a.P = s.head_dim;
+    a.N = s.d_state;
+    a.G = s.ngroups;
+    a.K = s.d_conv;
+    a.T = T;
+    a.conv_dim = cd;
+    a.state_bf16 = s.state_dtype == M2_BF16;
+    a.act_bf16 = s.act_dtype == M2_BF16;
+    a.A_log = ssm->A_log;
+    a.dt_bias = ssm->dt_bias;
+    a.D = ssm->D;
+    a.conv_w = conv->weight;
+    a.conv_b = conv->bias;
+    a.activation = conv->activation;
+    a.batch = batch;
+    a.xBC = xBC;
+    a.xBC_stride = xBC_row_stride;
+    a.dt = dt;
+    a.dt_stride = dt_row_stride;
+    a.z = z;
+    a.z_stride = z_row_stride;
+    a.y = y;
+    a.y_stride = y_row_stride;
+    a.slot_idx = slot_idx;
+    a.token_slots = token_slots;
+    return from_cuda(m2::launch_state_update_mt(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 m2_status m2_mixed_step(const m2_cache* c, const m2_ssm_params* ssm, const m2_conv_params* conv,
                         const m2_decode_rows* decode, const m2_prefill_rows* prefill, m2_stream stream) {
     const m2_status st = cache_status(c);

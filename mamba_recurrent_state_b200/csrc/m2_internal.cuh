@@ -125,6 +125,38 @@ struct ScanArgs {
     float* seg_decay;  // [batch][nseg][H] fp32 scratch (nseg > 1)
 };
 
+// Multi-token decode (speculative drafts): T tokens per row from slot_idx[b],
+// the state and conv window after token t stored into token_slots[b*T + t].
+constexpr int kMaxDraftTokens = 16;
+struct MtArgs {
+    void* ssm;
+    void* conv;
+    int32_t* error;
+    int64_t num_slots;
+    int H, P, N, G, K, T;
+    int64_t conv_dim;
+    int state_bf16, act_bf16;
+    const float* A_log;
+    const float* dt_bias;
+    const float* D;
+    const void* conv_w;
+    const void* conv_b;
+    int activation;
+    int batch;
+    const void* xBC;  // [batch, T, conv_dim] raw, token rows xBC_stride apart
+    int64_t xBC_stride;
+    const void* dt;   // [batch, T, H]
+    int64_t dt_stride;
+    const void* z;    // [batch, T, H*P] or NULL
+    int64_t z_stride;
+    void* y;          // [batch, T, H*P]
+    int64_t y_stride;
+    const int32_t* slot_idx;     // [batch], read only
+    const int32_t* token_slots;  // [batch, T], written
+};
+m2_status plan_multi_token(int H, int P, int N, int G, int K, int T);
+cudaError_t launch_state_update_mt(const MtArgs& a, cudaStream_t stream);
+
 // Launch-shape query for the decode kernels: M2_OK and the shape, or
 // M2_ERR_UNSUPPORTED. Pure host arithmetic.
 struct DecodePlan {
