@@ -57,9 +57,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--l2", choices=["rotate", "flush"], default="rotate",
                     help="rotate: disjoint slot sets, back to back; flush: 512 MiB write before each step")
-    ap.add_argument("--sections", default="decode,norm,prefill,longprompt,stack48",
+    ap.add_argument("--sections", default="decode,norm,multi,prefill,longprompt,stack48",
                     help="comma list: decode (the headline, always run), norm (decode with the "
-                         "fused gated RMSNorm), prefill (workload 4: "
+                         "fused gated RMSNorm), multi (4 speculative draft tokens), prefill (workload 4: "
                          "prefill conv and tensor-core scan), longprompt (one 16K-token prompt: "
                          "conv and varlen scan), stack48 (workload 2: 48-layer token)")
     return ap.parse_args()
@@ -451,6 +451,42 @@ def measure_decode_norm(peak_gbs: float, reps: int = 200) -> dict:
     return out
 
 
+def measure_multi(peak_gbs: float, reps: int = 50, T: int = 4) -> dict:
+    """Multi-token decode (speculative drafts): the Nemotron-H layer, 64
+    sequences x T = 4 draft tokens, every token's state stored into its own
+    slot (a cache of 64 + 64 T slots)."""
+    import torch
+    import mamba_recurrent_state_b200 as m2
+    import m2synth as S
+    from m2synth import torch_inputs as TI
+    from m2synth import workloads as W
+    w = W.WORKLOADS[1]
+    batch = w.batch
+    slots_n = batch * (T + 1)
+    shape = m2.Shape(w.H, w.P, w.N, w.G, w.K, w.state_dtype, w.act_dtype)
+    cache = m2.Cache(shape, slots_n)
+    t = TI.layer_tensors(w)
+    ssm = m2.SSMParams(t["A_log"], t["dt_bias"], t["D"])
+    conv = m2.ConvParams(t["conv_w"], t["conv_b"], 1)
+    d = TI.step_tensors(w, 0, rows=batch * T)
+    x, dt, z = (d[k].view(batch, T, -1) for k in ("xBC", "dt", "z"))
+    slots = torch.arange(batch, dtype=torch.int32, device="cuda")
+    dest = (batch + torch.arange(batch * T, dtype=torch.int32, device="cuda")).view(batch, T)
+    y = torch.empty((batch, T, w.H * w.P), dtype=torch.bfloat16, device="cuda")
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device="cuda")
+    fn = lambda: m2.state_update_multi(cache, ssm, conv, x, dt, slots, dest, z=z, y=y)
+    for _ in range(3):
+        fn()
+    us = statistics.median(_time_us(fn, flush, reps))
+    if cache.device_error() != 0:
+        raise RuntimeError("device error word set during the multi-token benchmark")
+    state = w.H * w.P * w.N * 2
+    bytes_ = batch * (state * (1 + T) + T * (w.conv_dim * 2 * 4 + w.H * 2 + 2 * w.H * w.P * 2))
+    return {"workload": f"Nemotron-H layer, {batch} sequences x {T} draft tokens, every token's state stored",
+            "us": us, "GBs": bytes_ / us / 1e3, "frac_hbm": bytes_ / us / 1e3 / peak_gbs,
+            "tokens_per_s": batch * T / us * 1e6}
+
+
 def measure_stack48(flush, reps: int = 10) -> dict:
     """Workload 2: one decode token for 384 sequences through 48 layers
     (36 GiB of bf16 state), one CUDA graph of 48 fused launches per token."""
@@ -639,6 +675,8 @@ def run_ours(args, world, rank, local):
         line["prefill"]["tensor_peak"] = f"{tpeak} TFLOP/s ({tkind} bf16_tflops)"
     if "norm" in sections:
         line["decode_norm"] = measure_decode_norm(peak)
+    if "multi" in sections:
+        line["multi_token"] = measure_multi(peak)
     if "longprompt" in sections:
         line["longprompt"] = measure_longprompt(flush, peak)
     if "stack48" in sections:

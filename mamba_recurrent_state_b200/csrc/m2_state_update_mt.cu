@@ -5,11 +5,11 @@
 // causal_conv1d_update tap (vllm.cpp issue #1311 "NemotronH runs the PREFILL
 // mamba kernels at decode", section "The divergence"), from the state and conv
 // window of slot_idx[b]. Speculative decoding verifies the T drafts afterwards
-// and keeps only an accepted prefix (the Nemotron-H-8B-Base-8K record lists
-// speculative decoding among the serving features), so the state and conv
-// window after token t are stored into cache slot token_slots[b*T + t] of the
-// same cache, and the input slot is only read: after verification the caller
-// adopts the slot of the last accepted token.
+// and keeps only an accepted prefix (the Nemotron-H-8B-Base-8K record notes
+// the engines serve NemotronH with MTP / EAGLE speculative decoding), so the
+// state and conv window after token t are stored into cache slot
+// token_slots[b*T + t] of the same cache, and the input slot is only read:
+// after verification the caller adopts the slot of the last accepted token.
 //
 // Work decomposition: one CTA of 256 threads per 64 state rows (the rows of
 // 64/P heads) of one sequence. The CTA stages its state tile (16 KB for bf16,
