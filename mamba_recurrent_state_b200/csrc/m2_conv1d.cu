@@ -175,6 +175,166 @@ conv1d_kernel(const ConvArgs a) {
     }
 }
 
+// ---- prefill conv with the input tile staged in shared memory ---------------
+//
+// For long sequences of 16-bit activations: a CTA of 128 threads owns 256
+// channels x 64 tokens. Warp 0 stages the 64 + K-1 input rows of the tile
+// (512 bytes each; the rows before the sequence start come from the slot's conv
+// cache) with bulk copies into shared memory, and every thread then computes 16
+// tokens of one 16-byte channel vector from shared memory.
+constexpr int kTileThreads = 128;
+constexpr int kTileCh = 256;   // channels per CTA
+constexpr int kTileTok = 64;   // tokens per tile
+constexpr uint64_t kTileWaitNs = 1000000000ull;
+
+template <typename OT, int K>
+__global__ void __launch_bounds__(kTileThreads) conv1d_tile_kernel(const ConvArgs a) {
+    using AT = bf16_t;
+    constexpr int VEC = Vec16<AT>::n;                    // 8 channels per vector
+    constexpr int NV = kTileCh / VEC;                    // 32 vectors per row
+    constexpr int TPT = kTileTok / (kTileThreads / NV);  // 8 tokens per thread
+    constexpr int ROWS = kTileTok + K - 1;
+    __shared__ __align__(128) AT s_rows[ROWS][kTileCh];
+    __shared__ __align__(8) uint64_t s_bar;
+
+    const int tid = threadIdx.x;
+    const int b = blockIdx.z;
+    const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kTileCh;
+    const int nch = static_cast<int>(a.conv_dim - c0 < kTileCh ? a.conv_dim - c0 : kTileCh);
+    const int64_t row0 = a.cu_seqlens ? static_cast<int64_t>(a.cu_seqlens[b]) : static_cast<int64_t>(b) * a.seqlen;
+    const int T = a.cu_seqlens ? a.cu_seqlens[b + 1] - a.cu_seqlens[b] : a.seqlen;
+    if (T <= 0) return;  // an empty sequence leaves its cache slot untouched
+    const int v = tid % NV;             // this thread's channel vector
+    const int tg = tid / NV;            // its token group within the tile
+    const bool vec_ok = v * VEC < nch;
+    const int32_t slot = a.slot_idx[b];
+    const AT* xb = static_cast<const AT*>(a.x) + row0 * a.x_stride;
+    OT* ob = static_cast<OT*>(a.out) + row0 * a.out_stride;
+    if (slot < 0) {  // padding row: zero output, cache untouched
+        float zeros[VEC] = {};
+        for (int t0 = blockIdx.y * kTileTok; t0 < T; t0 += gridDim.y * kTileTok)
+            for (int i = 0; i < TPT; ++i) {
+                const int t = t0 + tg * TPT + i;
+                if (t < T && vec_ok) store_vec<OT, VEC>(ob + t * a.out_stride + c0 + v * VEC, zeros);
+            }
+        return;
+    }
+    if (slot >= a.num_slots) {
+        if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0) record_error(a.error, M2_ERR_BAD_SLOT);
+        return;
+    }
+    AT* cache = static_cast<AT*>(a.conv) + static_cast<int64_t>(slot) * (K - 1) * a.conv_dim;
+
+    // weights and bias of the thread's 8 channels
+    float w[VEC][K];
+    float bias[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+        const int64_t c = c0 + v * VEC + e;
+        const bool ok = vec_ok;
+#pragma unroll
+        for (int k = 0; k < K; ++k) w[e][k] = ok ? to_f32(static_cast<const AT*>(a.w)[c * K + k]) : 0.f;
+        bias[e] = (ok && a.b) ? to_f32(static_cast<const AT*>(a.b)[c]) : 0.f;
+    }
+    if (tid == 0) {
+        mbar_init(&s_bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    float out_max = 0.f;
+    uint32_t phase = 0;
+    bool ok = true;
+#pragma unroll 1
+    for (int t0 = blockIdx.y * kTileTok; t0 < T && ok; t0 += gridDim.y * kTileTok) {
+        // stage rows t0-K+1 .. t0+63 (only those inside the sequence or, before
+        // its start, in the conv cache); rows past the end are never read
+        if (tid < 32) {  // warp 0: lane 0 sets the byte count, then the lanes issue the rows
+            const int r_end = min(ROWS, T - t0 + K - 1);
+            if (tid == 0) mbar_arrive_expect_tx(&s_bar, static_cast<uint32_t>(r_end) * nch * sizeof(AT));
+            __syncwarp();
+            for (int r = tid; r < r_end; r += 32) {
+                const int t = t0 - (K - 1) + r;
+                const AT* src = t >= 0 ? xb + t * a.x_stride + c0 : cache + (K - 1 + t) * a.conv_dim + c0;
+                bulk_g2s(&s_rows[r][0], src, static_cast<uint32_t>(nch) * sizeof(AT), &s_bar);
+            }
+        }
+        ok = mbar_wait_bounded(&s_bar, phase, kTileWaitNs);
+        phase ^= 1;
+        if (!__syncthreads_and(ok)) {
+            if (tid == 0) record_error(a.error, M2_ERR_TIMEOUT);
+            mbar_wait_bounded(&s_bar, phase ^ 1, kTileWaitNs);  // let this CTA's copies land
+            return;
+        }
+        if (vec_ok) {
+            // window of token t0 + tg*8 + i: staged rows tg*8 + i .. tg*8 + i + K-1
+            float hist[K - 1][VEC];
+#pragma unroll
+            for (int j = 0; j < K - 1; ++j) unpack16<AT>(*reinterpret_cast<const uint4*>(&s_rows[tg * TPT + j][v * VEC]), hist[j]);
+#pragma unroll
+            for (int i = 0; i < TPT; ++i) {
+                const int t = t0 + tg * TPT + i;
+                if (t >= T) break;
+                float cur[VEC];
+                unpack16<AT>(*reinterpret_cast<const uint4*>(&s_rows[tg * TPT + i + K - 1][v * VEC]), cur);
+                float o[VEC];
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) {
+                    float acc = bias[e];
+#pragma unroll
+                    for (int k = 0; k < K - 1; ++k) acc = fmaf(w[e][k], hist[k][e], acc);
+                    acc = fmaf(w[e][K - 1], cur[e], acc);
+                    o[e] = a.activation ? silu_f32(acc) : acc;
+                }
+                if constexpr (std::is_same<OT, f16_t>::value) {
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) out_max = fmaxf(out_max, fabsf(o[e]));
+                }
+                store_vec<OT, VEC>(ob + t * a.out_stride + c0 + v * VEC, o);
+#pragma unroll
+                for (int k = 0; k < K - 2; ++k) {
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) hist[k][e] = hist[k + 1][e];
+                }
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) hist[K - 2][e] = cur[e];
+            }
+        }
+        __syncthreads();  // the next tile's copies overwrite s_rows
+    }
+    if (out_max >= 65520.f) record_error(a.error, M2_ERR_RANGE);  // beyond fp16 (rounds to inf)
+    if (blockIdx.y == 0 && tg == 0 && vec_ok) {
+        // new cache row k = raw input of token T-(K-1)+k: from the input when
+        // that token exists, else old cache row k + T (read before it is written)
+#pragma unroll
+        for (int k = 0; k < K - 1; ++k) {
+            const int t = T - (K - 1) + k;
+            const int64_t c = c0 + v * VEC;
+            const uint4 val = t >= 0 ? *reinterpret_cast<const uint4*>(xb + t * a.x_stride + c)
+                                     : *reinterpret_cast<const uint4*>(cache + (k + T) * a.conv_dim + c);
+            *reinterpret_cast<uint4*>(cache + k * a.conv_dim + c) = val;
+        }
+    }
+}
+
+template <typename OT>
+cudaError_t conv_tile_by_k(const ConvArgs& a, cudaStream_t s) {
+    const int64_t tiles = std::min<int64_t>(std::max<int64_t>((a.seqlen + kTileTok - 1) / kTileTok, 1), 65535);
+    const dim3 grid(static_cast<unsigned>((a.conv_dim + kTileCh - 1) / kTileCh), static_cast<unsigned>(tiles),
+                    static_cast<unsigned>(a.batch));
+    switch (a.K) {
+        case 2: conv1d_tile_kernel<OT, 2><<<grid, kTileThreads, 0, s>>>(a); break;
+        case 3: conv1d_tile_kernel<OT, 3><<<grid, kTileThreads, 0, s>>>(a); break;
+        case 4: conv1d_tile_kernel<OT, 4><<<grid, kTileThreads, 0, s>>>(a); break;
+        case 5: conv1d_tile_kernel<OT, 5><<<grid, kTileThreads, 0, s>>>(a); break;
+        case 6: conv1d_tile_kernel<OT, 6><<<grid, kTileThreads, 0, s>>>(a); break;
+        case 7: conv1d_tile_kernel<OT, 7><<<grid, kTileThreads, 0, s>>>(a); break;
+        case 8: conv1d_tile_kernel<OT, 8><<<grid, kTileThreads, 0, s>>>(a); break;
+        default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
 template <typename AT, typename OT>
 cudaError_t conv_by_k(const ConvArgs& a, cudaStream_t s) {
     constexpr int VEC = Vec16<AT>::n;
@@ -218,6 +378,12 @@ __global__ void __launch_bounds__(256) zero_slots_kernel(const ZeroArgs a) {
 }  // namespace
 
 cudaError_t launch_conv1d_update(const ConvArgs& a, cudaStream_t s) {
+    // long sequences of bf16 activations: the shared-memory tile kernel
+    if (a.act_bf16 && a.seqlen >= kTileTok) {
+        if (a.out_dtype == M2_BF16) return conv_tile_by_k<bf16_t>(a, s);
+        if (a.out_dtype == M2_F16) return conv_tile_by_k<f16_t>(a, s);
+        return conv_tile_by_k<float>(a, s);
+    }
     if (a.act_bf16) {
         if (a.out_dtype == M2_BF16) return conv_by_k<bf16_t, bf16_t>(a, s);
         if (a.out_dtype == M2_F16) return conv_by_k<bf16_t, f16_t>(a, s);
