@@ -14,12 +14,13 @@
 // Work decomposition: one CTA of 256 threads per 64 state rows (the rows of
 // 64/P heads) of one sequence. The CTA stages its state tile (16 KB for bf16,
 // N = 128) and the conv rows of its x channels and of the group's B/C channels
-// with bulk copies, loads the T raw inputs, and then, token by token, runs the
-// conv tap (one thread per 16-byte channel vector; the group's B/C conv is
-// computed by every CTA of the group), the state update on the tile in shared
-// memory (rounded to the storage dtype after every token, exactly as T
-// separate decode steps store it), the y reduction, and the stores of the
-// token's state and conv rows. The first CTA of each group writes the group's
+// with bulk copies, loads the T raw inputs, computes the conv tap of every
+// (token, 16-byte channel vector) at once (the group's B/C conv is computed by
+// every CTA of the group), and then runs the T state updates on the tile in
+// shared memory (rounded to the storage dtype after every token, exactly as T
+// separate decode steps store it): each thread keeps the same state vectors for
+// all tokens, so the token loop needs no barrier. y and every token's conv
+// rows are stored at the end. The first CTA of each group writes the group's
 // B/C conv rows; no CTA writes the input slot, so nothing races with the reads.
 #include <cuda_runtime.h>
 
@@ -35,7 +36,7 @@ constexpr int kMtMaxHeads = kMtRows / 8 + 1;
 constexpr uint64_t kMtWaitNs = 1000000000ull;
 
 template <typename ST, typename AT, int N>
-__global__ void __launch_bounds__(kMtThreads) mt_decode_kernel(const MtArgs a) {
+__global__ void __launch_bounds__(kMtThreads, 4) mt_decode_kernel(const MtArgs a) {
     constexpr int EPV = Vec16<ST>::n;        // state elements per 16-byte vector
     constexpr int LPR = N / EPV;             // lanes per state row
     static_assert(LPR >= 1 && LPR <= 32 && 32 % LPR == 0, "row must fit a warp");
@@ -45,21 +46,24 @@ __global__ void __launch_bounds__(kMtThreads) mt_decode_kernel(const MtArgs a) {
     constexpr int AV = Vec16<AT>::n;         // activation elements per 16-byte vector
     constexpr int XV = kMtRows / AV;         // x-channel vectors of the tile
     constexpr int BV = N / AV;               // vectors of one B (or C) segment
+    constexpr int NVEC = XV + 2 * BV;        // conv vectors per token
 
     const int T = a.T;
     const int K = a.K;
     const int W = K - 1 + T;                 // window rows: K-1 cached, then T raw inputs
+    // dynamic shared memory: [state tile | raw x window | raw B|C window |
+    //                         post-conv x, B, C and y of every token (fp32)]
     extern __shared__ __align__(128) uint8_t s_dyn[];
     uint8_t* s_state = s_dyn;                                        // [64][N] ST
-    AT* s_xw = reinterpret_cast<AT*>(s_dyn + TILE_BYTES);            // [W][64] raw x window
-    AT* s_bcw = s_xw + static_cast<size_t>(W) * kMtRows;              // [W][2N] raw B|C window
+    AT* s_xw = reinterpret_cast<AT*>(s_dyn + TILE_BYTES);            // [W][64]
+    AT* s_bcw = s_xw + static_cast<size_t>(W) * kMtRows;              // [W][2N]
+    float* s_x = reinterpret_cast<float*>(s_bcw + static_cast<size_t>(W) * 2 * N);  // [T][64]
+    float* s_B = s_x + T * kMtRows;                                  // [T][N]
+    float* s_C = s_B + T * N;                                        // [T][N]
+    float* s_y = s_C + T * N;                                        // [T][64]
     __shared__ __align__(8) uint64_t s_bar;
-    __shared__ __align__(16) float s_x[kMtRows];                     // post-conv x of the token
-    __shared__ __align__(16) float s_B[N];
-    __shared__ __align__(16) float s_C[N];
-    __shared__ float s_y[kMtRows];
-    __shared__ float s_dt[kMtMaxHeads];
-    __shared__ float s_dA[kMtMaxHeads];
+    __shared__ float s_dt[kMaxDraftTokens][kMtMaxHeads];
+    __shared__ float s_dA[kMaxDraftTokens][kMtMaxHeads];
     __shared__ float s_D[kMtMaxHeads];
     __shared__ int s_fail;
 
@@ -78,6 +82,18 @@ __global__ void __launch_bounds__(kMtThreads) mt_decode_kernel(const MtArgs a) {
     const bool bc_writer = (r0 % (static_cast<int64_t>(hpg) * P)) == 0;  // first CTA of the group
     const AT* xbase = static_cast<const AT*>(a.xBC) + static_cast<int64_t>(b) * T * a.xBC_stride;
     AT* ybase = static_cast<AT*>(a.y) + static_cast<int64_t>(b) * T * a.y_stride;
+    // channel of conv vector u (0 .. NVEC-1) and where its window column sits
+    auto vec_channel = [&](int u) -> int64_t {
+        return u < XV ? r0 + u * AV : (u - XV < BV ? cB + (u - XV) * AV : cC + (u - XV - BV) * AV);
+    };
+    auto vec_window = [&](int u, int& pitch) -> const AT* {
+        if (u < XV) {
+            pitch = kMtRows;
+            return s_xw + u * AV;
+        }
+        pitch = 2 * N;
+        return s_bcw + (u - XV) * AV;
+    };
 
     const int32_t slot = a.slot_idx[b];
     if (slot < 0) {  // padding row: y = 0 for every token, no state stored
@@ -106,47 +122,25 @@ __global__ void __launch_bounds__(kMtThreads) mt_decode_kernel(const MtArgs a) {
         }
     }
     __syncthreads();  // the barrier is initialised before any thread waits on it
-    // raw inputs of the T tokens (x channels of the tile, the group's B and C)
-    for (int i = tid; i < T * (XV + 2 * BV); i += kMtThreads) {
-        const int t = i / (XV + 2 * BV);
-        const int v = i % (XV + 2 * BV);
-        const AT* row = xbase + static_cast<int64_t>(t) * a.xBC_stride;
-        if (v < XV) {
-            *reinterpret_cast<uint4*>(s_xw + (K - 1 + t) * kMtRows + v * AV) =
-                *reinterpret_cast<const uint4*>(row + r0 + v * AV);
-        } else {
-            const int u = v - XV;  // 0 .. 2*BV-1: B then C
-            const int64_t c0 = (u < BV ? cB : cC - BV * AV) + u * AV;
-            *reinterpret_cast<uint4*>(s_bcw + (K - 1 + t) * 2 * N + u * AV) =
-                *reinterpret_cast<const uint4*>(row + c0);
-        }
+    // raw inputs of the T tokens (x channels of the tile, the group's B and C);
+    // the head scalars of every token
+    for (int i = tid; i < T * NVEC; i += kMtThreads) {
+        const int t = i / NVEC;
+        const int u = i % NVEC;
+        int pitch;
+        AT* dst = const_cast<AT*>(vec_window(u, pitch)) + (K - 1 + t) * pitch;
+        *reinterpret_cast<uint4*>(dst) =
+            *reinterpret_cast<const uint4*>(xbase + static_cast<int64_t>(t) * a.xBC_stride + vec_channel(u));
     }
-    // this thread's conv channel vector (fixed for all tokens): weights and bias
-    const int nvec = XV + 2 * BV;
-    const bool conv_thread = tid < nvec;
-    int64_t c_vec = 0;
-    const AT* win = nullptr;   // window column of the vector in shared memory
-    int win_pitch = 0;
-    float wt[AV][8];
-    float bias[AV];
-    if (conv_thread) {
-        if (tid < XV) {
-            c_vec = r0 + tid * AV;
-            win = s_xw + tid * AV;
-            win_pitch = kMtRows;
-        } else {
-            const int u = tid - XV;
-            c_vec = (u < BV ? cB : cC - BV * AV) + u * AV;
-            win = s_bcw + u * AV;
-            win_pitch = 2 * N;
-        }
-        const AT* wp = static_cast<const AT*>(a.conv_w) + c_vec * K;
-#pragma unroll
-        for (int e = 0; e < AV; ++e) {
-#pragma unroll
-            for (int k = 0; k < 8; ++k) wt[e][k] = k < K ? to_f32(wp[e * K + k]) : 0.f;
-            bias[e] = a.conv_b ? to_f32(static_cast<const AT*>(a.conv_b)[c_vec + e]) : 0.f;
-        }
+    for (int i = tid; i < T * n_heads; i += kMtThreads) {
+        const int t = i / n_heads;
+        const int hl = i % n_heads;
+        const int h = h_first + hl;
+        const float dtr = to_f32(static_cast<const AT*>(a.dt)[(static_cast<int64_t>(b) * T + t) * a.dt_stride + h]);
+        const float dt = softplus_f32(dtr + a.dt_bias[h]);
+        s_dt[t][hl] = dt;
+        s_dA[t][hl] = expf(dt * -expf(a.A_log[h]));
+        if (t == 0) s_D[hl] = a.D[h];
     }
     const bool wait_ok = mbar_wait_bounded(&s_bar, 0, kMtWaitNs);
     if (!wait_ok) s_fail = 1;
@@ -157,121 +151,125 @@ __global__ void __launch_bounds__(kMtThreads) mt_decode_kernel(const MtArgs a) {
         return;
     }
 
+    // ---- the conv tap of every (token, channel vector) at once: token t's
+    // window is rows t .. t+K-1
+    for (int i = tid; i < T * NVEC; i += kMtThreads) {
+        const int t = i / NVEC;
+        const int u = i % NVEC;
+        int pitch;
+        const AT* win = vec_window(u, pitch);
+        const int64_t c = vec_channel(u);
+        const AT* wp = static_cast<const AT*>(a.conv_w) + c * K;
+        float out[AV];
+#pragma unroll
+        for (int e = 0; e < AV; ++e) out[e] = a.conv_b ? to_f32(static_cast<const AT*>(a.conv_b)[c + e]) : 0.f;
+        for (int k = 0; k < K; ++k) {
+            float rv[AV];
+            unpack16<AT>(*reinterpret_cast<const uint4*>(win + (t + k) * pitch), rv);
+#pragma unroll
+            for (int e = 0; e < AV; ++e) out[e] = fmaf(to_f32(wp[e * K + k]), rv[e], out[e]);
+        }
+        float* dst = u < XV ? s_x + t * kMtRows + u * AV
+                            : (u - XV < BV ? s_B + t * N + (u - XV) * AV : s_C + t * N + (u - XV - BV) * AV);
+#pragma unroll
+        for (int e = 0; e < AV; ++e) dst[e] = a.activation ? silu_f32(out[e]) : out[e];
+    }
+    __syncthreads();
+
+    // ---- the T tokens: every thread keeps the same state vectors for all of
+    // them, so the token loop needs no barrier
     const int lane = tid & 31;
     const int e0 = (lane % LPR) * EPV;
     const int64_t HPN = HP * N;
     for (int t = 0; t < T; ++t) {
-        // ---- conv tap of token t (window rows t .. t+K-1) and the head scalars
-        if (conv_thread) {
-            float out[AV];
-#pragma unroll
-            for (int e = 0; e < AV; ++e) out[e] = bias[e];
-            for (int k = 0; k < K; ++k) {
-                float rv[AV];
-                unpack16<AT>(*reinterpret_cast<const uint4*>(win + (t + k) * win_pitch), rv);
-#pragma unroll
-                for (int e = 0; e < AV; ++e) out[e] = fmaf(wt[e][k], rv[e], out[e]);
-            }
-#pragma unroll
-            for (int e = 0; e < AV; ++e) {
-                const float o = a.activation ? silu_f32(out[e]) : out[e];
-                if (tid < XV) {
-                    s_x[tid * AV + e] = o;
-                } else {
-                    const int u = tid - XV;
-                    if (u < BV) s_B[u * AV + e] = o;
-                    else s_C[(u - BV) * AV + e] = o;
-                }
-            }
-        } else if (tid >= 224 && tid - 224 < n_heads) {
-            const int hl = tid - 224;
-            const int h = h_first + hl;
-            const float dtr = to_f32(static_cast<const AT*>(a.dt)[(static_cast<int64_t>(b) * T + t) * a.dt_stride + h]);
-            const float dt = softplus_f32(dtr + a.dt_bias[h]);
-            s_dt[hl] = dt;
-            s_dA[hl] = expf(dt * -expf(a.A_log[h]));
-            s_D[hl] = a.D[h];
-        }
-        __syncthreads();
-
-        // ---- state update of the tile, y partial sums, token state stores
         const int32_t dest = a.token_slots[static_cast<int64_t>(b) * T + t];
         const bool store = dest >= 0 && dest < a.num_slots;
         if (dest >= a.num_slots && tid == 0) record_error(a.error, M2_ERR_BAD_SLOT);
         ST* dtile = store ? static_cast<ST*>(a.ssm) + static_cast<int64_t>(dest) * HPN + r0 * N : nullptr;
-        float Bv[EPV], Cv[EPV];
-#pragma unroll
-        for (int e = 0; e < EPV; ++e) {
-            Bv[e] = s_B[e0 + e];
-            Cv[e] = s_C[e0 + e];
-        }
+        const float* Bt = s_B + t * N + e0;
+        const float* Ct = s_C + t * N + e0;
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
             const int v = i * kMtThreads + tid;
             const int row = v / LPR;
             const int hl = static_cast<int>((r0 + row) / P) - h_first;
-            const float dtx = s_dt[hl] * s_x[row];
-            const float dA = s_dA[hl];
+            const float xr = s_x[t * kMtRows + row];
+            const float dtx = s_dt[t][hl] * xr;
+            const float dA = s_dA[t][hl];
             uint4* sp = reinterpret_cast<uint4*>(s_state + static_cast<uint32_t>(v) * 16u);
             float st[EPV];
             unpack16<ST>(*sp, st);
             float acc = 0.f;
 #pragma unroll
             for (int e = 0; e < EPV; ++e) {
-                st[e] = fmaf(st[e], dA, dtx * Bv[e]);
-                acc = fmaf(st[e], Cv[e], acc);
+                st[e] = fmaf(st[e], dA, dtx * Bt[e]);
+                acc = fmaf(st[e], Ct[e], acc);
             }
             const uint4 packed = pack16<ST>(st);  // the stored state, rounded once per token
             *sp = packed;
             if (store) st_stream(dtile + static_cast<int64_t>(row) * N + e0, packed);
 #pragma unroll
             for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-            if ((lane % LPR) == 0) s_y[row] = acc + s_D[hl] * s_x[row];
+            if ((lane % LPR) == 0) s_y[t * kMtRows + row] = acc + s_D[hl] * xr;
         }
-        __syncthreads();
-
-        // ---- gated y of the token; the token's conv window into the destination slot
-        if (tid < kMtRows) {
-            float yv = s_y[tid];
-            if (a.z) {
-                const AT* zr = static_cast<const AT*>(a.z) + (static_cast<int64_t>(b) * T + t) * a.z_stride;
-                yv *= silu_f32(to_f32(zr[r0 + tid]));
-            }
-            ybase[static_cast<int64_t>(t) * a.y_stride + r0 + tid] = from_f32<AT>(yv);
-        }
-        if (store && conv_thread && (tid < XV || bc_writer)) {
-            // new row k of the destination = window row t+1+k (raw inputs, exact copies)
-            AT* conv_out = static_cast<AT*>(a.conv) + static_cast<int64_t>(dest) * (K - 1) * cd;
-            for (int k = 0; k < K - 1; ++k)
-                *reinterpret_cast<uint4*>(conv_out + k * cd + c_vec) =
-                    *reinterpret_cast<const uint4*>(win + (t + 1 + k) * win_pitch);
-        }
-        // the next token's conv overwrites s_x / s_B / s_C read above
-        __syncthreads();
     }
+    __syncthreads();
+
+    // ---- gated y of every token; every token's conv window into its destination
+    for (int i = tid; i < T * kMtRows; i += kMtThreads) {
+        const int t = i / kMtRows;
+        const int row = i % kMtRows;
+        float yv = s_y[i];
+        if (a.z) {
+            const AT* zr = static_cast<const AT*>(a.z) + (static_cast<int64_t>(b) * T + t) * a.z_stride;
+            yv *= silu_f32(to_f32(zr[r0 + row]));
+        }
+        ybase[static_cast<int64_t>(t) * a.y_stride + r0 + row] = from_f32<AT>(yv);
+    }
+    const int nwrite = bc_writer ? NVEC : XV;  // the group's first CTA also writes B/C
+    for (int i = tid; i < T * nwrite * (K - 1); i += kMtThreads) {
+        const int k = i % (K - 1);
+        const int u = (i / (K - 1)) % nwrite;
+        const int t = i / ((K - 1) * nwrite);
+        const int32_t dest = a.token_slots[static_cast<int64_t>(b) * T + t];
+        if (dest < 0 || dest >= a.num_slots) continue;
+        int pitch;
+        const AT* win = vec_window(u, pitch);
+        // new row k of the destination = window row t+1+k (raw inputs, exact copies)
+        AT* conv_out = static_cast<AT*>(a.conv) + static_cast<int64_t>(dest) * (K - 1) * cd;
+        *reinterpret_cast<uint4*>(conv_out + k * cd + vec_channel(u)) =
+            *reinterpret_cast<const uint4*>(win + (t + 1 + k) * pitch);
+    }
+}
+
+// One kernel instantiation with its own once-per-device attribute setup.
+template <typename ST, typename AT, int N>
+cudaError_t mt_launch(const MtArgs& a, size_t smem, size_t smem_max, dim3 grid, cudaStream_t s) {
+    static AttrOnce attrs;
+    const cudaError_t e = attrs.ensure([&] {
+        return cudaFuncSetAttribute(mt_decode_kernel<ST, AT, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(smem_max));
+    });
+    if (e != cudaSuccess) return e;
+    mt_decode_kernel<ST, AT, N><<<grid, kMtThreads, smem, s>>>(a);
+    return cudaGetLastError();
 }
 
 template <typename ST, typename AT>
 cudaError_t mt_by_n(const MtArgs& a, cudaStream_t s) {
+    // tile + raw windows + per-token fp32 x, B, C, y (the largest N, K and T)
     const size_t smem_max = static_cast<size_t>(kMtRows) * 256 * sizeof(ST) +
-                            static_cast<size_t>(7 + kMaxDraftTokens) * (kMtRows + 2 * 256) * sizeof(AT);
+                            static_cast<size_t>(7 + kMaxDraftTokens) * (kMtRows + 2 * 256) * sizeof(AT) +
+                            static_cast<size_t>(kMaxDraftTokens) * (2 * kMtRows + 2 * 256) * sizeof(float);
     const size_t tile = static_cast<size_t>(kMtRows) * a.N * sizeof(ST);
-    const size_t smem = tile + static_cast<size_t>(a.K - 1 + a.T) * (kMtRows + 2 * a.N) * sizeof(AT);
+    const size_t smem = tile + static_cast<size_t>(a.K - 1 + a.T) * (kMtRows + 2 * a.N) * sizeof(AT) +
+                        static_cast<size_t>(a.T) * (2 * kMtRows + 2 * a.N) * sizeof(float);
     const dim3 grid(static_cast<unsigned>(static_cast<int64_t>(a.H) * a.P / kMtRows), static_cast<unsigned>(a.batch));
-    auto launch = [&](auto kern) -> cudaError_t {
-        static AttrOnce attrs;
-        const cudaError_t e = attrs.ensure([&] {
-            return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem_max));
-        });
-        if (e != cudaSuccess) return e;
-        kern<<<grid, kMtThreads, smem, s>>>(a);
-        return cudaGetLastError();
-    };
     switch (a.N) {
-        case 64: return launch(mt_decode_kernel<ST, AT, 64>);
-        case 128: return launch(mt_decode_kernel<ST, AT, 128>);
+        case 64: return mt_launch<ST, AT, 64>(a, smem, smem_max, grid, s);
+        case 128: return mt_launch<ST, AT, 128>(a, smem, smem_max, grid, s);
         case 256:
-            if constexpr (sizeof(ST) == 2) return launch(mt_decode_kernel<ST, AT, 256>);
+            if constexpr (sizeof(ST) == 2) return mt_launch<ST, AT, 256>(a, smem, smem_max, grid, s);
             return cudaErrorInvalidValue;
         default: return cudaErrorInvalidValue;
     }
