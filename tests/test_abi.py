@@ -99,3 +99,45 @@ def test_no_torch_types_in_the_abi():
         code = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
         for banned in ("at::", "c10::", "torch", "Tensor"):
             assert banned not in code, banned
+
+
+def test_newer_entry_points_validate_on_the_host(lib):
+    """The variable-length, norm, multi-token and mixed entry points reject bad
+    arguments (or return early on empty work) before touching a GPU: a cache
+    wrapped around made-up aligned addresses is never dereferenced here."""
+    shape = m2.Shape(128, 64, 128, 8, 4, m2.M2_BF16, m2.M2_BF16).c()
+    cache = m2.m2_cache()
+    assert lib.m2_cache_wrap(ctypes.byref(shape), 4, 0x100000, 0x200000, None, ctypes.byref(cache)) == m2.M2_OK
+    ssm = m2.m2_ssm_params(0x300000, 0x300100, 0x300200)
+    conv = m2.m2_conv_params(0x400000, None, 1)
+    norm = m2.m2_norm_params(0x500000, 1e-5)
+    cd, hp = 10240, 8192
+    buf = 0x600000  # aligned made-up buffer address
+    # the norm is fused only with the conv
+    assert lib.m2_state_update_norm(ctypes.byref(cache), ctypes.byref(ssm), None, ctypes.byref(norm), 1, buf,
+                                    cd, buf, 128, buf, hp, buf, hp, buf, None) == m2.M2_ERR_INVALID_ARG
+    # multi-token decode: T = 0 is a no-op, T above 16 is not supported, an
+    # unaligned row stride is an argument error
+    args = (buf, cd, buf, 128, buf, hp, buf, hp, buf, buf, None)
+    assert lib.m2_state_update_multi(ctypes.byref(cache), ctypes.byref(ssm), ctypes.byref(conv), 2, 0,
+                                     *args) == m2.M2_OK
+    assert lib.m2_state_update_multi(ctypes.byref(cache), ctypes.byref(ssm), ctypes.byref(conv), 2, 17,
+                                     *args) == m2.M2_ERR_UNSUPPORTED
+    assert lib.m2_state_update_multi(ctypes.byref(cache), ctypes.byref(ssm), ctypes.byref(conv), 2, 4,
+                                     buf, cd + 1, *args[2:]) == m2.M2_ERR_INVALID_ARG
+    # varlen scan and conv: empty batches return OK, oversized or missing offsets are refused
+    scan_tail = (128, buf, m2.M2_F16, cd, buf, 128, buf, hp, buf, hp, buf, None, None)
+    assert lib.m2_chunk_scan_varlen(ctypes.byref(cache), ctypes.byref(ssm), 0, None, 0, 0, *scan_tail) == m2.M2_OK
+    assert lib.m2_chunk_scan_varlen(ctypes.byref(cache), ctypes.byref(ssm), 1, buf, 2**31, 2**31 - 1,
+                                    *scan_tail) == m2.M2_ERR_UNSUPPORTED
+    assert lib.m2_chunk_scan_varlen(ctypes.byref(cache), ctypes.byref(ssm), 2, None, 100, 50,
+                                    *scan_tail) == m2.M2_ERR_INVALID_ARG
+    assert lib.m2_chunk_scan_varlen_static(ctypes.byref(cache), ctypes.byref(ssm), 2, None, 100, 50,
+                                           *scan_tail) == m2.M2_ERR_INVALID_ARG
+    assert lib.m2_conv1d_update_varlen(ctypes.byref(cache), ctypes.byref(conv), 2, None, 100, 50, buf, cd, buf,
+                                       m2.M2_F16, cd, buf, None) == m2.M2_ERR_INVALID_ARG
+    # the mixed step needs the conv parameters; with nothing to do it returns OK
+    assert lib.m2_mixed_step(ctypes.byref(cache), ctypes.byref(ssm), None, None, None,
+                             None) == m2.M2_ERR_INVALID_ARG
+    assert lib.m2_mixed_step(ctypes.byref(cache), ctypes.byref(ssm), ctypes.byref(conv), None, None,
+                             None) == m2.M2_OK
