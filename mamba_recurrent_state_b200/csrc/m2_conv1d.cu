@@ -181,10 +181,13 @@ conv1d_kernel(const ConvArgs a) {
 // channels x 64 tokens. Warp 0 stages the 64 + K-1 input rows of the tile
 // (512 bytes each; the rows before the sequence start come from the slot's conv
 // cache) with bulk copies into shared memory, and every thread then computes 16
-// tokens of one 16-byte channel vector from shared memory.
+// tokens of one 16-byte channel vector from shared memory. A CTA walks several
+// tiles of its sequence with two buffers: the next tile's rows land while the
+// current one is computed.
 constexpr int kTileThreads = 128;
 constexpr int kTileCh = 256;   // channels per CTA
 constexpr int kTileTok = 64;   // tokens per tile
+constexpr int kMaxTilesPerCta = 8;  // token tiles a CTA walks, double-buffered (at most)
 constexpr uint64_t kTileWaitNs = 1000000000ull;
 
 template <typename OT, int K>
@@ -194,8 +197,11 @@ __global__ void __launch_bounds__(kTileThreads) conv1d_tile_kernel(const ConvArg
     constexpr int NV = kTileCh / VEC;                    // 32 vectors per row
     constexpr int TPT = kTileTok / (kTileThreads / NV);  // 8 tokens per thread
     constexpr int ROWS = kTileTok + K - 1;
-    __shared__ __align__(128) AT s_rows[ROWS][kTileCh];
-    __shared__ __align__(8) uint64_t s_bar;
+    // two tile buffers (dynamic shared memory): the next tile's rows land while
+    // this one is computed
+    extern __shared__ __align__(128) uint8_t s_conv_dyn[];
+    AT (*s_buf)[ROWS][kTileCh] = reinterpret_cast<AT (*)[ROWS][kTileCh]>(s_conv_dyn);
+    __shared__ __align__(8) uint64_t s_bar[2];
 
     const int tid = threadIdx.x;
     const int b = blockIdx.z;
@@ -237,35 +243,50 @@ __global__ void __launch_bounds__(kTileThreads) conv1d_tile_kernel(const ConvArg
         bias[e] = (ok && a.b) ? to_f32(static_cast<const AT*>(a.b)[c]) : 0.f;
     }
     if (tid == 0) {
-        mbar_init(&s_bar, 1);
+        mbar_init(&s_bar[0], 1);
+        mbar_init(&s_bar[1], 1);
         fence_mbar_init();
     }
     __syncthreads();
 
-    float out_max = 0.f;
-    uint32_t phase = 0;
-    bool ok = true;
-#pragma unroll 1
-    for (int t0 = blockIdx.y * kTileTok; t0 < T && ok; t0 += gridDim.y * kTileTok) {
-        // stage rows t0-K+1 .. t0+63 (only those inside the sequence or, before
-        // its start, in the conv cache); rows past the end are never read
-        if (tid < 32) {  // warp 0: lane 0 sets the byte count, then the lanes issue the rows
+    // this CTA's tiles: t0 = (blockIdx.y + j * gridDim.y) * 64, j = 0, 1, ...
+    const int stride = gridDim.y * kTileTok;
+    // stage rows t0-K+1 .. t0+63 of a tile into buffer q (only rows inside the
+    // sequence or, before its start, in the conv cache; rows past the end are
+    // never read); warp 0: lane 0 sets the byte count, then the lanes issue rows
+    auto issue = [&](int t0, int q) {
+        if (tid < 32) {
             const int r_end = min(ROWS, T - t0 + K - 1);
-            if (tid == 0) mbar_arrive_expect_tx(&s_bar, static_cast<uint32_t>(r_end) * nch * sizeof(AT));
+            if (tid == 0) mbar_arrive_expect_tx(&s_bar[q], static_cast<uint32_t>(r_end) * nch * sizeof(AT));
             __syncwarp();
             for (int r = tid; r < r_end; r += 32) {
                 const int t = t0 - (K - 1) + r;
                 const AT* src = t >= 0 ? xb + t * a.x_stride + c0 : cache + (K - 1 + t) * a.conv_dim + c0;
-                bulk_g2s(&s_rows[r][0], src, static_cast<uint32_t>(nch) * sizeof(AT), &s_bar);
+                bulk_g2s(&s_buf[q][r][0], src, static_cast<uint32_t>(nch) * sizeof(AT), &s_bar[q]);
             }
         }
-        ok = mbar_wait_bounded(&s_bar, phase, kTileWaitNs);
-        phase ^= 1;
+    };
+    const int first = blockIdx.y * kTileTok;
+    if (first < T) issue(first, 0);
+    if (first + stride < T) issue(first + stride, 1);
+
+    float out_max = 0.f;
+    uint32_t phase[2] = {0, 0};
+    int in_flight[2] = {first < T ? 1 : 0, first + stride < T ? 1 : 0};
+#pragma unroll 1
+    for (int j = 0, t0 = first; t0 < T; ++j, t0 += stride) {
+        const int q = j & 1;
+        const bool ok = mbar_wait_bounded(&s_bar[q], phase[q], kTileWaitNs);
+        phase[q] ^= 1;
+        in_flight[q] = 0;
         if (!__syncthreads_and(ok)) {
             if (tid == 0) record_error(a.error, M2_ERR_TIMEOUT);
-            mbar_wait_bounded(&s_bar, phase ^ 1, kTileWaitNs);  // let this CTA's copies land
+            // let this CTA's copies land (bounded) before its shared memory goes
+            if (!ok) mbar_wait_bounded(&s_bar[q], phase[q] ^ 1, kTileWaitNs);
+            if (in_flight[q ^ 1]) mbar_wait_bounded(&s_bar[q ^ 1], phase[q ^ 1], kTileWaitNs);
             return;
         }
+        AT (*s_rows)[kTileCh] = s_buf[q];
         if (vec_ok) {
             // window of token t0 + tg*8 + i: staged rows tg*8 + i .. tg*8 + i + K-1
             float hist[K - 1][VEC];
@@ -300,7 +321,11 @@ __global__ void __launch_bounds__(kTileThreads) conv1d_tile_kernel(const ConvArg
                 for (int e = 0; e < VEC; ++e) hist[K - 2][e] = cur[e];
             }
         }
-        __syncthreads();  // the next tile's copies overwrite s_rows
+        __syncthreads();  // every thread is done with buffer q
+        if (t0 + 2 * stride < T) {  // the tile after next lands in buffer q
+            issue(t0 + 2 * stride, q);
+            in_flight[q] = 1;
+        }
     }
     if (out_max >= 65520.f) record_error(a.error, M2_ERR_RANGE);  // beyond fp16 (rounds to inf)
     if (blockIdx.y == 0 && tg == 0 && vec_ok) {
@@ -317,22 +342,43 @@ __global__ void __launch_bounds__(kTileThreads) conv1d_tile_kernel(const ConvArg
     }
 }
 
+template <typename OT, int K>
+cudaError_t conv_tile_launch(const ConvArgs& a, dim3 grid, cudaStream_t s) {
+    constexpr size_t smem = 2 * static_cast<size_t>(kTileTok + K - 1) * kTileCh * sizeof(bf16_t);
+    static AttrOnce attrs;
+    const cudaError_t e = attrs.ensure([] {
+        return cudaFuncSetAttribute(conv1d_tile_kernel<OT, K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(smem));
+    });
+    if (e != cudaSuccess) return e;
+    conv1d_tile_kernel<OT, K><<<grid, kTileThreads, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
 template <typename OT>
 cudaError_t conv_tile_by_k(const ConvArgs& a, cudaStream_t s) {
-    const int64_t tiles = std::min<int64_t>(std::max<int64_t>((a.seqlen + kTileTok - 1) / kTileTok, 1), 65535);
-    const dim3 grid(static_cast<unsigned>((a.conv_dim + kTileCh - 1) / kTileCh), static_cast<unsigned>(tiles),
-                    static_cast<unsigned>(a.batch));
+    // Each CTA walks up to 8 token tiles of its sequence, double-buffered, as
+    // long as the grid keeps about six CTAs per SM (three resident, two waves).
+    // Measured on the 8 x 2048 Nemotron-H prefill: one tile per CTA 221 us,
+    // 2 tiles 205 us, 4 tiles 196 us, 8 tiles 192 us.
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        sms = 148;
+    const int64_t ch_blocks = (a.conv_dim + kTileCh - 1) / kTileCh;
+    const int64_t tiles = std::max<int64_t>((a.seqlen + kTileTok - 1) / kTileTok, 1);
+    const int64_t per_cta = std::clamp<int64_t>(ch_blocks * a.batch * tiles / (6LL * sms), 1, kMaxTilesPerCta);
+    const int64_t ctas_y = std::min<int64_t>((tiles + per_cta - 1) / per_cta, 65535);
+    const dim3 grid(static_cast<unsigned>(ch_blocks), static_cast<unsigned>(ctas_y), static_cast<unsigned>(a.batch));
     switch (a.K) {
-        case 2: conv1d_tile_kernel<OT, 2><<<grid, kTileThreads, 0, s>>>(a); break;
-        case 3: conv1d_tile_kernel<OT, 3><<<grid, kTileThreads, 0, s>>>(a); break;
-        case 4: conv1d_tile_kernel<OT, 4><<<grid, kTileThreads, 0, s>>>(a); break;
-        case 5: conv1d_tile_kernel<OT, 5><<<grid, kTileThreads, 0, s>>>(a); break;
-        case 6: conv1d_tile_kernel<OT, 6><<<grid, kTileThreads, 0, s>>>(a); break;
-        case 7: conv1d_tile_kernel<OT, 7><<<grid, kTileThreads, 0, s>>>(a); break;
-        case 8: conv1d_tile_kernel<OT, 8><<<grid, kTileThreads, 0, s>>>(a); break;
+        case 2: return conv_tile_launch<OT, 2>(a, grid, s);
+        case 3: return conv_tile_launch<OT, 3>(a, grid, s);
+        case 4: return conv_tile_launch<OT, 4>(a, grid, s);
+        case 5: return conv_tile_launch<OT, 5>(a, grid, s);
+        case 6: return conv_tile_launch<OT, 6>(a, grid, s);
+        case 7: return conv_tile_launch<OT, 7>(a, grid, s);
+        case 8: return conv_tile_launch<OT, 8>(a, grid, s);
         default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 template <typename AT, typename OT>
