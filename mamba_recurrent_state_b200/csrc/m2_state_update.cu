@@ -86,34 +86,6 @@ __device__ __forceinline__ void st_cluster_f32(float* local, uint32_t rank, floa
 
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // bounded waits: one second
 
-// Sums VPT row partials over the LPR lanes that share each row. For VPT = 4
-// the first two levels exchange only the halves each lane keeps
-// (reduce-scatter), so 4 rows cost 5 shuffles instead of 16. On return the
-// lanes with (lane % (LPR/VPT)) == 0 hold the sum of row `which`.
-template <int LPR, int VPT>
-__device__ __forceinline__ float reduce_rows(const float (&acc)[VPT], int lane, int& which) {
-    static_assert(VPT == 1 || VPT == 4, "one or four rows per thread");
-    static_assert(LPR >= VPT, "reduce-scatter needs at least one lane per row");
-    if constexpr (VPT == 1) {
-        float v = acc[0];
-#pragma unroll
-        for (int off = LPR / 2; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-        which = 0;
-        return v;
-    } else {
-        const bool hi1 = (lane & (LPR / 2)) != 0;   // keeps rows 2,3 instead of 0,1
-        const float s0 = hi1 ? acc[0] : acc[2];
-        const float s1 = hi1 ? acc[1] : acc[3];
-        const float k0 = (hi1 ? acc[2] : acc[0]) + __shfl_xor_sync(0xffffffffu, s0, LPR / 2);
-        const float k1 = (hi1 ? acc[3] : acc[1]) + __shfl_xor_sync(0xffffffffu, s1, LPR / 2);
-        const bool hi2 = (lane & (LPR / 4)) != 0;   // keeps the odd row of the pair
-        float v = (hi2 ? k1 : k0) + __shfl_xor_sync(0xffffffffu, hi2 ? k0 : k1, LPR / 4);
-#pragma unroll
-        for (int off = LPR / 8; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-        which = (hi1 ? 2 : 0) + (hi2 ? 1 : 0);
-        return v;
-    }
-}
 
 // Slot-independent inputs of one conv vector (AV channels c0..): the raw
 // input, the bias and, for K = 4, the AV x K weight block, which is exactly

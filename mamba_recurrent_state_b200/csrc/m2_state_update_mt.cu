@@ -36,7 +36,7 @@ constexpr int kMtMaxHeads = kMtRows / 8 + 1;
 constexpr uint64_t kMtWaitNs = 1000000000ull;
 
 template <typename ST, typename AT, int N>
-__global__ void __launch_bounds__(kMtThreads, 4) mt_decode_kernel(const MtArgs a) {
+__global__ void __launch_bounds__(kMtThreads, 3) mt_decode_kernel(const MtArgs a) {
     constexpr int EPV = Vec16<ST>::n;        // state elements per 16-byte vector
     constexpr int LPR = N / EPV;             // lanes per state row
     static_assert(LPR >= 1 && LPR <= 32 && 32 % LPR == 0, "row must fit a warp");
@@ -161,56 +161,108 @@ __global__ void __launch_bounds__(kMtThreads, 4) mt_decode_kernel(const MtArgs a
         const int64_t c = vec_channel(u);
         const AT* wp = static_cast<const AT*>(a.conv_w) + c * K;
         float out[AV];
+        if (a.conv_b) {
+            unpack16<AT>(__ldg(reinterpret_cast<const uint4*>(static_cast<const AT*>(a.conv_b) + c)), out);
+        } else {
 #pragma unroll
-        for (int e = 0; e < AV; ++e) out[e] = a.conv_b ? to_f32(static_cast<const AT*>(a.conv_b)[c + e]) : 0.f;
-        for (int k = 0; k < K; ++k) {
-            float rv[AV];
-            unpack16<AT>(*reinterpret_cast<const uint4*>(win + (t + k) * pitch), rv);
+            for (int e = 0; e < AV; ++e) out[e] = 0.f;
+        }
+        if (K == 4) {
+            // the AV x 4 weight block is four 16-byte vectors, (e, k) at e*4 + k
+            float wf[AV * 4];
 #pragma unroll
-            for (int e = 0; e < AV; ++e) out[e] = fmaf(to_f32(wp[e * K + k]), rv[e], out[e]);
+            for (int q = 0; q < 4; ++q) unpack16<AT>(__ldg(reinterpret_cast<const uint4*>(wp) + q), wf + q * AV);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                float rv[AV];
+                unpack16<AT>(*reinterpret_cast<const uint4*>(win + (t + k) * pitch), rv);
+#pragma unroll
+                for (int e = 0; e < AV; ++e) out[e] = fmaf(wf[e * 4 + k], rv[e], out[e]);
+            }
+        } else {
+            for (int k = 0; k < K; ++k) {
+                float rv[AV];
+                unpack16<AT>(*reinterpret_cast<const uint4*>(win + (t + k) * pitch), rv);
+#pragma unroll
+                for (int e = 0; e < AV; ++e) out[e] = fmaf(to_f32(wp[e * K + k]), rv[e], out[e]);
+            }
         }
         float* dst = u < XV ? s_x + t * kMtRows + u * AV
                             : (u - XV < BV ? s_B + t * N + (u - XV) * AV : s_C + t * N + (u - XV - BV) * AV);
 #pragma unroll
-        for (int e = 0; e < AV; ++e) dst[e] = a.activation ? silu_f32(out[e]) : out[e];
+        for (int e = 0; e < AV; e += 4) {
+            float4 o;
+            o.x = a.activation ? silu_f32(out[e]) : out[e];
+            o.y = a.activation ? silu_f32(out[e + 1]) : out[e + 1];
+            o.z = a.activation ? silu_f32(out[e + 2]) : out[e + 2];
+            o.w = a.activation ? silu_f32(out[e + 3]) : out[e + 3];
+            *reinterpret_cast<float4*>(dst + e) = o;
+        }
     }
     __syncthreads();
 
-    // ---- the T tokens: every thread keeps the same state vectors for all of
-    // them, so the token loop needs no barrier
+    // ---- the T tokens: every thread keeps the same VPT state vectors in
+    // registers for all of them (carrying the stored, rounded value), so the
+    // token loop needs no barrier
+    constexpr int RPP = kMtThreads / LPR;  // rows per pass
     const int lane = tid & 31;
     const int e0 = (lane % LPR) * EPV;
     const int64_t HPN = HP * N;
+    float st[VPT][EPV];
+#pragma unroll
+    for (int i = 0; i < VPT; ++i)
+        unpack16<ST>(*reinterpret_cast<const uint4*>(s_state + static_cast<uint32_t>(i * kMtThreads + tid) * 16u), st[i]);
     for (int t = 0; t < T; ++t) {
         const int32_t dest = a.token_slots[static_cast<int64_t>(b) * T + t];
         const bool store = dest >= 0 && dest < a.num_slots;
         if (dest >= a.num_slots && tid == 0) record_error(a.error, M2_ERR_BAD_SLOT);
         ST* dtile = store ? static_cast<ST*>(a.ssm) + static_cast<int64_t>(dest) * HPN + r0 * N : nullptr;
-        const float* Bt = s_B + t * N + e0;
-        const float* Ct = s_C + t * N + e0;
+        float Bv[EPV], Cv[EPV];
+#pragma unroll
+        for (int e = 0; e < EPV; e += 4) {
+            const float4 b4 = *reinterpret_cast<const float4*>(s_B + t * N + e0 + e);
+            const float4 c4 = *reinterpret_cast<const float4*>(s_C + t * N + e0 + e);
+            Bv[e] = b4.x; Bv[e + 1] = b4.y; Bv[e + 2] = b4.z; Bv[e + 3] = b4.w;
+            Cv[e] = c4.x; Cv[e + 1] = c4.y; Cv[e + 2] = c4.z; Cv[e + 3] = c4.w;
+        }
+        float acc[VPT];
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
-            const int v = i * kMtThreads + tid;
-            const int row = v / LPR;
+            const int row = i * RPP + tid / LPR;
             const int hl = static_cast<int>((r0 + row) / P) - h_first;
-            const float xr = s_x[t * kMtRows + row];
-            const float dtx = s_dt[t][hl] * xr;
+            const float dtx = s_dt[t][hl] * s_x[t * kMtRows + row];
             const float dA = s_dA[t][hl];
-            uint4* sp = reinterpret_cast<uint4*>(s_state + static_cast<uint32_t>(v) * 16u);
-            float st[EPV];
-            unpack16<ST>(*sp, st);
-            float acc = 0.f;
+            float a2 = 0.f;
 #pragma unroll
             for (int e = 0; e < EPV; ++e) {
-                st[e] = fmaf(st[e], dA, dtx * Bt[e]);
-                acc = fmaf(st[e], Ct[e], acc);
+                st[i][e] = fmaf(st[i][e], dA, dtx * Bv[e]);
+                a2 = fmaf(st[i][e], Cv[e], a2);
             }
-            const uint4 packed = pack16<ST>(st);  // the stored state, rounded once per token
-            *sp = packed;
+            const uint4 packed = pack16<ST>(st[i]);  // the stored state, rounded once per token
+            unpack16<ST>(packed, st[i]);              // ... and carried as stored
             if (store) st_stream(dtile + static_cast<int64_t>(row) * N + e0, packed);
+            acc[i] = a2;
+        }
+        if constexpr (VPT == 4 && LPR >= 4) {
+            int which;
+            const float sum = reduce_rows<LPR, 4>(acc, lane, which);
+            if ((lane % (LPR / 4)) == 0) {
+                const int row = which * RPP + tid / LPR;
+                const int hl = static_cast<int>((r0 + row) / P) - h_first;
+                s_y[t * kMtRows + row] = sum + s_D[hl] * s_x[t * kMtRows + row];
+            }
+        } else {
 #pragma unroll
-            for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-            if ((lane % LPR) == 0) s_y[t * kMtRows + row] = acc + s_D[hl] * xr;
+            for (int i = 0; i < VPT; ++i) {
+                float v = acc[i];
+#pragma unroll
+                for (int off = LPR / 2; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+                if ((lane % LPR) == 0) {
+                    const int row = i * RPP + tid / LPR;
+                    const int hl = static_cast<int>((r0 + row) / P) - h_first;
+                    s_y[t * kMtRows + row] = v + s_D[hl] * s_x[t * kMtRows + row];
+                }
+            }
         }
     }
     __syncthreads();
