@@ -661,6 +661,524 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
     }
 }
 
+// ---------------------------------------------------------------------------
+// Pipelined variant: warp-specialised, two chunks in flight (fp16 post-conv
+// input). The per-chunk chain of the kernel above is latency-bound (load, CB,
+// epilogue 1, M X and W^T X, epilogue 2, one after the other). Only epilogue 2
+// and C S^T depend on the carried state, so here they form the sequential
+// chain while epilogue 1 of the next chunk runs beside them:
+//   warp 0        TMA producer: stage (c & 1) <- x, B, C tiles of chunk c
+//   warp 1        MMA issuer: CB, then M X and W^T X, then C S^T
+//   warps 2..9    epilogue 1 (256 threads): dt and decay sums, M (into TMEM,
+//                 as the A operand of M X, so the C tile stays intact for
+//                 C S^T) and W = w o B (in place in the B tile)
+//   warps 10..17  epilogue 2 (256 threads): the fp32 state carry of chunk c
+//                 and its fp16 copy for C S^T of chunk c+1 first, then y of
+//                 chunk c
+// The issuer starts CB of chunk c+1 before it waits for epilogue 1 of chunk c,
+// so epilogue 1 runs chunk after chunk; the state copy is double-buffered, so
+// the carry (the only step that must follow the previous chunk's) is not held
+// up by C S^T of the previous chunk, and y leaves the chain.
+// One CTA per SM (two shared-memory stages of 80 KB and two 16 KB state
+// copies, 512 TMEM columns: per stage CB at 0..127, later dS at 0..63 and
+// Ydiag at 64..127, M at 128..191 (fp16 pairs), Yoff at 192..255). Every
+// hand-off is an mbarrier; every wait is bounded and a timeout ends all roles
+// with M2_ERR_TIMEOUT.
+#ifndef M2_SCAN_PIPELINED
+#define M2_SCAN_PIPELINED 1
+#endif
+constexpr int kP2Threads = 576;
+constexpr uint32_t kP2Stage = 81920;                       // C 32 KB | B 32 KB | X 16 KB
+constexpr uint32_t kP2OffS = 2 * kP2Stage;                 // two fp16 state copies, 16 KB each
+constexpr uint32_t kP2Smem = kP2OffS + 2 * 16384 + 1024;   // + alignment slack
+constexpr uint32_t kP2TmemCols = 512;
+
+// D (TMEM) = A (TMEM, K-major fp16 pairs) . B (shared memory descriptor)
+__device__ __forceinline__ void mma_f16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 8 consecutive 32-bit TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n" ::"r"(taddr),
+                 "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
+
+// Barrier of one 256-thread role (named barrier `id`) that also ORs `flag`
+// over the role: every thread gets the same answer.
+__device__ __forceinline__ bool role_sync_or(int id, bool flag) {
+    uint32_t out;
+    asm volatile(
+        "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n"
+        " bar.red.or.pred q, %2, 256, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+        : "=r"(out)
+        : "r"(flag ? 1u : 0u), "r"(id)
+        : "memory");
+    return out != 0;
+}
+
+// Waits for phase `parity` of `bar`, giving up after the time limit or as soon
+// as another role has aborted.
+__device__ __forceinline__ bool p2_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort_flag || global_ns() - t0 > kLimitNs) return false;
+    }
+    return true;
+}
+
+__device__ __forceinline__ void mbar_arrive1(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];\n" ::"r"(smem_addr(bar)) : "memory");
+}
+
+template <typename ST>
+__global__ void __launch_bounds__(kP2Threads, 1)
+chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs a) {
+    extern __shared__ uint8_t s_raw[];
+    __shared__ __align__(8) uint64_t s_full[2], s_cb[2], s_m[2], s_d[2], s_yoff[2], s_free[2], s_tfree[2];
+    __shared__ __align__(8) uint64_t s_sready[2];  // state copy (i & 1) holds the state entering chunk i
+    __shared__ __align__(8) uint64_t s_drain;
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_abort;
+    __shared__ __align__(16) float s_cum[4][kQ];  // ring of 4 chunks (E2 reads c & 3 while E1 writes ahead)
+    __shared__ __align__(16) float s_dt[4][kQ];
+    __shared__ __align__(16) float s_gam[192];
+    __shared__ float s_wsum[kQ / 32];
+    volatile int* abort_flag = &s_abort;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int h = blockIdx.x;
+    const int nseg = a.nseg;
+    const int b = blockIdx.y / nseg;
+    const int seg = blockIdx.y - b * nseg;
+    const int H = a.H;
+    const int G = a.G;
+    const int g = h / (H / G);
+    const int64_t HP = static_cast<int64_t>(H) * kP;
+    const int64_t row0 = a.cu_seqlens ? static_cast<int64_t>(a.cu_seqlens[b]) : static_cast<int64_t>(b) * a.seqlen;
+    const int T = a.cu_seqlens ? a.cu_seqlens[b + 1] - a.cu_seqlens[b] : a.seqlen;
+    if (T <= 0) return;
+    const int nchunks_seq = (T + kQ - 1) / kQ;
+    const int nseg_s = segments_of(nchunks_seq, nseg, a.seg_chunks);
+    const bool split = nseg_s > 1;
+    if (seg >= nseg_s) return;
+    const int c_begin = split ? seg * a.seg_chunks : 0;
+    const int c_end = (split && seg < nseg_s - 1) ? c_begin + a.seg_chunks : nchunks_seq;
+    const int nloc = c_end - c_begin;
+    const int32_t slot = a.slot_idx[b];
+    bf16_t* y = static_cast<bf16_t*>(a.y);
+    if (slot < 0) {  // padding row: y = 0 over this segment's tokens, cache untouched
+        const int64_t tb = static_cast<int64_t>(c_begin) * kQ;
+        const int64_t te = min(static_cast<int64_t>(c_end) * kQ, static_cast<int64_t>(T));
+        for (int64_t i = tb * (kP / 8) + tid; i < te * (kP / 8); i += kP2Threads) {
+            const int64_t t = i / (kP / 8);
+            *reinterpret_cast<uint4*>(y + (row0 + t) * a.y_stride + h * kP + (i % (kP / 8)) * 8) = make_uint4(0, 0, 0, 0);
+        }
+        return;
+    }
+    if (slot >= a.num_slots) {
+        if (tid == 0) record_error(a.error, M2_ERR_BAD_SLOT);
+        return;
+    }
+
+    const uint32_t raw_addr = smem_addr(s_raw);
+    const uint32_t base = (raw_addr + 1023u) & ~1023u;
+    uint8_t* sm = s_raw + (base - raw_addr);
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_addr(&s_tmem)),
+                     "r"(kP2TmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+    }
+    if (tid == 32) {
+        s_abort = 0;
+        for (int q = 0; q < 2; ++q) {
+            mbar_init(&s_full[q], 1);
+            mbar_init(&s_cb[q], 1);
+            mbar_init(&s_m[q], 1);
+            mbar_init(&s_d[q], 1);
+            mbar_init(&s_yoff[q], 1);
+            mbar_init(&s_free[q], 1);
+            mbar_init(&s_tfree[q], 1);
+        }
+        mbar_init(&s_sready[0], 1);
+        mbar_init(&s_sready[1], 1);
+        mbar_init(&s_drain, 1);
+        fence_mbar_init();
+        asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+
+    const float A = -expf(a.A_log[h]);
+    const float A2 = A * 1.4426950408889634f;
+    const float dt_bias = a.dt_bias[h];
+    const float Dh = a.D[h];
+    const int xcol = h * kP;
+    const int bcol = static_cast<int>(HP) + g * kN;
+    const int ccol = static_cast<int>(HP) + G * kN + g * kN;
+    float range_max = 0.f;
+    __half2 hmax = __float2half2_rn(0.f);
+    int loads_issued = 0;  // producer bookkeeping (lane 0 of warp 0)
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0) {
+            for (int i = 0; i < nloc; ++i) {
+                const int q = i & 1;
+                if (i >= 2 && !p2_wait(&s_free[q], ((i >> 1) - 1) & 1, abort_flag)) {
+                    s_abort = 1;
+                    break;
+                }
+                const int ty = static_cast<int>(row0 + static_cast<int64_t>(c_begin + i) * kQ);
+                const uint32_t st = base + q * kP2Stage;
+                mbar_arrive_expect_tx(&s_full[q], 5u * 16384u);
+                tma_load_2d(st + 65536, &tmap_x, xcol, ty, &s_full[q]);
+                tma_load_2d(st + 32768, &tmap_x, bcol, ty, &s_full[q]);
+                tma_load_2d(st + 32768 + 16384, &tmap_x, bcol + 64, ty, &s_full[q]);
+                tma_load_2d(st, &tmap_x, ccol, ty, &s_full[q]);
+                tma_load_2d(st + 16384, &tmap_x, ccol + 64, ty, &s_full[q]);
+                ++loads_issued;
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t id_cb = idesc_f16(128, 128, false, false);
+            const uint32_t id_yoff = idesc_f16(128, 64, false, false);
+            const uint32_t id_ydiag = idesc_f16(128, 64, false, true);
+            const uint32_t id_ds = idesc_f16(128, 64, true, true);
+            // CB = C . B^T of chunk j into stage j & 1, once its tiles have landed
+            // and epilogue 2 is done with that stage's TMEM (chunk j - 2)
+            auto issue_cb = [&](int j) -> bool {
+                const int q = j & 1;
+                bool ok = p2_wait(&s_full[q], (j >> 1) & 1, abort_flag);
+                if (ok && j >= 2) ok = p2_wait(&s_tfree[q], ((j >> 1) - 1) & 1, abort_flag);
+                if (!ok) return false;
+                tc_fence_after();
+                const uint32_t st = base + q * kP2Stage;
+                for (int k = 0; k < kN / 16; ++k) {
+                    const uint32_t koff = (k >> 2) * 16384u + (k & 3) * 32u;
+                    mma_f16(tmem + q * 256, sw128_desc(st + koff, 16, 1024), sw128_desc(st + 32768 + koff, 16, 1024),
+                            id_cb, k > 0);
+                }
+                mma_commit(&s_cb[q]);
+                return true;
+            };
+            bool ok = nloc <= 0 || issue_cb(0);
+            for (int i = 0; ok && i < nloc; ++i) {
+                const int q = i & 1;
+                const uint32_t par = (i >> 1) & 1;
+                const uint32_t st = base + q * kP2Stage;
+                const uint32_t tq = tmem + q * 256;
+                // CB of the next chunk runs while epilogue 1 works on this one
+                if (i + 1 < nloc && !issue_cb(i + 1)) { ok = false; break; }
+                if (!p2_wait(&s_m[q], par, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                for (int k = 0; k < kQ / 16; ++k)  // Ydiag = M . X (M from TMEM)
+                    mma_f16_ta(tq + 64, tq + 128 + k * 8, sw128_desc(st + 65536 + k * 2048u, 16384, 1024), id_ydiag,
+                               k > 0);
+                for (int k = 0; k < kQ / 16; ++k)  // dS^T = W^T . X
+                    mma_f16(tq + 0, sw128_desc(st + 32768 + k * 2048u, 16384, 1024),
+                            sw128_desc(st + 65536 + k * 2048u, 16384, 1024), id_ds, k > 0);
+                mma_commit(&s_d[q]);
+                // the state entering chunk i, in copy q
+                if (!p2_wait(&s_sready[q], par, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                for (int k = 0; k < kN / 16; ++k) {  // Yoff = C . S^T
+                    const uint32_t koff = (k >> 2) * 16384u + (k & 3) * 32u;
+                    const uint32_t soff = (k >> 2) * 8192u + (k & 3) * 32u;
+                    mma_f16(tq + 192, sw128_desc(st + koff, 16, 1024),
+                            sw128_desc(base + kP2OffS + q * 16384u + soff, 16, 1024), id_yoff, k > 0);
+                }
+                mma_commit(&s_yoff[q]);
+                mma_commit(&s_free[q]);
+            }
+            if (!ok) s_abort = 1;
+        }
+    } else if (warp < 10) {
+        // ------------------------------------------------------- epilogue 1
+        const int e1 = tid - 64;
+        const int quarter = warp & 3;           // TMEM lane quarter of this warp
+        const int t = quarter * 32 + lane;      // row (token) of this thread
+        const int h2 = e1 >> 7;                 // column half
+        const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+        float dt_raw_next = 0.f;
+        if (h2 == 0 && c_begin * kQ + t < T)
+            dt_raw_next = to_f32(static_cast<const bf16_t*>(a.dt)[(row0 + c_begin * kQ + t) * a.dt_stride + h]);
+        for (int i = 0; i < nloc; ++i) {
+            const int c = c_begin + i;
+            const int q = i & 1;
+            const uint32_t par = (i >> 1) & 1;
+            const int ring = i & 3;
+            const int valid = min(kQ, T - c * kQ);
+            // dt and the cumulative decay (log2 units) of chunk c
+            float dt = 0.f, cum = 0.f;
+            if (h2 == 0) {
+                dt = (t < valid) ? softplus_f32(dt_raw_next + dt_bias) : 0.f;
+                if (c + 1 < c_end && t < min(kQ, T - (c + 1) * kQ))
+                    dt_raw_next = to_f32(static_cast<const bf16_t*>(a.dt)[(row0 + (c + 1) * kQ + t) * a.dt_stride + h]);
+                cum = dt * A2;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float o = __shfl_up_sync(0xffffffffu, cum, off);
+                    if (lane >= off) cum += o;
+                }
+                if (lane == 31) s_wsum[quarter] = cum;
+            }
+            role_sync_or(1, false);
+            if (h2 == 0) {
+                for (int w = 0; w < quarter; ++w) cum += s_wsum[w];
+                s_cum[ring][t] = cum;
+                s_dt[ring][t] = dt;
+            }
+            role_sync_or(1, false);
+            const float* cum_c = s_cum[ring];
+            const float* dt_c = s_dt[ring];
+            if (e1 < 192) {
+                const int bq = e1 < 32 ? 1 : (e1 < 96 ? 2 : 3);
+                const int u = e1 - (bq == 1 ? 0 : (bq == 2 ? 32 : 96));
+                s_gam[e1] = ex2(cum_c[32 * bq] - cum_c[u]) * dt_c[u];
+            }
+            const bool got = p2_wait(&s_cb[q], par, abort_flag);
+            if (role_sync_or(1, !got)) { s_abort = 1; break; }
+            tc_fence_after();
+            const uint32_t tq = tmem + q * 256;
+            uint8_t* stB = sm + q * kP2Stage + 32768;
+            const float cum_t = cum_c[t];
+            const float cum_end = cum_c[kQ - 1];
+            const int wq = quarter;
+            const float alpha = ex2(cum_t - cum_c[32 * wq]);
+            const float2 alpha2 = make_float2(alpha, alpha);
+            const float* gam = s_gam + (wq == 1 ? 0 : (wq == 2 ? 32 : 96));
+#pragma unroll 1
+            for (int qb = 0; qb < 4; ++qb) {
+                const int u0 = qb * 32 + 16 * h2;  // this thread's 16 columns of M
+                float m[16];
+                if (qb > wq) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) m[e] = 0.f;
+                } else {
+                    tmem_ld16(tq + lane_base + u0, m);
+                    if (qb < wq) {
+                        const float4* g4 = reinterpret_cast<const float4*>(gam + u0);
+#pragma unroll
+                        for (int i4 = 0; i4 < 4; ++i4) {
+                            const float4 gv = g4[i4];
+                            float2 lo = __fmul2_rn(make_float2(m[4 * i4], m[4 * i4 + 1]), make_float2(gv.x, gv.y));
+                            float2 hi = __fmul2_rn(make_float2(m[4 * i4 + 2], m[4 * i4 + 3]), make_float2(gv.z, gv.w));
+                            lo = __fmul2_rn(lo, alpha2);
+                            hi = __fmul2_rn(hi, alpha2);
+                            m[4 * i4] = lo.x;
+                            m[4 * i4 + 1] = lo.y;
+                            m[4 * i4 + 2] = hi.x;
+                            m[4 * i4 + 3] = hi.y;
+                        }
+                    } else {
+                        const float4* cu4 = reinterpret_cast<const float4*>(cum_c + u0);
+                        const float4* du4 = reinterpret_cast<const float4*>(dt_c + u0);
+#pragma unroll
+                        for (int i4 = 0; i4 < 4; ++i4) {
+                            const float4 cu = cu4[i4], du = du4[i4];
+                            const float cuv[4] = {cu.x, cu.y, cu.z, cu.w};
+                            const float duv[4] = {du.x, du.y, du.z, du.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int u = u0 + 4 * i4 + e;
+                                float v = m[4 * i4 + e] * ex2(cum_t - cuv[e]) * duv[e];
+                                if (u > t) v = 0.f;
+                                if (u == t) v += Dh;
+                                m[4 * i4 + e] = v;
+                            }
+                        }
+                    }
+                }
+                uint32_t hw[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const __half2 hv = __floats2half2_rn(m[2 * j], m[2 * j + 1]);
+                    hmax = __hmax2(hmax, __habs2(hv));
+                    hw[j] = *reinterpret_cast<const uint32_t*>(&hv);
+                }
+                tmem_st8(tq + lane_base + 128 + u0 / 2, hw);  // M row t, columns u0 .. u0+15 as fp16 pairs
+            }
+            // W row t = w_t * B row t (fp16 pairs, in place)
+            const float wu = (t < valid) ? ex2(cum_end - cum_t) * dt_c[t] : 0.f;
+            const __half2 w2 = __float2half2_rn(wu);
+            hmax = __hmax2(hmax, __habs2(w2));
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                uint4* pw = reinterpret_cast<uint4*>(stB + h2 * 16384 + sw128(t, j));
+                uint4 v = *pw;
+                uint32_t* vw = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const __half2 r2 = __hmul2(*reinterpret_cast<const __half2*>(&vw[e]), w2);
+                    hmax = __hmax2(hmax, __habs2(r2));
+                    vw[e] = *reinterpret_cast<const uint32_t*>(&r2);
+                }
+                *pw = v;
+            }
+            tmem_wait_st();
+            fence_proxy_async();
+            tc_fence_before();
+            role_sync_or(1, false);
+            if (e1 == 0) mbar_arrive1(&s_m[q]);
+        }
+    } else {
+        // ------------------------------------------------------- epilogue 2
+        const int e2 = tid - 320;
+        const int quarter = warp & 3;
+        const int t = quarter * 32 + lane;   // row t (y) and state column n = t
+        const int h2 = e2 >> 7;
+        const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+        constexpr int kPH = kP / 2;
+        const int n = t;
+        const int p0 = h2 * kPH;
+        ST* state = static_cast<ST*>(a.ssm) + (static_cast<int64_t>(slot) * HP + static_cast<int64_t>(h) * kP) * kN;
+        float S[kPH];
+        if (split) {
+            const float* src = a.seg_state + ((static_cast<int64_t>(b) * nseg + seg) * H + h) * (kP * kN);
+#pragma unroll
+            for (int k = 0; k < kPH; ++k) S[k] = src[(p0 + k) * kN + n];
+        } else {
+            const bool init = a.has_init != nullptr && a.has_init[b] != 0;
+#pragma unroll
+            for (int k = 0; k < kPH; ++k) S[k] = init ? to_f32(state[(p0 + k) * kN + n]) : 0.f;
+        }
+        auto write_state_copy = [&](int buf) {
+            uint8_t* sS = sm + kP2OffS + buf * 16384 + (n >> 6) * 8192;
+            const uint32_t j = (n & 63) >> 3;
+#pragma unroll
+            for (int k = 0; k < kPH; k += 2) {
+                const __half2 hv = __floats2half2_rn(S[k], S[k + 1]);
+                hmax = __hmax2(hmax, __habs2(hv));
+                *reinterpret_cast<__half*>(sS + sw128(p0 + k, j) + (n & 7) * 2) = __low2half(hv);
+                *reinterpret_cast<__half*>(sS + sw128(p0 + k + 1, j) + (n & 7) * 2) = __high2half(hv);
+            }
+        };
+        write_state_copy(0);
+        fence_proxy_async();
+        role_sync_or(2, false);
+        if (e2 == 0) mbar_arrive1(&s_sready[0]);
+        bool ok = true;
+        for (int i = 0; i < nloc; ++i) {
+            const int c = c_begin + i;
+            const int q = i & 1;
+            const uint32_t par = (i >> 1) & 1;
+            const int ring = i & 3;
+            const int t0 = c * kQ;
+            const int valid = min(kQ, T - t0);
+            // z of this row half, loaded before the waits
+            uint4 zpre[4];
+            {
+                const bool zok = a.z != nullptr && t < valid;
+                const bf16_t* zr = zok ? static_cast<const bf16_t*>(a.z) + (row0 + t0 + t) * a.z_stride + xcol + 32 * h2
+                                       : nullptr;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) zpre[j] = zok ? *reinterpret_cast<const uint4*>(zr + 8 * j) : make_uint4(0, 0, 0, 0);
+            }
+            // s_m: epilogue 1 of chunk c is done (its decay sums, read below, are
+            // published by that release); s_d: dS and Ydiag are in TMEM
+            bool got = p2_wait(&s_m[q], par, abort_flag);
+            if (got) got = p2_wait(&s_d[q], par, abort_flag);
+            if (role_sync_or(2, !got)) { s_abort = 1; ok = false; break; }
+            tc_fence_after();
+            const uint32_t tq = tmem + q * 256;
+            {
+                const float eend = ex2(s_cum[ring][kQ - 1]);
+                float ds[32];
+                tmem_ld32(tq + lane_base + p0, ds);
+#pragma unroll
+                for (int k = 0; k < kPH; ++k) S[k] = fmaf(eend, S[k], ds[k]);
+            }
+            // the state leaving chunk c, for C S^T of chunk c+1: copy (i+1) & 1,
+            // last read by C S^T of chunk c-1, which has completed (s_yoff, below)
+            if (i + 1 < nloc) {
+                write_state_copy((i + 1) & 1);
+                fence_proxy_async();
+                role_sync_or(2, false);
+                if (e2 == 0) mbar_arrive1(&s_sready[(i + 1) & 1]);
+            }
+            got = p2_wait(&s_yoff[q], par, abort_flag);
+            if (role_sync_or(2, !got)) { s_abort = 1; ok = false; break; }
+            tc_fence_after();
+            const float et = ex2(s_cum[ring][t]);
+            const bool row_ok = t < valid;
+            const bool gate = a.z != nullptr;
+            bf16_t* yrow = y + (row0 + t0 + t) * a.y_stride + xcol;
+            const float2 et2 = make_float2(et, et);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                float yd[16], yo[16];
+                tmem_ld16(tq + lane_base + 64 + h2 * 32 + 16 * hh, yd);
+                tmem_ld16(tq + lane_base + 192 + h2 * 32 + 16 * hh, yo);
+#pragma unroll
+                for (int jh = 0; jh < 2; ++jh) {
+                    const int jj = 2 * hh + jh;
+                    float out[8];
+                    float zv[8];
+                    unpack16<bf16_t>(zpre[jj], zv);
+#pragma unroll
+                    for (int e = 0; e < 8; e += 2) {
+                        float2 v = __ffma2_rn(et2, make_float2(yo[8 * jh + e], yo[8 * jh + e + 1]),
+                                              make_float2(yd[8 * jh + e], yd[8 * jh + e + 1]));
+                        if (gate) v = __fmul2_rn(v, silu2_tanh(zv[e], zv[e + 1]));
+                        out[e] = v.x;
+                        out[e + 1] = v.y;
+                    }
+                    if (row_ok) *reinterpret_cast<uint4*>(yrow + 8 * (h2 * 4 + jj)) = pack16<bf16_t>(out);
+                }
+            }
+            // TMEM of stage q is read: chunk c+2 may reuse it
+            tc_fence_before();
+            role_sync_or(2, false);
+            if (e2 == 0) mbar_arrive1(&s_tfree[q]);
+        }
+        if (ok && (!split || seg == nseg_s - 1)) {  // the sequence's final state, in place
+#pragma unroll
+            for (int k = 0; k < kPH; ++k) state[(p0 + k) * kN + n] = from_f32<ST>(S[k]);
+        }
+    }
+
+    // every role is done (or aborted): settle outstanding MMAs and copies, free TMEM
+    if (tid == 32) {  // the MMA issuer: one more commit arrives once all its MMAs have completed
+        mma_commit(&s_drain);
+        mbar_wait_bounded(&s_drain, 0, kLimitNs);
+    }
+    if (tid == 0) {  // the producer: the last load of each stage has landed
+        for (int q = 0; q < 2; ++q) {
+            const int uses = (loads_issued - q + 1) / 2;
+            if (uses > 0) mbar_wait_bounded(&s_full[q], (uses - 1) & 1, kLimitNs);
+        }
+    }
+    __syncthreads();
+    range_max = fmaxf(range_max, fmaxf(__low2float(hmax), __high2float(hmax)));
+    if (s_abort) {
+        if (tid == 0) record_error(a.error, M2_ERR_TIMEOUT);
+    } else if (range_max >= kF16Limit) {
+        record_error(a.error, M2_ERR_RANGE);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kP2TmemCols) : "memory");
+    }
+}
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
 using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                               const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -763,6 +1281,18 @@ cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t stream) {
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
+#if M2_SCAN_PIPELINED
+    if (f16_in) {  // the pipelined, warp-specialised scan (one CTA per SM)
+        static AttrOnce attrs_p2;
+        const cudaError_t e = attrs_p2.ensure([] {
+            return cudaFuncSetAttribute(chunk_scan_p2_kernel<bf16_t>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(kP2Smem));
+        });
+        if (e != cudaSuccess) return e;
+        chunk_scan_p2_kernel<bf16_t><<<grid, kP2Threads, kP2Smem, stream>>>(map, a);
+        return cudaGetLastError();
+    }
+#endif
     auto kern = f16_in ? chunk_scan_tc_kernel<bf16_t, f16_t, false> : chunk_scan_tc_kernel<bf16_t, bf16_t, false>;
     kern<<<grid, kTC, kSmemBytes, stream>>>(map, a);
     return cudaGetLastError();
