@@ -365,18 +365,19 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
     bool ok = true;
     int loads_issued = c_begin < c_end ? 1 : 0, loads_done = 0, mma_issued = 0, mma_done = 0;
     const int t = r;  // token (row) of this thread within a chunk
-    float dt_raw_next = 0.f;  // raw dt of this thread's token in the chunk to be prepared next
-    if (tid < kQ && c_begin * kQ + tid < T)
-        dt_raw_next = to_f32(static_cast<const bf16_t*>(a.dt)[(row0 + c_begin * kQ + tid) * a.dt_stride + h]);
+    // raw dt bits of this thread's token in the chunk to be prepared next: kept
+    // unconverted so the load stays in flight until that chunk needs it
+    bf16_t dt_raw_next = 0;
+    if (tid < kQ && c_begin * kQ + tid < T) dt_raw_next = static_cast<const bf16_t*>(a.dt)[(row0 + c_begin * kQ + tid) * a.dt_stride + h];
     float seg_log2 = 0.f;  // total decay of the chunks done so far, log2 units
     // dt and the cumulative decay c_t of chunk cn, in two parts around a block
     // barrier (warps 0..3, thread = token): the in-warp scan, then the
     // cross-warp prefix and the store into buffer cn & 1.
     auto cum_scan = [&](int cn, float& dt, float& cum) {
         const int vn = min(kQ, T - cn * kQ);
-        dt = (t < vn) ? softplus_f32(dt_raw_next + dt_bias) : 0.f;
+        dt = (t < vn) ? softplus_f32(to_f32(dt_raw_next) + dt_bias) : 0.f;
         if (cn + 1 < c_end && t < min(kQ, T - (cn + 1) * kQ))  // prefetch the following chunk's raw dt
-            dt_raw_next = to_f32(static_cast<const bf16_t*>(a.dt)[(row0 + (cn + 1) * kQ + t) * a.dt_stride + h]);
+            dt_raw_next = static_cast<const bf16_t*>(a.dt)[(row0 + (cn + 1) * kQ + t) * a.dt_stride + h];
         cum = dt * A2;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -675,10 +676,12 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
 //   warps 10..17  epilogue 2 (256 threads): the fp32 state carry of chunk c
 //                 and its fp16 copy for C S^T of chunk c+1 first, then y of
 //                 chunk c
-// The issuer starts CB of chunk c+1 before it waits for epilogue 1 of chunk c,
-// so epilogue 1 runs chunk after chunk; the state copy is double-buffered, so
-// the carry (the only step that must follow the previous chunk's) is not held
-// up by C S^T of the previous chunk, and y leaves the chain.
+// Per chunk the issuer runs C S^T as soon as the state entering the chunk is
+// ready (normally while epilogue 1 still works on M), then M X and W^T X,
+// after which the stage's tiles are free for the load of chunk c+2, then CB of
+// chunk c+1. The state copy is double-buffered, so the carry (the only step
+// that must follow the previous chunk's) is not held up by C S^T of the
+// previous chunk, and y leaves the chain.
 // One CTA per SM (two shared-memory stages of 80 KB and two 16 KB state
 // copies, 512 TMEM columns: per stage CB at 0..127, later dS at 0..63 and
 // Ydiag at 64..127, M at 128..191 (fp16 pairs), Yoff at 192..255). Every
@@ -877,23 +880,15 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
                 mma_commit(&s_cb[q]);
                 return true;
             };
+            // Per chunk: C S^T as soon as the state entering it is ready (well
+            // before epilogue 1 is done with M), then M X and W^T X, which free
+            // the stage, then CB of the next chunk.
             bool ok = nloc <= 0 || issue_cb(0);
             for (int i = 0; ok && i < nloc; ++i) {
                 const int q = i & 1;
                 const uint32_t par = (i >> 1) & 1;
                 const uint32_t st = base + q * kP2Stage;
                 const uint32_t tq = tmem + q * 256;
-                // CB of the next chunk runs while epilogue 1 works on this one
-                if (i + 1 < nloc && !issue_cb(i + 1)) { ok = false; break; }
-                if (!p2_wait(&s_m[q], par, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-                for (int k = 0; k < kQ / 16; ++k)  // Ydiag = M . X (M from TMEM)
-                    mma_f16_ta(tq + 64, tq + 128 + k * 8, sw128_desc(st + 65536 + k * 2048u, 16384, 1024), id_ydiag,
-                               k > 0);
-                for (int k = 0; k < kQ / 16; ++k)  // dS^T = W^T . X
-                    mma_f16(tq + 0, sw128_desc(st + 32768 + k * 2048u, 16384, 1024),
-                            sw128_desc(st + 65536 + k * 2048u, 16384, 1024), id_ds, k > 0);
-                mma_commit(&s_d[q]);
                 // the state entering chunk i, in copy q
                 if (!p2_wait(&s_sready[q], par, abort_flag)) { ok = false; break; }
                 tc_fence_after();
@@ -904,7 +899,17 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
                             sw128_desc(base + kP2OffS + q * 16384u + soff, 16, 1024), id_yoff, k > 0);
                 }
                 mma_commit(&s_yoff[q]);
+                if (!p2_wait(&s_m[q], par, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                for (int k = 0; k < kQ / 16; ++k)  // Ydiag = M . X (M from TMEM)
+                    mma_f16_ta(tq + 64, tq + 128 + k * 8, sw128_desc(st + 65536 + k * 2048u, 16384, 1024), id_ydiag,
+                               k > 0);
+                for (int k = 0; k < kQ / 16; ++k)  // dS^T = W^T . X
+                    mma_f16(tq + 0, sw128_desc(st + 32768 + k * 2048u, 16384, 1024),
+                            sw128_desc(st + 65536 + k * 2048u, 16384, 1024), id_ds, k > 0);
+                mma_commit(&s_d[q]);
                 mma_commit(&s_free[q]);
+                if (i + 1 < nloc && !issue_cb(i + 1)) { ok = false; break; }
             }
             if (!ok) s_abort = 1;
         }
