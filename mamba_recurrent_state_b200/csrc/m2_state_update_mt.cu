@@ -217,13 +217,15 @@ __global__ void __launch_bounds__(kMtThreads, 3) mt_decode_kernel(const MtArgs a
         const bool store = dest >= 0 && dest < a.num_slots;
         if (dest >= a.num_slots && tid == 0) record_error(a.error, M2_ERR_BAD_SLOT);
         ST* dtile = store ? static_cast<ST*>(a.ssm) + static_cast<int64_t>(dest) * HPN + r0 * N : nullptr;
-        float Bv[EPV], Cv[EPV];
+        float2 B2[EPV / 2], C2[EPV / 2];
 #pragma unroll
         for (int e = 0; e < EPV; e += 4) {
             const float4 b4 = *reinterpret_cast<const float4*>(s_B + t * N + e0 + e);
             const float4 c4 = *reinterpret_cast<const float4*>(s_C + t * N + e0 + e);
-            Bv[e] = b4.x; Bv[e + 1] = b4.y; Bv[e + 2] = b4.z; Bv[e + 3] = b4.w;
-            Cv[e] = c4.x; Cv[e + 1] = c4.y; Cv[e + 2] = c4.z; Cv[e + 3] = c4.w;
+            B2[e / 2] = make_float2(b4.x, b4.y);
+            B2[e / 2 + 1] = make_float2(b4.z, b4.w);
+            C2[e / 2] = make_float2(c4.x, c4.y);
+            C2[e / 2 + 1] = make_float2(c4.z, c4.w);
         }
         float acc[VPT];
 #pragma unroll
@@ -232,12 +234,20 @@ __global__ void __launch_bounds__(kMtThreads, 3) mt_decode_kernel(const MtArgs a
             const int hl = static_cast<int>((r0 + row) / P) - h_first;
             const float dtx = s_dt[t][hl] * s_x[t * kMtRows + row];
             const float dA = s_dA[t][hl];
-            float a2 = 0.f;
+            // packed f32x2: per element the rounded product dt*x*B, then one FMA
+            // (the arithmetic of the single-step kernel, element for element)
+            const float2 dtx2 = make_float2(dtx, dtx);
+            const float2 dA2 = make_float2(dA, dA);
+            float2 a2v = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int e = 0; e < EPV; ++e) {
-                st[i][e] = fmaf(st[i][e], dA, dtx * Bv[e]);
-                a2 = fmaf(st[i][e], Cv[e], a2);
+            for (int e = 0; e < EPV / 2; ++e) {
+                float2 s2 = make_float2(st[i][2 * e], st[i][2 * e + 1]);
+                s2 = __ffma2_rn(s2, dA2, __fmul2_rn(dtx2, B2[e]));
+                a2v = __ffma2_rn(s2, C2[e], a2v);
+                st[i][2 * e] = s2.x;
+                st[i][2 * e + 1] = s2.y;
             }
+            const float a2 = a2v.x + a2v.y;
             const uint4 packed = pack16<ST>(st[i]);  // the stored state, rounded once per token
             unpack16<ST>(packed, st[i]);              // ... and carried as stored
             if (store) st_stream(dtile + static_cast<int64_t>(row) * N + e0, packed);
