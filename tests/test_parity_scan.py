@@ -35,14 +35,14 @@ def prefill_inputs(w, xdtype=None):
             d["z"].view(w.batch, w.seqlen, -1))
 
 
-def oracle_scan_row(ol, w, b, s, init: bool, x_code):
+def oracle_scan_row(ol, w, b, s, init: bool, x_code, with_z: bool = True):
     rows = np.arange(b * w.seqlen, (b + 1) * w.seqlen)
     xbc = f64(W.step_rows(w, T_XBC, 0, rows), w.act_dtype)
     if x_code != w.act_dtype:  # xBC handed over in another precision
         mode = {S.F32: O.ROUND_F32, S.BF16: O.ROUND_BF16, S.F16: O.ROUND_F16}[x_code]
         xbc = ol.orc.round_array(xbc, mode)
     dt = f64(W.step_rows(w, T_DT, 0, rows), w.act_dtype)
-    z = f64(W.step_rows(w, T_Z, 0, rows), w.act_dtype)
+    z = f64(W.step_rows(w, T_Z, 0, rows), w.act_dtype) if with_z else None
     state = ol.initial_ssm(s) if init else np.zeros((w.H, w.P, w.N))
     y = ol.orc.ssm_scan(state, O.round_mode_for(w.state_dtype), xbc, dt, ol.dt_bias, ol.A_log,
                         ol.D, z, w.G)
@@ -99,6 +99,31 @@ def test_scan_other_xbc_dtypes(xdt, code, T):
         state, y_ref = oracle_scan_row(ol, w, b, s, False, code)
         assert_close(f64(TI.to_storage_np(y[b]), w.act_dtype), y_ref, w.act_dtype, "y")
         assert_close(f64(TI.to_storage_np(cache.ssm[s]), w.state_dtype), state, w.state_dtype, "S")
+
+
+@pytest.mark.parametrize("xdt,code,T", [(None, S.BF16, 300), (torch.float16, S.F16, 300),
+                                       (torch.float32, S.F32, 40)],
+                         ids=["bf16_tensor_core", "f16_pipelined", "f32_cuda_core"])
+def test_scan_without_gate(xdt, code, T):
+    """z = NULL: y is the ungated scan output, on each scan kernel (bf16 input:
+    the single-chain tensor-core kernel; fp16: the pipelined one; fp32: the
+    CUDA-core scan), with and without an initial state."""
+    w = wl(330 + T, T=T)
+    cache = make_cache(w)
+    t, ssm, _ = layer_objs(w)
+    slot_list, init_list = [1, 2, 5], [1, 0, 1]
+    slots = torch.tensor(slot_list, dtype=torch.int32, device="cuda")
+    init = torch.tensor(init_list, dtype=torch.uint8, device="cuda")
+    x, dt, _ = prefill_inputs(w, xdtype=xdt)
+    y = m2.chunk_scan(cache, ssm, x, dt, slots, has_initial_state=init)
+    torch.cuda.synchronize()
+    assert cache.device_error() == 0
+    ol = OracleLayer(w)
+    for b, s in enumerate(slot_list):
+        state, y_ref = oracle_scan_row(ol, w, b, s, bool(init_list[b]), code, with_z=False)
+        assert_close(f64(TI.to_storage_np(y[b]), w.act_dtype), y_ref, w.act_dtype, f"y row {b}")
+        assert_close(f64(TI.to_storage_np(cache.ssm[s]), w.state_dtype), state, w.state_dtype,
+                     f"final state row {b}")
 
 
 @pytest.mark.parametrize("G", [1, 8])
