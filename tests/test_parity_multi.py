@@ -27,7 +27,7 @@ def bits(a):
     return a.view(np.uint32) if a.dtype == np.float32 else a.view(np.uint16)
 
 
-def run_multi(w, T, slot_list, dest):
+def run_multi(w, T, slot_list, dest, with_z=True):
     """dest: [batch][T] destination slots (negative: not stored)."""
     cache = make_cache(w)
     ssm0, conv0 = cache.ssm.clone(), cache.conv.clone()
@@ -39,7 +39,7 @@ def run_multi(w, T, slot_list, dest):
     z = d["z"].view(batch, T, -1)
     slots = torch.tensor(slot_list, dtype=torch.int32, device="cuda")
     tok = torch.tensor(dest, dtype=torch.int32, device="cuda")
-    y = m2.state_update_multi(cache, ssm, conv, x, dt, slots, tok, z=z)
+    y = m2.state_update_multi(cache, ssm, conv, x, dt, slots, tok, z=z if with_z else None)
     torch.cuda.synchronize()
     assert cache.device_error() == 0
     ol = OracleLayer(w)
@@ -53,7 +53,7 @@ def run_multi(w, T, slot_list, dest):
         for t in range(T):
             r = [b * T + t]
             inp = {k: f64(W.step_rows(w, tid, 0, r), w.act_dtype) for k, tid in (("xBC", T_XBC), ("dt", T_DT), ("z", T_Z))}
-            y_ref = ol.decode(ssm_rows, conv_rows, inp)
+            y_ref = ol.decode(ssm_rows, conv_rows, inp, with_z=with_z)
             assert_close(f64(TI.to_storage_np(y[b, t:t + 1]), w.act_dtype), y_ref, w.act_dtype, f"y row {b} token {t}")
             q = dest[b][t]
             if q >= 0:
@@ -84,6 +84,12 @@ def test_nemotron_h_layer_three_drafts():
 ], ids=lambda w: f"N{w.N}K{w.K}s{w.state_dtype}a{w.act_dtype}")
 def test_dtypes_and_shapes(w):
     run_multi(w, 5, [0, 1], [[2, 3, 4, 5, 6], [7, 8, -1, 9, 10]])
+
+
+def test_without_gate():
+    """z = NULL: every token's y is the ungated output."""
+    w = W.Workload(445, "multi_nogate", 8, 64, 128, 2, 4, S.BF16, S.BF16, 12, 2)
+    run_multi(w, 3, [0, 1], [[2, 3, 4], [5, -1, 6]], with_z=False)
 
 
 def test_one_token_equals_the_fused_decode_step():

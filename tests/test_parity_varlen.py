@@ -47,7 +47,7 @@ def gen_cols(w, tid, rows, c0, c1):
     return f64(out, w.act_dtype)
 
 
-def oracle_heads(ol, w, row0, T, state0, heads):
+def oracle_heads(ol, w, row0, T, state0, heads, with_z=True):
     """The oracle scan of one packed sequence, head by head (a head only sees
     its own x, dt, z and its group's B, C: one-group runs of H = 1)."""
     rows = np.arange(row0, row0 + T)
@@ -61,7 +61,7 @@ def oracle_heads(ol, w, row0, T, state0, heads):
                               gen_cols(w, T_XBC, rows, HP + G * N + g * N, HP + G * N + (g + 1) * N)],
                              axis=1)
         dt = gen_cols(w, T_DT, rows, h, h + 1)
-        z = gen_cols(w, T_Z, rows, h * P, (h + 1) * P)
+        z = gen_cols(w, T_Z, rows, h * P, (h + 1) * P) if with_z else None
         st = np.ascontiguousarray(state0[h:h + 1])
         ys[h] = ol.orc.ssm_scan(st, O.round_mode_for(w.state_dtype), sub, dt, ol.dt_bias[h:h + 1],
                                 ol.A_log[h:h + 1], ol.D[h:h + 1], z, 1)
@@ -69,7 +69,7 @@ def oracle_heads(ol, w, row0, T, state0, heads):
     return ys, states
 
 
-def run_case(w, lengths, slot_list, init_list, heads=None, max_seqlen=None):
+def run_case(w, lengths, slot_list, init_list, heads=None, max_seqlen=None, with_z=True):
     cache = make_cache(w)
     ssm0 = cache.ssm.clone()
     t, ssm, _ = layer_objs(w)
@@ -79,7 +79,7 @@ def run_case(w, lengths, slot_list, init_list, heads=None, max_seqlen=None):
     cu_d = torch.from_numpy(cu).cuda()
     slots = torch.tensor(slot_list, dtype=torch.int32, device="cuda")
     init = torch.tensor(init_list, dtype=torch.uint8, device="cuda")
-    y = m2.chunk_scan_varlen(cache, ssm, x, dt, cu_d, slots, max_seqlen=max_seqlen, z=z,
+    y = m2.chunk_scan_varlen(cache, ssm, x, dt, cu_d, slots, max_seqlen=max_seqlen, z=z if with_z else None,
                              has_initial_state=init)
     torch.cuda.synchronize()
     assert cache.device_error() == 0
@@ -95,7 +95,7 @@ def run_case(w, lengths, slot_list, init_list, heads=None, max_seqlen=None):
             assert torch.equal(cache.ssm[s], ssm0[s]), f"empty sequence {b} touched its slot"
             continue
         state0 = ol.initial_ssm(s) if init_list[b] else np.zeros((w.H, w.P, w.N))
-        ys, states = oracle_heads(ol, w, r0, L, state0, heads)
+        ys, states = oracle_heads(ol, w, r0, L, state0, heads, with_z=with_z)
         y_ref = np.concatenate([ys[h] for h in heads], axis=1)
         y_gpu = f64(TI.to_storage_np(y[r0:r0 + L][:, torch.as_tensor(cols, device="cuda")]), w.act_dtype)
         assert_close(y_gpu, y_ref, w.act_dtype, f"y of sequence {b} (length {L})")
@@ -140,6 +140,13 @@ def test_nemotron_h_one_long_prompt_sampled_heads():
     w = W.Workload(403, "varlen_nemotron", 128, 64, 128, 8, 4, S.BF16, S.BF16, 4, 1, seqlen=4096,
                    chunk=128)
     run_case(w, lengths=[4096], slot_list=[2], init_list=[1], heads=[0, 77, 127])
+
+
+def test_varlen_split_without_gate():
+    """z = NULL through the split path (summary pass, combine, scan pass) and an
+    unsplit short sequence."""
+    w = wl(405, batch=3)
+    run_case(w, lengths=[1200, 90, 700], slot_list=[2, 5, 7], init_list=[1, 0, 1], with_z=False)
 
 
 def test_split_matches_fixed_length_scan():
