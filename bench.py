@@ -57,11 +57,13 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--l2", choices=["rotate", "flush"], default="rotate",
                     help="rotate: disjoint slot sets, back to back; flush: 512 MiB write before each step")
-    ap.add_argument("--sections", default="decode,norm,multi,prefill,longprompt,stack48",
+    ap.add_argument("--sections", default="decode,norm,multi,prefill,longprompt,stack48,fp32_23l,t1_ab",
                     help="comma list: decode (the headline, always run), norm (decode with the "
                          "fused gated RMSNorm), multi (4 speculative draft tokens), prefill (workload 4: "
                          "prefill conv and tensor-core scan), longprompt (one 16K-token prompt: "
-                         "conv and varlen scan), stack48 (workload 2: 48-layer token)")
+                         "conv and varlen scan), stack48 (workload 2: 48-layer token), fp32_23l "
+                         "(workload 3: fp32 state, 23 layers, 64 steps), t1_ab (one decode token "
+                         "through the prefill path, conv + chunk scan at T = 1, against the decode step)")
     return ap.parse_args()
 
 
@@ -527,6 +529,141 @@ def measure_stack48(flush, reps: int = 10) -> dict:
             "seq_layer_steps_per_s": w.layers * w.batch / token_us * 1e6}
 
 
+def measure_fp32_23l(peak_gbs: float) -> dict:
+    """Workload 3: the fp32-state mixer (H=64, P=64, N=128, G=8, 2 MiB of fp32
+    state per layer per sequence), 23 layers of 512-slot caches, 128 sequences,
+    64 consecutive decode steps carried in place. One step is the 23 fused
+    launches of the layer loop, captured once as a CUDA graph and replayed per
+    step; every step is timed with CUDA events. A layer's 128 x 2 MiB of state
+    (256 MiB) exceeds L2 (126 MB), and a slot comes back only after the 22
+    other layers, so no flush is needed."""
+    import torch
+    import mamba_recurrent_state_b200 as m2
+    from m2synth import torch_inputs as TI
+    from m2synth import workloads as W
+    w = W.WORKLOADS[3]
+    shape = m2.Shape(w.H, w.P, w.N, w.G, w.K, w.state_dtype, w.act_dtype)
+    caches, objs, ys = [], [], []
+    inputs = [[TI.step_tensors(w, s, layer) for layer in range(w.layers)] for s in range(2)]
+    staged = {k: [torch.empty_like(inputs[0][layer][k]) for layer in range(w.layers)]
+              for k in ("xBC", "dt", "z")}
+    for layer in range(w.layers):
+        c = m2.Cache(shape, w.num_slots)
+        TI.fill_caches(w, c.ssm, c.conv, layer)
+        caches.append(c)
+        t = TI.layer_tensors(w, layer)
+        objs.append((t, m2.SSMParams(t["A_log"], t["dt_bias"], t["D"]),
+                     m2.ConvParams(t["conv_w"], t["conv_b"], 1)))
+        ys.append(torch.empty((w.batch, w.H * w.P), dtype=torch.bfloat16, device="cuda"))
+
+    def stage(step):  # the step's inputs into the graph's buffers (outside the timed region)
+        for layer in range(w.layers):
+            for k in ("xBC", "dt", "z"):
+                staged[k][layer].copy_(inputs[step % 2][layer][k])
+
+    stage(0)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for layer in range(w.layers):
+            t, ssm, conv = objs[layer]
+            m2.state_update(caches[layer], ssm, staged["xBC"][layer], staged["dt"][layer], t["slots"],
+                            z=staged["z"][layer], conv=conv, y=ys[layer])
+    stream = torch.cuda.current_stream()
+    for i in range(3):
+        stage(i)
+        g.replay()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(w.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(w.steps)]
+    torch.cuda.synchronize()
+    for i in range(w.steps):
+        stage(i)
+        starts[i].record(stream)
+        g.replay()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    step_us = [1e3 * a.elapsed_time(b) for a, b in zip(starts, ends)]
+    for c in caches:
+        if c.device_error() != 0:
+            raise RuntimeError("device error word set during the fp32-state benchmark")
+    del g
+    bytes_step = w.layers * (W.bytes_per_unit(w) * w.batch + W.param_bytes_per_launch(w))
+    mean_us = statistics.mean(step_us)
+    return {"workload": "fp32 state (H=64 P=64 N=128 G=8, 2 MiB per layer per sequence), 23 layers x "
+                        "128 sequences in 512-slot caches, 64 steps in place, one CUDA graph of 23 "
+                        "launches per step",
+            "steps": w.steps, "ms_per_step_mean": mean_us / 1e3,
+            "ms_per_step_median": statistics.median(step_us) / 1e3,
+            "bytes_per_step": bytes_step, "GBs": bytes_step / mean_us / 1e3,
+            "frac_hbm": bytes_step / mean_us / 1e3 / peak_gbs,
+            "seq_layer_steps_per_s": w.layers * w.batch / mean_us * 1e6}
+
+
+def measure_t1_ab(reps: int = 200) -> dict:
+    """One decode token of the workload-1 layer (Nemotron-H, 64 sequences,
+    bf16) taken two ways from the same cache: the decode step (one fused
+    launch: conv tap and roll, state update) against the prefill path at
+    T = 1 (the prefill conv writing its fp16 post-conv buffer, then the chunk
+    scan with the cached state as its initial state). Steps rotate over the
+    four disjoint 64-slot sets like the headline loop; each way is timed as
+    one region per step with CUDA events. This library's scan keeps its chunk
+    state on chip and takes no scratch memory, so the prefill path here is two
+    launches and no allocation, not the five launches with scratch of the
+    chunk-scan-at-decode design it is compared with on the pages."""
+    import torch
+    import mamba_recurrent_state_b200 as m2
+    from m2synth import torch_inputs as TI
+    from m2synth import workloads as W
+    w = W.WORKLOADS[1]
+    shape = m2.Shape(w.H, w.P, w.N, w.G, w.K, w.state_dtype, w.act_dtype)
+    cache = m2.Cache(shape, w.num_slots)
+    TI.fill_caches(w, cache.ssm, cache.conv)
+    t = TI.layer_tensors(w)
+    ssm = m2.SSMParams(t["A_log"], t["dt_bias"], t["D"])
+    conv = m2.ConvParams(t["conv_w"], t["conv_b"], 1)
+    sets = [torch.from_numpy(x).to("cuda") for x in W.slot_sets(w)]
+    inputs = [TI.step_tensors(w, s) for s in range(len(sets))]
+    y = torch.empty((w.batch, w.H * w.P), dtype=torch.bfloat16, device="cuda")
+    xp = torch.empty((w.batch, 1, w.conv_dim), dtype=torch.float16, device="cuda")
+    ones = torch.ones(w.batch, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def decode(i):
+        inp = inputs[i % len(sets)]
+        m2.state_update(cache, ssm, inp["xBC"], inp["dt"], sets[i % len(sets)], z=inp["z"], conv=conv, y=y)
+
+    def prefill_t1(i):
+        inp = inputs[i % len(sets)]
+        s = sets[i % len(sets)]
+        m2.conv1d_update(cache, conv, inp["xBC"].view(w.batch, 1, -1), s, out=xp)
+        m2.chunk_scan(cache, ssm, xp, inp["dt"].view(w.batch, 1, -1), s, z=inp["z"].view(w.batch, 1, -1),
+                      chunk_size=128, has_initial_state=ones, y=y.view(w.batch, 1, -1))
+
+    out = {}
+    for tag, fn in (("decode", decode), ("prefill_path_t1", prefill_t1)):
+        for i in range(8):
+            fn(i)
+        a = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+        b = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+        torch.cuda.synchronize()
+        for i in range(reps):
+            a[i].record(stream)
+            fn(i)
+            b[i].record(stream)
+        torch.cuda.synchronize()
+        out[f"{tag}_us"] = statistics.median(x.elapsed_time(e) * 1e3 for x, e in zip(a, b))
+    if cache.device_error() != 0:
+        raise RuntimeError("device error word set during the T = 1 comparison")
+    out.update({
+        "workload": "one decode token, Nemotron-H layer, 64 sequences in 256 slots, bf16",
+        "decode_launches": 1, "prefill_path_launches": 2,
+        "decode_scratch_bytes": 0, "prefill_path_scratch_bytes": 0,
+        "prefill_path_buffer_bytes": w.batch * w.conv_dim * 2,
+        "ratio": out["prefill_path_t1_us"] / out["decode_us"],
+    })
+    return out
+
+
 def run_ours(args, world, rank, local):
     import torch
     import mamba_recurrent_state_b200 as m2
@@ -584,61 +721,94 @@ def run_ours(args, world, rank, local):
     if cache.device_error() != 0:
         raise RuntimeError("device error word set during the benchmark")
 
-    # ---- end to end through the public API: every step copies its inputs from
-    # pinned host memory to the device, runs the step and copies y back to
-    # pinned host memory. The copies run on two copy streams, double-buffered,
-    # so step i+1's inputs and step i-1's y cross PCIe while step i computes;
-    # the timed region is the whole K-step loop, from the first input copy to
-    # the last y landing in host memory.
-    host_in = [{k: v.cpu().pin_memory() for k, v in inp.items()} for inp in inputs]
-    dev_in = [{k: torch.empty_like(v) for k, v in inputs[0].items()} for _ in range(2)]
-    ys = [torch.empty_like(y) for _ in range(2)]
-    host_y = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for _ in range(2)]
-    h2d = sum(v.numel() * v.element_size() for v in host_in[0].values())
+    # ---- end to end through the C ABI with host buffers: every step copies its
+    # inputs from pinned host memory to the device, runs the step and copies y
+    # back to pinned host memory. A step's xBC, z and dt sit back to back in one
+    # pinned buffer and cross PCIe as one copy; y comes back as one copy. The
+    # copies run on two copy streams over a ring of four device buffers, so the
+    # inputs of later steps and the y of earlier ones cross PCIe while a step
+    # computes. The C entry point is called with arguments marshalled once per
+    # ring slot. The timed region is the whole K-step loop, from the first input
+    # copy to the last y landing in host memory (CUDA events); the host's own
+    # issue time for the loop is reported beside it.
+    import ctypes
+    ring = 4
+    parts = [("xBC", inputs[0]["xBC"]), ("z", inputs[0]["z"]), ("dt", inputs[0]["dt"])]
+    offs, off = {}, 0
+    for k, v in parts:
+        offs[k] = off
+        off += (v.numel() * v.element_size() + 255) // 256 * 256
+    packed_bytes = off
+    host_in = []
+    for inp in inputs:
+        hb = torch.empty(packed_bytes, dtype=torch.uint8).pin_memory()
+        for k, v in parts:
+            n = v.numel() * v.element_size()
+            hb[offs[k]:offs[k] + n].copy_(inp[k].contiguous().view(torch.uint8).view(-1).cpu())
+        host_in.append(hb)
+    dev_in = [torch.empty(packed_bytes, dtype=torch.uint8, device="cuda") for _ in range(ring)]
+    ys = [torch.empty_like(y) for _ in range(ring)]
+    host_y = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for _ in range(ring)]
+    h2d = sum(v.numel() * v.element_size() for _, v in parts)  # bytes of the step's inputs
     d2h = host_y[0].numel() * host_y[0].element_size()
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    L = m2.lib()
+    sp, cp = ssm.c(), conv.c()
+    cache_ref, sp_ref, cp_ref = ctypes.byref(cache.c), ctypes.byref(sp), ctypes.byref(cp)
+    hp, cd = w.H * w.P, w.conv_dim
+    call_args = []
+    for r in range(ring):
+        base = dev_in[r].data_ptr()
+        call_args.append((base + offs["xBC"], base + offs["dt"], base + offs["z"], ys[r].data_ptr()))
+    set_ptrs = [ss.data_ptr() for ss in slot_sets]
+    stream_ptr = stream.cuda_stream
 
     def e2e_loop(n, t_start=None, t_end=None):
-        in_done = [torch.cuda.Event() for _ in range(2)]
-        comp_done = [torch.cuda.Event() for _ in range(2)]
-        out_done = [torch.cuda.Event() for _ in range(2)]
+        in_done = [torch.cuda.Event() for _ in range(ring)]
+        comp_done = [torch.cuda.Event() for _ in range(ring)]
+        out_done = [torch.cuda.Event() for _ in range(ring)]
         if t_start is not None:
             t_start.record(stream)
         s_in.wait_stream(stream)
         s_out.wait_stream(stream)
         for i in range(n):
-            bi = i % 2
+            r = i % ring
+            if i >= ring:
+                s_in.wait_event(comp_done[r])  # step i-ring has read this input buffer
             with torch.cuda.stream(s_in):
-                if i >= 2:
-                    s_in.wait_event(comp_done[bi])  # step i-2 has read this input buffer
-                for k, v in host_in[i % n_sets].items():
-                    dev_in[bi][k].copy_(v, non_blocking=True)
-                in_done[bi].record(s_in)
-            stream.wait_event(in_done[bi])
-            if i >= 2:
-                stream.wait_event(out_done[bi])  # y of step i-2 has been copied out
-            m2.state_update(cache, ssm, dev_in[bi]["xBC"], dev_in[bi]["dt"], slot_sets[i % len(slot_sets)],
-                            z=dev_in[bi]["z"], conv=conv, y=ys[bi])
-            comp_done[bi].record(stream)
+                dev_in[r].copy_(host_in[i % n_sets], non_blocking=True)
+            in_done[r].record(s_in)
+            stream.wait_event(in_done[r])
+            if i >= ring:
+                stream.wait_event(out_done[r])  # y of step i-ring has been copied out
+            xp, dtp, zp, yp = call_args[r]
+            st = L.m2_state_update(cache_ref, sp_ref, cp_ref, w.batch, xp, m2.M2_BF16, cd, dtp, w.H, zp, hp,
+                                   yp, hp, set_ptrs[i % len(set_ptrs)], stream_ptr)
+            if st != m2.M2_OK:
+                raise m2.M2Error(st, "m2_state_update")
+            comp_done[r].record(stream)
+            s_out.wait_event(comp_done[r])
             with torch.cuda.stream(s_out):
-                s_out.wait_event(comp_done[bi])
-                host_y[bi].copy_(ys[bi], non_blocking=True)
-                out_done[bi].record(s_out)
+                host_y[r].copy_(ys[r], non_blocking=True)
+            out_done[r].record(s_out)
         stream.wait_stream(s_in)
         stream.wait_stream(s_out)
         if t_end is not None:
             t_end.record(stream)
 
-    e2e_loop(max(args.warmup, 2))
+    e2e_loop(max(args.warmup, ring))
     torch.cuda.synchronize()
     e_start = torch.cuda.Event(enable_timing=True)
     e_end = torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
+    h0 = time.perf_counter()
     e2e_loop(args.steps, e_start, e_end)
+    host_issue_s = time.perf_counter() - h0
     torch.cuda.synchronize()
     barrier(world)
-    e2e_value, _ = job_throughput(w.batch * args.steps, e_start.elapsed_time(e_end), world)
+    e2e_ms = e_start.elapsed_time(e_end)
+    e2e_value, _ = job_throughput(w.batch * args.steps, e2e_ms, world)
     bytes_per_launch = W.bytes_per_unit(w) * w.batch + W.param_bytes_per_launch(w)
     avg_s = (sum(kern_ms) / len(kern_ms)) / 1e3
     achieved = bytes_per_launch / avg_s / 1e9
@@ -660,9 +830,11 @@ def run_ours(args, world, rank, local):
                      "algorithmic_bytes_per_launch": bytes_per_launch,
                      "kernel_us_median": 1e3 * statistics.median(kern_ms)},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h,
-                "how": "pinned host inputs -> device -> m2.state_update -> y to pinned host, every "
-                       "step; copies on two copy streams, double-buffered, overlapping the steps"},
+                "d2h_bytes_per_step": d2h, "us_per_step": 1e3 * e2e_ms / args.steps,
+                "host_issue_us_per_step": 1e6 * host_issue_s / args.steps,
+                "how": "pinned host buffer (xBC|z|dt packed) -> device, one copy; m2_state_update "
+                       "through the C ABI; y -> pinned host, one copy; every step, on two copy "
+                       "streams over a ring of 4 buffers, overlapping the steps"},
         "gpu_launches": args.steps,  # one fused decode launch per timed step (device-resident loop)
         "clocks": clocks,
     }
@@ -681,6 +853,10 @@ def run_ours(args, world, rank, local):
         line["longprompt"] = measure_longprompt(flush, peak)
     if "stack48" in sections:
         line["stack48"] = measure_stack48(flush)
+    if "fp32_23l" in sections:
+        line["fp32_state_23l"] = measure_fp32_23l(peak)
+    if "t1_ab" in sections:
+        line["t1_ab"] = measure_t1_ab()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     if rank == 0:

@@ -79,7 +79,9 @@ typedef enum m2_status {
     M2_ERR_CUDA = -3,        /* a CUDA runtime call or a launch failed */
     M2_ERR_OOM = -4,         /* device allocation failed (m2_cache_alloc only) */
     M2_ERR_BAD_SLOT = -5,    /* device: a slot index >= num_slots was seen */
-    M2_ERR_TIMEOUT = -6,     /* device: a bounded wait inside a kernel ran out */
+    M2_ERR_TIMEOUT = -6,     /* device: a bounded wait inside a kernel ran out; only the
+                                error word is then meaningful: the launch's outputs (y, the
+                                state and conv cache rows it touches) are undefined */
     M2_ERR_RANGE = -7        /* device: a value exceeded the fp16 range of the tensor-core
                                 scan's operands (|v| >= 65520); that row's results are not valid */
 } m2_status;
@@ -304,20 +306,28 @@ m2_status m2_chunk_scan_varlen(const m2_cache* cache, const m2_ssm_params* ssm, 
                                m2_stream stream);
 
 /*
- * m2_chunk_scan_varlen without any allocation, for callers that must not
- * allocate device memory once they are running: a serving runtime that fixes
- * its device memory budget at start-up (the fixed-size state allocator of the
- * Nemotron-H-8B-Base-8K record) and must not fail a step on an allocation, or
- * a process whose stream-ordered memory pool is unavailable. Same arguments,
- * results and split plan as m2_chunk_scan_varlen (bit for bit); the scratch of
- * a split is a file-scope device array of 16 MiB, enough for every split plan
- * on GPUs of up to 511 SMs (one 32 KB state and one decay per SM at most). A
- * plan that needs more returns M2_ERR_UNSUPPORTED before launching. Nothing in the array needs clearing:
- * every slot the scan pass reads is written earlier in the same call.
+ * m2_chunk_scan_varlen without any allocation. This entry point has no
+ * counterpart in the sources the library follows; it exists for callers that
+ * cannot allocate device memory once they are running: a serving runtime that
+ * reserves all of its device memory at start-up and must not fail a step on an
+ * allocation, or a process in which no stream-ordered memory pool can be used.
+ * Same arguments, results and split plan as m2_chunk_scan_varlen (bit for
+ * bit); the scratch of a split is a file-scope device array of 16 MiB, enough
+ * for every split plan on GPUs of up to 511 SMs (one 32 KB state and one decay
+ * per SM at most). A plan that needs more returns M2_ERR_UNSUPPORTED before
+ * launching. Nothing in the array needs clearing: every slot the scan pass
+ * reads is written earlier in the same call.
  *   - The first call on a device looks up the array's address with
  *     cudaGetSymbolAddress (once per device; its error is returned as
  *     M2_ERR_CUDA) and may load the module that holds it: make that first call
- *     before any stream capture begins on that device.
+ *     before any stream capture begins on that device. The address is cached
+ *     per device for the life of the process; after a cudaDeviceReset the
+ *     cached address is stale, so do not call this entry point again in that
+ *     process.
+ *   - Every GPU on which the library's module is loaded holds the 16 MiB until
+ *     the process exits. Under lazy module loading (the CUDA default) that is
+ *     only a device where a libm2 call has run; with CUDA_MODULE_LOADING=EAGER
+ *     it is every device the process initialises.
  *   - All calls on a device share the one array: two calls whose executions
  *     overlap (other streams, other host threads) race on it and corrupt each
  *     other's results. Serialise them, e.g. on one stream.
@@ -358,7 +368,7 @@ m2_status m2_state_update_multi(const m2_cache* cache, const m2_ssm_params* ssm,
                                 const void* z, int64_t z_row_stride, void* y, int64_t y_row_stride,
                                 const int32_t* slot_idx, const int32_t* token_slots, m2_stream stream);
 
-/* The decode rows of a mixed step: one token each, raw xBC (the conv is/* The decode rows of a mixed step: one token each, raw xBC (the conv is
+/* The decode rows of a mixed step: one token each, raw xBC (the conv is
  * fused), as for m2_state_update with conv != NULL. */
 typedef struct m2_decode_rows {
     int32_t batch;

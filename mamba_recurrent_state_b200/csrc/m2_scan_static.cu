@@ -5,8 +5,11 @@
 // at prefill) keeps one fp32 P x N state per (sequence, segment, head) plus one
 // decay each between its passes. This translation unit holds that scratch as
 // a file-scope device array, so the entry point that uses it allocates
-// nothing. The array lives in its own module: it is only loaded (and its
-// device memory only reserved) on a device where the static entry point runs.
+// nothing. The array's 16 MiB is reserved on every device where the library's
+// module is loaded: under lazy module loading (the CUDA default) a device on
+// which a libm2 call has run, with CUDA_MODULE_LOADING=EAGER every device the
+// process initialises. The address looked up per device is cached for the
+// life of the process; it does not survive a cudaDeviceReset.
 #include <cuda_runtime.h>
 
 #include <mutex>
