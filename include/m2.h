@@ -81,7 +81,10 @@ typedef enum m2_status {
     M2_ERR_BAD_SLOT = -5,    /* device: a slot index >= num_slots was seen */
     M2_ERR_TIMEOUT = -6,     /* device: a bounded wait inside a kernel ran out; only the
                                 error word is then meaningful: the launch's outputs (y, the
-                                state and conv cache rows it touches) are undefined */
+                                state and conv cache rows it touches) are undefined, and a
+                                bulk copy that had still not landed when its CTA gave up
+                                may write into shared memory of a later launch, so treat
+                                the CUDA context as unreliable from then on */
     M2_ERR_RANGE = -7        /* device: a value exceeded the fp16 range of the tensor-core
                                 scan's operands (|v| >= 65520); that row's results are not valid */
 } m2_status;

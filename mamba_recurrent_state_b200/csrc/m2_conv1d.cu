@@ -178,20 +178,25 @@ conv1d_kernel(const ConvArgs a) {
 // ---- prefill conv with the input tile staged in shared memory ---------------
 //
 // For long sequences of 16-bit activations: a CTA of 128 threads owns 256
-// channels x 64 tokens. Warp 0 stages the 64 + K-1 input rows of the tile
+// channels x 32 tokens. Warp 0 stages the 32 + K-1 input rows of the tile
 // (512 bytes each; the rows before the sequence start come from the slot's conv
-// cache) with bulk copies into shared memory, and every thread then computes 16
-// tokens of one 16-byte channel vector from shared memory. A CTA walks several
-// tiles of its sequence with two buffers: the next tile's rows land while the
-// current one is computed.
+// cache) with bulk copies into shared memory, and every thread then computes 8
+// tokens of one 16-byte channel vector from shared memory, two channels at a
+// time with packed f32x2 FMAs (per channel the same FMA chain as the other
+// conv kernels, so the outputs agree bit for bit). A CTA walks several tiles of
+// its sequence with two buffers: the next tile's rows land while the current
+// one is computed. Small tiles keep five CTAs on an SM (96 registers), which
+// the latency of the conv's FMA and SiLU chains needs.
 constexpr int kTileThreads = 128;
 constexpr int kTileCh = 256;   // channels per CTA
-constexpr int kTileTok = 64;   // tokens per tile
+constexpr int kTileTok = 32;   // tokens per tile
+constexpr int kTileMinBlocks = 5;
 constexpr int kMaxTilesPerCta = 8;  // token tiles a CTA walks, double-buffered (at most)
 constexpr uint64_t kTileWaitNs = 1000000000ull;
 
+// (wider convs keep more taps per channel in registers: three CTAs per SM)
 template <typename OT, int K>
-__global__ void __launch_bounds__(kTileThreads) conv1d_tile_kernel(const ConvArgs a) {
+__global__ void __launch_bounds__(kTileThreads, K <= 4 ? kTileMinBlocks : 3) conv1d_tile_kernel(const ConvArgs a) {
     using AT = bf16_t;
     constexpr int VEC = Vec16<AT>::n;                    // 8 channels per vector
     constexpr int NV = kTileCh / VEC;                    // 32 vectors per row
@@ -271,6 +276,7 @@ __global__ void __launch_bounds__(kTileThreads) conv1d_tile_kernel(const ConvArg
     if (first + stride < T) issue(first + stride, 1);
 
     float out_max = 0.f;
+    __half2 hmax = __float2half2_rn(0.f);  // largest |fp16 output| (packed)
     uint32_t phase[2] = {0, 0};
     int in_flight[2] = {first < T ? 1 : 0, first + stride < T ? 1 : 0};
 #pragma unroll 1
@@ -300,18 +306,26 @@ __global__ void __launch_bounds__(kTileThreads) conv1d_tile_kernel(const ConvArg
                 unpack16<AT>(*reinterpret_cast<const uint4*>(&s_rows[tg * TPT + i + K - 1][v * VEC]), cur);
                 float o[VEC];
 #pragma unroll
-                for (int e = 0; e < VEC; ++e) {
-                    float acc = bias[e];
+                for (int e = 0; e < VEC; e += 2) {  // channel pairs: per channel bias, then taps 0..K-1
+                    float2 acc = make_float2(bias[e], bias[e + 1]);
 #pragma unroll
-                    for (int k = 0; k < K - 1; ++k) acc = fmaf(w[e][k], hist[k][e], acc);
-                    acc = fmaf(w[e][K - 1], cur[e], acc);
-                    o[e] = a.activation ? silu_f32(acc) : acc;
+                    for (int k = 0; k < K - 1; ++k)
+                        acc = __ffma2_rn(make_float2(w[e][k], w[e + 1][k]), make_float2(hist[k][e], hist[k][e + 1]), acc);
+                    acc = __ffma2_rn(make_float2(w[e][K - 1], w[e + 1][K - 1]), make_float2(cur[e], cur[e + 1]), acc);
+                    if (a.activation) acc = silu2_f32(acc);
+                    o[e] = acc.x;
+                    o[e + 1] = acc.y;
                 }
                 if constexpr (std::is_same<OT, f16_t>::value) {
+                    // the range check on the packed halves: |v| >= 65520 rounds to inf
+                    const uint4 pk = pack16<OT>(o);
+                    const uint32_t pw[4] = {pk.x, pk.y, pk.z, pk.w};
 #pragma unroll
-                    for (int e = 0; e < VEC; ++e) out_max = fmaxf(out_max, fabsf(o[e]));
+                    for (int e = 0; e < 4; ++e) hmax = __hmax2(hmax, __habs2(*reinterpret_cast<const __half2*>(&pw[e])));
+                    *reinterpret_cast<uint4*>(ob + t * a.out_stride + c0 + v * VEC) = pk;
+                } else {
+                    store_vec<OT, VEC>(ob + t * a.out_stride + c0 + v * VEC, o);
                 }
-                store_vec<OT, VEC>(ob + t * a.out_stride + c0 + v * VEC, o);
 #pragma unroll
                 for (int k = 0; k < K - 2; ++k) {
 #pragma unroll
@@ -327,6 +341,7 @@ __global__ void __launch_bounds__(kTileThreads) conv1d_tile_kernel(const ConvArg
             in_flight[q] = 1;
         }
     }
+    out_max = fmaxf(out_max, fmaxf(__low2float(hmax), __high2float(hmax)));
     if (out_max >= 65520.f) record_error(a.error, M2_ERR_RANGE);  // beyond fp16 (rounds to inf)
     if (blockIdx.y == 0 && tg == 0 && vec_ok) {
         // new cache row k = raw input of token T-(K-1)+k: from the input when
@@ -358,15 +373,17 @@ cudaError_t conv_tile_launch(const ConvArgs& a, dim3 grid, cudaStream_t s) {
 template <typename OT>
 cudaError_t conv_tile_by_k(const ConvArgs& a, cudaStream_t s) {
     // Each CTA walks up to 8 token tiles of its sequence, double-buffered, as
-    // long as the grid keeps about six CTAs per SM (three resident, two waves).
-    // Measured on the 8 x 2048 Nemotron-H prefill: one tile per CTA 221 us,
-    // 2 tiles 205 us, 4 tiles 196 us, 8 tiles 192 us.
+    // long as the grid keeps about two waves of resident CTAs per SM.
+    // Measured on the 8 x 2048 Nemotron-H prefill with 64-token tiles at three
+    // CTAs per SM: one tile per CTA 221 us, 2 tiles 205 us, 4 tiles 196 us,
+    // 8 tiles 192 us; with 32-token tiles at five CTAs per SM and 8 tiles, 154 us.
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         sms = 148;
     const int64_t ch_blocks = (a.conv_dim + kTileCh - 1) / kTileCh;
     const int64_t tiles = std::max<int64_t>((a.seqlen + kTileTok - 1) / kTileTok, 1);
-    const int64_t per_cta = std::clamp<int64_t>(ch_blocks * a.batch * tiles / (6LL * sms), 1, kMaxTilesPerCta);
+    const int64_t per_cta = std::clamp<int64_t>(ch_blocks * a.batch * tiles / (2LL * kTileMinBlocks * sms), 1,
+                                                kMaxTilesPerCta);
     const int64_t ctas_y = std::min<int64_t>((tiles + per_cta - 1) / per_cta, 65535);
     const dim3 grid(static_cast<unsigned>(ch_blocks), static_cast<unsigned>(ctas_y), static_cast<unsigned>(a.batch));
     switch (a.K) {

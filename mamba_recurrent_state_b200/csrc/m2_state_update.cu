@@ -213,6 +213,8 @@ state_update_kernel(const StateUpdateArgs a) {
     const int64_t HP = static_cast<int64_t>(H) * P;
     const int hpg = H / a.G;
     const int h_first = static_cast<int>(r0 / P);
+    // r0's row within its head: head offsets below use 32-bit arithmetic
+    const int rr0 = static_cast<int>(r0 - static_cast<int64_t>(h_first) * P);
     const int g = h_first / hpg;
     const int n_heads_tile = static_cast<int>((r0 + TILE - 1) / P) - h_first + 1;
     const int64_t cd = a.conv_dim;
@@ -221,6 +223,12 @@ state_update_kernel(const StateUpdateArgs a) {
 
     const AT* zrow = a.z ? static_cast<const AT*>(a.z) + b * a.z_stride : nullptr;
     AT* yrow = static_cast<AT*>(a.y) + b * a.y_stride;
+
+    // Launched as a programmatic dependent of the previous kernel on the stream:
+    // nothing here may read global memory before that kernel has completed and
+    // its writes are visible (the inputs, the slots and the cache may all come
+    // from it). Only the launch and the CTA set-up overlap its tail.
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
 
     // ---- slot-independent inputs first: under a saturated memory system every
     // dependent round trip costs microseconds, so these loads are issued before
@@ -298,6 +306,10 @@ state_update_kernel(const StateUpdateArgs a) {
                      CHUNK_BYTES, &s_bar[c]);
         }
     }
+    // every CTA of this grid has its copies in flight: the next kernel on the
+    // stream may be scheduled (it waits for this grid's completion before it
+    // reads anything)
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
     // per-head scalars (n_heads_tile <= kMaxHeadsPerTile < kThreads: one per thread)
     if (tid < n_heads_tile) {
         const float dt = softplus_f32(hs_dtr + hs_bias);
@@ -351,12 +363,11 @@ state_update_kernel(const StateUpdateArgs a) {
                     const uint4 nv = (k < K - 2) ? *reinterpret_cast<const uint4*>(rows + (k + 1) * row_pitch) : xin;
                     *reinterpret_cast<uint4*>(conv0 + k * cd + c0) = nv;
                 }
+                // the AV rows of one vector lie in one head (r0 and P are multiples of 8)
+                const int hl = (rr0 + v * AV) / P;
+                const float dtv = s_dt[hl], dAv = s_dA[hl], Dv = s_D[hl];
 #pragma unroll
-                for (int e = 0; e < AV; ++e) {
-                    const int r = v * AV + e;
-                    const int hl = static_cast<int>((r0 + r) / P) - h_first;
-                    s_rp[r] = make_float4(s_dt[hl] * out[e], s_dA[hl], s_D[hl] * out[e], 0.f);
-                }
+                for (int e = 0; e < AV; ++e) s_rp[v * AV + e] = make_float4(dtv * out[e], dAv, Dv * out[e], 0.f);
             } else {
                 float* dstf = (v / BV) ? s_C : s_B;
 #pragma unroll
@@ -368,7 +379,7 @@ state_update_kernel(const StateUpdateArgs a) {
     } else {
         const XT* xrow = static_cast<const XT*>(a.xBC) + b * a.xBC_stride;
         for (int i = tid; i < TILE; i += kThreads) {
-            const int hl = static_cast<int>((r0 + i) / P) - h_first;
+            const int hl = (rr0 + i) / P;
             const float xv = (i == tid) ? x_first : to_f32(xrow[r0 + i]);
             s_rp[i] = make_float4(s_dt[hl] * xv, s_dA[hl], s_D[hl] * xv, 0.f);
         }
@@ -532,13 +543,18 @@ cudaError_t launch_one(const StateUpdateArgs& a, const DecodePlan& plan, cudaStr
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = FUSED ? plan.cluster : 1;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // programmatic dependent launch: the grid may be scheduled while the
+    // previous kernel on the stream finishes (the kernel waits for it with
+    // griddepcontrol.wait before any global read)
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, kern, a);
 }
 

@@ -52,19 +52,20 @@ __global__ void __launch_bounds__(kMtThreads, 3) mt_decode_kernel(const MtArgs a
     const int K = a.K;
     const int W = K - 1 + T;                 // window rows: K-1 cached, then T raw inputs
     // dynamic shared memory: [state tile | raw x window | raw B|C window |
-    //                         post-conv x, B, C and y of every token (fp32)]
+    //   per (token, row) dt*x, dA, D*x | post-conv B, C of every token | y (fp32)]
     extern __shared__ __align__(128) uint8_t s_dyn[];
     uint8_t* s_state = s_dyn;                                        // [64][N] ST
     AT* s_xw = reinterpret_cast<AT*>(s_dyn + TILE_BYTES);            // [W][64]
     AT* s_bcw = s_xw + static_cast<size_t>(W) * kMtRows;              // [W][2N]
-    float* s_x = reinterpret_cast<float*>(s_bcw + static_cast<size_t>(W) * 2 * N);  // [T][64]
-    float* s_B = s_x + T * kMtRows;                                  // [T][N]
+    float4* s_rp = reinterpret_cast<float4*>(s_bcw + static_cast<size_t>(W) * 2 * N);  // [T][64]
+    float* s_B = reinterpret_cast<float*>(s_rp + T * kMtRows);       // [T][N]
     float* s_C = s_B + T * N;                                        // [T][N]
     float* s_y = s_C + T * N;                                        // [T][64]
     __shared__ __align__(8) uint64_t s_bar;
     __shared__ float s_dt[kMaxDraftTokens][kMtMaxHeads];
     __shared__ float s_dA[kMaxDraftTokens][kMtMaxHeads];
     __shared__ float s_D[kMtMaxHeads];
+    __shared__ int32_t s_tok[kMaxDraftTokens];  // destination slot of every token
     __shared__ int s_fail;
 
     const int tid = threadIdx.x;
@@ -74,8 +75,10 @@ __global__ void __launch_bounds__(kMtThreads, 3) mt_decode_kernel(const MtArgs a
     const int64_t HP = static_cast<int64_t>(a.H) * P;
     const int hpg = a.H / a.G;
     const int h_first = static_cast<int>(r0 / P);
+    // r0's row within its head: head offsets below use 32-bit arithmetic
+    const int rr0 = static_cast<int>(r0 - static_cast<int64_t>(h_first) * P);
     const int g = h_first / hpg;
-    const int n_heads = (kMtRows + P - 1) / P;
+    const int n_heads = (rr0 + kMtRows - 1) / P + 1;  // heads the tile's rows touch
     const int64_t cd = a.conv_dim;
     const int64_t cB = HP + static_cast<int64_t>(g) * N;
     const int64_t cC = HP + static_cast<int64_t>(a.G) * N + static_cast<int64_t>(g) * N;
@@ -132,6 +135,7 @@ __global__ void __launch_bounds__(kMtThreads, 3) mt_decode_kernel(const MtArgs a
         *reinterpret_cast<uint4*>(dst) =
             *reinterpret_cast<const uint4*>(xbase + static_cast<int64_t>(t) * a.xBC_stride + vec_channel(u));
     }
+    if (tid < T) s_tok[tid] = a.token_slots[static_cast<int64_t>(b) * T + tid];
     for (int i = tid; i < T * n_heads; i += kMtThreads) {
         const int t = i / n_heads;
         const int hl = i % n_heads;
@@ -187,16 +191,23 @@ __global__ void __launch_bounds__(kMtThreads, 3) mt_decode_kernel(const MtArgs a
                 for (int e = 0; e < AV; ++e) out[e] = fmaf(to_f32(wp[e * K + k]), rv[e], out[e]);
             }
         }
-        float* dst = u < XV ? s_x + t * kMtRows + u * AV
-                            : (u - XV < BV ? s_B + t * N + (u - XV) * AV : s_C + t * N + (u - XV - BV) * AV);
+        if (a.activation) {
 #pragma unroll
-        for (int e = 0; e < AV; e += 4) {
-            float4 o;
-            o.x = a.activation ? silu_f32(out[e]) : out[e];
-            o.y = a.activation ? silu_f32(out[e + 1]) : out[e + 1];
-            o.z = a.activation ? silu_f32(out[e + 2]) : out[e + 2];
-            o.w = a.activation ? silu_f32(out[e + 3]) : out[e + 3];
-            *reinterpret_cast<float4*>(dst + e) = o;
+            for (int e = 0; e < AV; ++e) out[e] = silu_f32(out[e]);
+        }
+        if (u < XV) {
+            // x: the row parameters of token t; the AV rows of one vector lie in
+            // one head (r0 and P are multiples of 8)
+            const int hl = (rr0 + u * AV) / P;
+            const float dtv = s_dt[t][hl], dAv = s_dA[t][hl], Dv = s_D[hl];
+#pragma unroll
+            for (int e = 0; e < AV; ++e)
+                s_rp[t * kMtRows + u * AV + e] = make_float4(dtv * out[e], dAv, Dv * out[e], 0.f);
+        } else {
+            float* dst = u - XV < BV ? s_B + t * N + (u - XV) * AV : s_C + t * N + (u - XV - BV) * AV;
+#pragma unroll
+            for (int e = 0; e < AV; e += 4)
+                *reinterpret_cast<float4*>(dst + e) = make_float4(out[e], out[e + 1], out[e + 2], out[e + 3]);
         }
     }
     __syncthreads();
@@ -213,7 +224,7 @@ __global__ void __launch_bounds__(kMtThreads, 3) mt_decode_kernel(const MtArgs a
     for (int i = 0; i < VPT; ++i)
         unpack16<ST>(*reinterpret_cast<const uint4*>(s_state + static_cast<uint32_t>(i * kMtThreads + tid) * 16u), st[i]);
     for (int t = 0; t < T; ++t) {
-        const int32_t dest = a.token_slots[static_cast<int64_t>(b) * T + t];
+        const int32_t dest = s_tok[t];
         const bool store = dest >= 0 && dest < a.num_slots;
         if (dest >= a.num_slots && tid == 0) record_error(a.error, M2_ERR_BAD_SLOT);
         ST* dtile = store ? static_cast<ST*>(a.ssm) + static_cast<int64_t>(dest) * HPN + r0 * N : nullptr;
@@ -231,9 +242,9 @@ __global__ void __launch_bounds__(kMtThreads, 3) mt_decode_kernel(const MtArgs a
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
             const int row = i * RPP + tid / LPR;
-            const int hl = static_cast<int>((r0 + row) / P) - h_first;
-            const float dtx = s_dt[t][hl] * s_x[t * kMtRows + row];
-            const float dA = s_dA[t][hl];
+            const float4 rp = s_rp[t * kMtRows + row];
+            const float dtx = rp.x;
+            const float dA = rp.y;
             // packed f32x2: per element the rounded product dt*x*B, then one FMA
             // (the arithmetic of the single-step kernel, element for element)
             const float2 dtx2 = make_float2(dtx, dtx);
@@ -258,8 +269,7 @@ __global__ void __launch_bounds__(kMtThreads, 3) mt_decode_kernel(const MtArgs a
             const float sum = reduce_rows<LPR, 4>(acc, lane, which);
             if ((lane % (LPR / 4)) == 0) {
                 const int row = which * RPP + tid / LPR;
-                const int hl = static_cast<int>((r0 + row) / P) - h_first;
-                s_y[t * kMtRows + row] = sum + s_D[hl] * s_x[t * kMtRows + row];
+                s_y[t * kMtRows + row] = sum + s_rp[t * kMtRows + row].z;
             }
         } else {
 #pragma unroll
@@ -269,8 +279,7 @@ __global__ void __launch_bounds__(kMtThreads, 3) mt_decode_kernel(const MtArgs a
                 for (int off = LPR / 2; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
                 if ((lane % LPR) == 0) {
                     const int row = i * RPP + tid / LPR;
-                    const int hl = static_cast<int>((r0 + row) / P) - h_first;
-                    s_y[t * kMtRows + row] = v + s_D[hl] * s_x[t * kMtRows + row];
+                    s_y[t * kMtRows + row] = v + s_rp[t * kMtRows + row].z;
                 }
             }
         }
@@ -293,7 +302,7 @@ __global__ void __launch_bounds__(kMtThreads, 3) mt_decode_kernel(const MtArgs a
         const int k = i % (K - 1);
         const int u = (i / (K - 1)) % nwrite;
         const int t = i / ((K - 1) * nwrite);
-        const int32_t dest = a.token_slots[static_cast<int64_t>(b) * T + t];
+        const int32_t dest = s_tok[t];
         if (dest < 0 || dest >= a.num_slots) continue;
         int pitch;
         const AT* win = vec_window(u, pitch);
@@ -319,13 +328,14 @@ cudaError_t mt_launch(const MtArgs& a, size_t smem, size_t smem_max, dim3 grid, 
 
 template <typename ST, typename AT>
 cudaError_t mt_by_n(const MtArgs& a, cudaStream_t s) {
-    // tile + raw windows + per-token fp32 x, B, C, y (the largest N, K and T)
+    // tile + raw windows + per token: row parameters (4 floats), fp32 B, C and y
+    // (the largest N, K and T)
     const size_t smem_max = static_cast<size_t>(kMtRows) * 256 * sizeof(ST) +
                             static_cast<size_t>(7 + kMaxDraftTokens) * (kMtRows + 2 * 256) * sizeof(AT) +
-                            static_cast<size_t>(kMaxDraftTokens) * (2 * kMtRows + 2 * 256) * sizeof(float);
+                            static_cast<size_t>(kMaxDraftTokens) * (5 * kMtRows + 2 * 256) * sizeof(float);
     const size_t tile = static_cast<size_t>(kMtRows) * a.N * sizeof(ST);
     const size_t smem = tile + static_cast<size_t>(a.K - 1 + a.T) * (kMtRows + 2 * a.N) * sizeof(AT) +
-                        static_cast<size_t>(a.T) * (2 * kMtRows + 2 * a.N) * sizeof(float);
+                        static_cast<size_t>(a.T) * (5 * kMtRows + 2 * a.N) * sizeof(float);
     const dim3 grid(static_cast<unsigned>(static_cast<int64_t>(a.H) * a.P / kMtRows), static_cast<unsigned>(a.batch));
     switch (a.N) {
         case 64: return mt_launch<ST, AT, 64>(a, smem, smem_max, grid, s);

@@ -60,6 +60,7 @@ def run_and_check(w, steps=1, with_z=True, activation=1, slots=None):
     wl(105, 64, 64, 128, 1, batch=3),           # 64 heads per group: 16-CTA cluster
     wl(106, 8, 16, 64, 4, batch=7),             # P=16
     wl(107, 8, 64, 128, 2, sd=F32, ad=BF, batch=1, steps=3),
+    wl(108, 8, 24, 128, 1),                     # P=24: 64-row tiles start inside a head
 ], ids=lambda w: f"H{w.H}P{w.P}N{w.N}G{w.G}K{w.K}s{w.state_dtype}a{w.act_dtype}b{w.batch}")
 def test_shapes(w):
     run_and_check(w, steps=w.steps)

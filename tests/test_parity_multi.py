@@ -81,7 +81,9 @@ def test_nemotron_h_layer_three_drafts():
     W.Workload(442, "multi_f32", 8, 64, 64, 2, 4, S.F32, S.BF16, 12, 2),
     W.Workload(443, "multi_f32a", 8, 64, 128, 1, 3, S.F32, S.F32, 12, 2),
     W.Workload(444, "multi_n256", 4, 64, 256, 1, 4, S.BF16, S.BF16, 12, 2),
-], ids=lambda w: f"N{w.N}K{w.K}s{w.state_dtype}a{w.act_dtype}")
+    # P = 24 does not divide the 64-row tiles, so tiles start and end inside a head
+    W.Workload(446, "multi_p24", 8, 24, 128, 1, 4, S.BF16, S.BF16, 12, 2),
+], ids=lambda w: f"P{w.P}N{w.N}K{w.K}s{w.state_dtype}a{w.act_dtype}")
 def test_dtypes_and_shapes(w):
     run_multi(w, 5, [0, 1], [[2, 3, 4, 5, 6], [7, 8, -1, 9, 10]])
 
