@@ -275,21 +275,20 @@ __global__ void __launch_bounds__(kTileThreads, K <= 4 ? kTileMinBlocks : 3) con
     if (first < T) issue(first, 0);
     if (first + stride < T) issue(first + stride, 1);
 
-    float out_max = 0.f;
     __half2 hmax = __float2half2_rn(0.f);  // largest |fp16 output| (packed)
-    uint32_t phase[2] = {0, 0};
-    int in_flight[2] = {first < T ? 1 : 0, first + stride < T ? 1 : 0};
+    uint32_t phase = 0;  // bit q: parity of buffer q's next completion
 #pragma unroll 1
     for (int j = 0, t0 = first; t0 < T; ++j, t0 += stride) {
         const int q = j & 1;
-        const bool ok = mbar_wait_bounded(&s_bar[q], phase[q], kTileWaitNs);
-        phase[q] ^= 1;
-        in_flight[q] = 0;
+        const uint32_t par = (phase >> q) & 1u;
+        const bool ok = mbar_wait_bounded(&s_bar[q], par, kTileWaitNs);
+        phase ^= 1u << q;
         if (!__syncthreads_and(ok)) {
             if (tid == 0) record_error(a.error, M2_ERR_TIMEOUT);
-            // let this CTA's copies land (bounded) before its shared memory goes
-            if (!ok) mbar_wait_bounded(&s_bar[q], phase[q] ^ 1, kTileWaitNs);
-            if (in_flight[q ^ 1]) mbar_wait_bounded(&s_bar[q ^ 1], phase[q ^ 1], kTileWaitNs);
+            // let this CTA's copies land (bounded) before its shared memory goes:
+            // this buffer's, and the next tile's in the other buffer if issued
+            if (!ok) mbar_wait_bounded(&s_bar[q], par, kTileWaitNs);
+            if (t0 + stride < T) mbar_wait_bounded(&s_bar[q ^ 1], (phase >> (q ^ 1)) & 1u, kTileWaitNs);
             return;
         }
         AT (*s_rows)[kTileCh] = s_buf[q];
@@ -336,13 +335,10 @@ __global__ void __launch_bounds__(kTileThreads, K <= 4 ? kTileMinBlocks : 3) con
             }
         }
         __syncthreads();  // every thread is done with buffer q
-        if (t0 + 2 * stride < T) {  // the tile after next lands in buffer q
-            issue(t0 + 2 * stride, q);
-            in_flight[q] = 1;
-        }
+        if (t0 + 2 * stride < T) issue(t0 + 2 * stride, q);  // the tile after next lands in buffer q
     }
-    out_max = fmaxf(out_max, fmaxf(__low2float(hmax), __high2float(hmax)));
-    if (out_max >= 65520.f) record_error(a.error, M2_ERR_RANGE);  // beyond fp16 (rounds to inf)
+    if (fmaxf(__low2float(hmax), __high2float(hmax)) >= 65520.f)
+        record_error(a.error, M2_ERR_RANGE);  // beyond fp16 (rounds to inf)
     if (blockIdx.y == 0 && tg == 0 && vec_ok) {
         // new cache row k = raw input of token T-(K-1)+k: from the input when
         // that token exists, else old cache row k + T (read before it is written)

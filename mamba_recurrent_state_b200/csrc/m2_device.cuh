@@ -214,40 +214,36 @@ __device__ __forceinline__ float softplus_f32(float v) {
     return v > 20.f ? v : log1pf(expf(v));
 }
 
-// silu(v) = v / (1 + exp(-v)) with a single special-function (SFU) operation:
-// the hardware exponential gives d = 1 + exp(-v), and 1/d comes from three
-// Newton-Raphson steps r <- r (2 - d r) started at the bit-level estimate
-// r0 = float(0x7EF311C3 - bits(d)). Over every d in [1, e^87] the estimate is
-// within 5.1% of 1/d, the three steps bring that to 1.5e-7, and silu to within
-// 2.5e-7 relative (an fp32 division: 1.7e-7). The SFU retires a quarter warp
-// per cycle where the FMA pipe retires a whole one, so the conv kernels, which
-// take a SiLU per output, are bound by the SFU with two such operations and by
-// the FMA pipe with this one. The exponent is clamped at 87 so that d stays
-// finite; below v = -87 the result is v * e^-87 (~1e-36) instead of smaller.
-// Every kernel uses this one definition (silu2_f32 is the same arithmetic on a
-// pair), so fused and unfused paths agree bit for bit.
-__device__ __forceinline__ float recip_newton(float d) {
-    float r = __int_as_float(0x7EF311C3 - __float_as_int(d));
-    r = r * fmaf(-d, r, 2.f);
-    r = r * fmaf(-d, r, 2.f);
-    r = r * fmaf(-d, r, 2.f);
-    return r;
+// 2^x and 1/x on the special-function unit (ex2.approx / rcp.approx, flush to
+// zero; a couple of ulp each).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+constexpr float kNegLog2E = -1.4426950408889634f;  // -log2(e): exp(-v) = 2^(v * -log2 e)
+
+// silu(v) = v / (1 + exp(-v)): exp(-v) = 2^(v * -log2 e) and the reciprocal of
+// 1 + exp(-v) on the special-function unit, about 3 ulp in all. The limits
+// come out right: for v -> -inf the exponential overflows to inf and its
+// reciprocal to 0, for v -> +inf it underflows to 0. silu2_f32 is the same
+// arithmetic on a pair, with packed f32x2 multiplies and adds (bit for bit
+// silu_f32 of each half; the conv kernels, bound by instruction issue, take
+// SiLUs in pairs). Every kernel uses these, so fused and unfused paths agree
+// bit for bit.
 __device__ __forceinline__ float silu_f32(float v) {
-    const float d = 1.f + __expf(-fmaxf(v, -87.f));
-    return v * recip_newton(d);
+    const float d = 1.f + ex2_approx(v * kNegLog2E);
+    return v * rcp_approx(d);
 }
-// Two SiLUs with packed f32x2 operations, bit for bit silu_f32 of each half.
 __device__ __forceinline__ float2 silu2_f32(float2 v) {
-    const float2 d = make_float2(1.f + __expf(-fmaxf(v.x, -87.f)), 1.f + __expf(-fmaxf(v.y, -87.f)));
-    const float2 nd = make_float2(-d.x, -d.y);
-    const float2 two = make_float2(2.f, 2.f);
-    float2 r = make_float2(__int_as_float(0x7EF311C3 - __float_as_int(d.x)),
-                           __int_as_float(0x7EF311C3 - __float_as_int(d.y)));
-    r = __fmul2_rn(r, __ffma2_rn(nd, r, two));
-    r = __fmul2_rn(r, __ffma2_rn(nd, r, two));
-    r = __fmul2_rn(r, __ffma2_rn(nd, r, two));
-    return __fmul2_rn(v, r);
+    const float2 t = __fmul2_rn(v, make_float2(kNegLog2E, kNegLog2E));
+    const float2 d = __fadd2_rn(make_float2(1.f, 1.f), make_float2(ex2_approx(t.x), ex2_approx(t.y)));
+    return __fmul2_rn(v, make_float2(rcp_approx(d.x), rcp_approx(d.y)));
 }
 
 }  // namespace m2

@@ -13,8 +13,8 @@
 //
 // Work decomposition: one CTA of 256 threads per 64 state rows (the rows of
 // 64/P heads) of one sequence. The CTA stages its state tile (16 KB for bf16,
-// N = 128) and the conv rows of its x channels and of the group's B/C channels
-// with bulk copies, loads the T raw inputs, computes the conv tap of every
+// N = 128), the conv rows of its x channels and of the group's B/C channels
+// and their T raw input rows with bulk copies, computes the conv tap of every
 // (token, 16-byte channel vector) at once (the group's B/C conv is computed by
 // every CTA of the group), and then runs the T state updates on the tile in
 // shared memory (rounded to the storage dtype after every token, exactly as T
@@ -116,25 +116,25 @@ __global__ void __launch_bounds__(kMtThreads, 3) mt_decode_kernel(const MtArgs a
         s_fail = 0;
         mbar_init(&s_bar, 1);
         fence_mbar_init();
-        mbar_arrive_expect_tx(&s_bar, TILE_BYTES + static_cast<uint32_t>(K - 1) * (kMtRows + 2 * N) * sizeof(AT));
+        // the state tile, the K-1 cached rows and the T raw input rows of the
+        // window (x channels of the tile, the group's B and C), all row segments
+        mbar_arrive_expect_tx(&s_bar, TILE_BYTES + static_cast<uint32_t>(W) * (kMtRows + 2 * N) * sizeof(AT));
         bulk_g2s(s_state, tile, TILE_BYTES, &s_bar);
         for (int k = 0; k < K - 1; ++k) {
             bulk_g2s(s_xw + k * kMtRows, conv_in + k * cd + r0, kMtRows * sizeof(AT), &s_bar);
             bulk_g2s(s_bcw + k * 2 * N, conv_in + k * cd + cB, N * sizeof(AT), &s_bar);
             bulk_g2s(s_bcw + k * 2 * N + N, conv_in + k * cd + cC, N * sizeof(AT), &s_bar);
         }
+        for (int t = 0; t < T; ++t) {
+            const AT* xr = xbase + static_cast<int64_t>(t) * a.xBC_stride;
+            const int k = K - 1 + t;
+            bulk_g2s(s_xw + k * kMtRows, xr + r0, kMtRows * sizeof(AT), &s_bar);
+            bulk_g2s(s_bcw + k * 2 * N, xr + cB, N * sizeof(AT), &s_bar);
+            bulk_g2s(s_bcw + k * 2 * N + N, xr + cC, N * sizeof(AT), &s_bar);
+        }
     }
     __syncthreads();  // the barrier is initialised before any thread waits on it
-    // raw inputs of the T tokens (x channels of the tile, the group's B and C);
-    // the head scalars of every token
-    for (int i = tid; i < T * NVEC; i += kMtThreads) {
-        const int t = i / NVEC;
-        const int u = i % NVEC;
-        int pitch;
-        AT* dst = const_cast<AT*>(vec_window(u, pitch)) + (K - 1 + t) * pitch;
-        *reinterpret_cast<uint4*>(dst) =
-            *reinterpret_cast<const uint4*>(xbase + static_cast<int64_t>(t) * a.xBC_stride + vec_channel(u));
-    }
+    // the head scalars of every token, while the copies land
     if (tid < T) s_tok[tid] = a.token_slots[static_cast<int64_t>(b) * T + tid];
     for (int i = tid; i < T * n_heads; i += kMtThreads) {
         const int t = i / n_heads;
