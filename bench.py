@@ -834,6 +834,22 @@ def run_ours(args, world, rank, local):
     barrier(world)
     e2e_ms = e_start.elapsed_time(e_end)
     e2e_value, _ = job_throughput(w.batch * args.steps, e2e_ms, world)
+    # the link itself on this machine: one step's packed inputs host -> device and
+    # its y device -> host, each timed alone (CUDA events on its copy stream)
+    def link_us(copy, strm, reps=20):
+        with torch.cuda.stream(strm):
+            for _ in range(3):
+                copy()
+            a_ = torch.cuda.Event(enable_timing=True)
+            b_ = torch.cuda.Event(enable_timing=True)
+            a_.record(strm)
+            for _ in range(reps):
+                copy()
+            b_.record(strm)
+        torch.cuda.synchronize()
+        return 1e3 * a_.elapsed_time(b_) / reps
+    h2d_us = link_us(lambda: dev_in[0].copy_(host_in[0], non_blocking=True), s_in)
+    d2h_us = link_us(lambda: host_y[0].copy_(ys[0], non_blocking=True), s_out)
     bytes_per_launch = W.bytes_per_unit(w) * w.batch + W.param_bytes_per_launch(w)
     avg_s = local_ms / args.steps / 1e3
     achieved = bytes_per_launch / avg_s / 1e9
@@ -860,6 +876,10 @@ def run_ours(args, world, rank, local):
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "us_per_step": 1e3 * e2e_ms / args.steps,
                 "host_issue_us_per_step": 1e6 * host_issue_s / args.steps,
+                "link": {"h2d_us_per_step": h2d_us, "h2d_GBs": packed_bytes / h2d_us / 1e3,
+                         "d2h_us_per_step": d2h_us, "d2h_GBs": d2h / d2h_us / 1e3,
+                         "note": "each direction timed alone on this box; the steps overlap them with "
+                                 "the kernel, so the slowest of the three bounds us_per_step"},
                 "how": "pinned host buffer (xBC|z|dt packed) -> device, one copy; m2_state_update "
                        "through the C ABI; y -> pinned host, one copy; every step, on two copy "
                        "streams over a ring of 4 buffers, overlapping the steps"},

@@ -85,6 +85,7 @@ def stream_key(seed: int, tensor_id: int, step: int = 0) -> int:
 
 def words(key: int, start: int, count: int) -> np.ndarray:
     """Outputs start .. start+count-1 of the SplitMix64 sequence seeded with key."""
+    start, count = int(start), int(count)  # Python ints: no fixed-width overflow
     with np.errstate(over="ignore"):
         i = np.arange(start + 1, start + count + 1, dtype=np.uint64)
         z = np.uint64(key) + i * np.uint64(GAMMA)

@@ -139,12 +139,14 @@ CONV_STD = 1.0
 
 def ssm_slot(w: Workload, slot: int, layer: int = 0) -> np.ndarray:
     """Initial SSM state of one slot, storage form [H, P, N]."""
+    slot = int(slot)  # a numpy int32 slot would overflow the element offset
     n = w.H * w.P * w.N
     return normal_storage(ssm_key(w, layer), slot * n, n, 0.0, SSM_STD, w.state_dtype).reshape(w.H, w.P, w.N)
 
 
 def conv_slot(w: Workload, slot: int, layer: int = 0) -> np.ndarray:
     """Initial conv cache of one slot, storage form [K-1, conv_dim]."""
+    slot = int(slot)
     n = (w.K - 1) * w.conv_dim
     return normal_storage(conv_key(w, layer), slot * n, n, 0.0, CONV_STD, w.act_dtype).reshape(w.K - 1, w.conv_dim)
 

@@ -150,7 +150,8 @@ def test_16bit_conv_output_between_launches(buf):
 
 def test_workload2_stack48_graph_sampled():
     """48 layers x 384 sequences, one token, captured as one CUDA graph of 48
-    launches; sampled (layer, row) pairs against the oracle."""
+    launches; sampled (layer, row) pairs against the oracle: five layers, with
+    the rows holding slots 0 and 383 in each."""
     w = W.WORKLOADS[2]
     caches, objs, inps = [], [], []
     for layer in range(w.layers):
@@ -167,8 +168,11 @@ def test_workload2_stack48_graph_sampled():
                                         t["slots"], z=inps[layer]["z"], conv=conv)
     g.replay()
     torch.cuda.synchronize()
-    for layer, rows in ((0, [0, 383]), (23, [191]), (47, [5, 300])):
+    for layer, rows in ((0, [0, 383]), (11, [17]), (23, [191]), (35, [250]), (47, [5, 300])):
         ol = OracleLayer(w, layer)
+        # also the rows whose slots sit at the two ends of the cache
+        rows = sorted(set(rows) | {int(np.argmax(ol.slots)), int(np.argmin(ol.slots))})
+        assert int(ol.slots[rows].max()) == w.num_slots - 1 and int(ol.slots[rows].min()) == 0
         ssm_rows = [ol.initial_ssm(ol.slots[r]) for r in rows]
         conv_rows = [ol.initial_conv(ol.slots[r]) for r in rows]
         y_ref = ol.decode(ssm_rows, conv_rows, ol.inputs(0, rows))
@@ -187,13 +191,17 @@ def test_workload2_stack48_graph_sampled():
 
 def test_workload3_fp32_state_64_steps_sampled():
     """23 layers, fp32 state, batch 128 in 512 slots, 64 steps carried in place;
-    sampled (layer, row) pairs followed through all 64 steps by the oracle."""
+    sampled (layer, row) pairs (five layers, the row with the layer's highest
+    slot among them) followed through all 64 steps by the oracle."""
     w = W.WORKLOADS[3]
-    samples = {0: [0, 127], 11: [64], 22: [1]}
+    samples = {0: [0, 127], 5: [33], 11: [64], 17: [100], 22: [1]}
     caches, objs = [], []
     for layer in range(w.layers):
         caches.append(make_cache(w, layer))
         objs.append(layer_objs(w, layer))
+    for layer in samples:  # also the row holding the layer's highest slot
+        slots = W.slot_indices(w, layer)
+        samples[layer] = sorted(set(samples[layer]) | {int(np.argmax(slots))})
     y_hist = {layer: [] for layer in samples}
     buf = None
     for step in range(w.steps):

@@ -70,3 +70,20 @@ def test_workload_sizes_match_pages():
     assert w1.state_bytes_per_slot() == 2 * 1024 * 1024
     assert W.WORKLOADS[3].state_bytes_per_slot() == 2 * 1024 * 1024
     assert W.bytes_per_unit(w1) == 4370692 and W.param_bytes_per_launch(w1) == 103936
+
+
+def test_slot_streams_take_numpy_slot_indices():
+    """A slot index taken from a numpy int32 array regenerates the same state as
+    a Python int, also where the element offset passes 2^31 (slot 383 of the
+    Nemotron-H shape: 6 * 383 * 2^20 words)."""
+    from m2synth import workloads as W
+    w = W.WORKLOADS[2]
+    for slot in (0, 341, 383):
+        a = W.ssm_slot(w, np.int32(slot), 11)
+        b = W.ssm_slot(w, slot, 11)
+        assert np.array_equal(a, b)
+        assert np.array_equal(W.conv_slot(w, np.int32(slot), 11), W.conv_slot(w, slot, 11))
+    # the last slot is the tail of the whole-cache stream
+    n = w.H * w.P * w.N
+    tail = S.normal_storage(W.ssm_key(w, 11), 383 * n + n - 4, 4, 0.0, W.SSM_STD, w.state_dtype)
+    assert np.array_equal(W.ssm_slot(w, np.int32(383), 11).reshape(-1)[-4:], tail)
