@@ -216,9 +216,10 @@ def job_throughput(units_per_rank: int, local_ms: float, world: int) -> tuple[fl
     return units_per_rank * world / (ms / 1e3), ms
 
 
-def oracle_sample(rows: int = 16):
+def oracle_sample(rows: int = 16, threads: int | None = None):
     """A bounded sample of the workload step for the oracle: ``rows`` of the 64
-    sequences, inputs generated up front. Returns (step function, rows, threads)."""
+    sequences, inputs generated up front, run on ``threads`` host threads (all
+    of them by default). Returns (step function, rows, threads)."""
     import numpy as np
     import m2synth as S
     import oracle as O
@@ -234,7 +235,7 @@ def oracle_sample(rows: int = 16):
     inp = {k: f64(v, w.act_dtype) for k, v in W.step_inputs(w, 0, rows=idx).items()}
     params = (f64(p.conv_w, w.act_dtype), f64(p.conv_b, w.act_dtype), p.dt_bias.astype(np.float64),
               p.A_log.astype(np.float64), p.D.astype(np.float64))
-    threads = os.cpu_count() or 1
+    threads = threads or os.cpu_count() or 1
 
     def step():
         O.decode_rows(orc, w.H, w.P, w.N, w.G, O.ROUND_BF16, ssm_rows, conv_rows, inp["xBC"],
@@ -255,9 +256,21 @@ def cpu_baseline(seconds: float) -> dict:
         el = time.perf_counter() - t0
         if el >= seconds:
             break
+    # the same oracle on one thread, on a smaller sample (a fifth of the budget)
+    step1, rows1, _ = oracle_sample(rows=4, threads=1)
+    done1 = 0
+    t1 = time.perf_counter()
+    while True:
+        step1()
+        done1 += rows1
+        el1 = time.perf_counter() - t1
+        if el1 >= seconds / 5:
+            break
     return {"value": done / el, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"{rows} of the 64 sequences of the workload step, decoded "
-                      f"{done // rows} times ({done} seq*layer-steps in {el:.1f} s)"}
+                      f"{done // rows} times ({done} seq*layer-steps in {el:.1f} s)",
+            "one_thread": {"value": done1 / el1, "unit": UNIT, "cores": 1,
+                           "sample": f"{rows1} sequences, {done1 // rows1} times ({el1:.1f} s)"}}
 
 
 def run_reference(args, world, rank):

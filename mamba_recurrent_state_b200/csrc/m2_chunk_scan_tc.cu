@@ -754,7 +754,6 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
     __shared__ __align__(16) float s_cum[4][kQ];  // ring of 4 chunks (E2 reads c & 3 while E1 writes ahead)
     __shared__ __align__(16) float s_dt[4][kQ];
     __shared__ __align__(16) float s_gam[192];
-    __shared__ __half2 s_w2[kQ];  // per token row u: w_u = exp(c_end - c_u) dt_u (0 past the end), as a pair
     __shared__ float s_wsum[kQ / 32];
     volatile int* abort_flag = &s_abort;
 
@@ -958,16 +957,13 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
                 const int u = e1 - (bq == 1 ? 0 : (bq == 2 ? 32 : 96));
                 s_gam[e1] = ex2(cum_c[32 * bq] - cum_c[u]) * dt_c[u];
             }
-            if (h2 == 0) {  // W row scale of row t (published by the barrier after the CB wait)
-                const float wu = (t < valid) ? ex2(cum_c[kQ - 1] - cum_c[t]) * dt_c[t] : 0.f;
-                s_w2[t] = __float2half2_rn(wu);
-            }
             const bool got = p2_wait(&s_cb[q], par, abort_flag);
             if (role_sync_or(1, !got)) { s_abort = 1; break; }
             tc_fence_after();
             const uint32_t tq = tmem + q * 256;
             uint8_t* stB = sm + q * kP2Stage + 32768;
             const float cum_t = cum_c[t];
+            const float cum_end = cum_c[kQ - 1];
             const int wq = quarter;
             const float alpha = ex2(cum_t - cum_c[32 * wq]);
             const float2 alpha2 = make_float2(alpha, alpha);
@@ -1023,34 +1019,22 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
                 }
                 tmem_st8(tq + lane_base + 128 + u0 / 2, hw);  // M row t, columns u0 .. u0+15 as fp16 pairs
             }
-            // W = w o B (fp16 pairs, in place). M above costs a lane quarter
-            // wq + 1 blocks of 32 columns (its rows reach past more of the
-            // causal mask), so W's 2048 16-byte vectors are handed out in
-            // reverse: 11, 9, 7 and 5 per thread for quarters 0..3, which
-            // evens out the quarters' work (every warp then waits least at the
-            // barrier below). Vector v is 16-byte chunk v % 16 of row v / 16.
-            {
-                const int nvw = 11 - 2 * wq;                                  // vectors of this thread
-                const int voff = 64 * (wq == 0 ? 0 : (wq == 1 ? 11 : (wq == 2 ? 20 : 27)));
-                const int idx = h2 * 32 + lane;                               // thread within its quarter
-                hmax = __hmax2(hmax, __habs2(s_w2[t]));
-#pragma unroll 1
-                for (int i = 0; i < nvw; ++i) {
-                    const int v = voff + i * 64 + idx;
-                    const int u = v >> 4;
-                    const int j16 = v & 15;
-                    const __half2 w2 = s_w2[u];
-                    uint4* pw = reinterpret_cast<uint4*>(stB + (j16 >> 3) * 16384 + sw128(u, j16 & 7));
-                    uint4 vv = *pw;
-                    uint32_t* vw = reinterpret_cast<uint32_t*>(&vv);
+            // W row t = w_t * B row t (fp16 pairs, in place)
+            const float wu = (t < valid) ? ex2(cum_end - cum_t) * dt_c[t] : 0.f;
+            const __half2 w2 = __float2half2_rn(wu);
+            hmax = __hmax2(hmax, __habs2(w2));
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const __half2 r2 = __hmul2(*reinterpret_cast<const __half2*>(&vw[e]), w2);
-                        hmax = __hmax2(hmax, __habs2(r2));
-                        vw[e] = *reinterpret_cast<const uint32_t*>(&r2);
-                    }
-                    *pw = vv;
+            for (int j = 0; j < 8; ++j) {
+                uint4* pw = reinterpret_cast<uint4*>(stB + h2 * 16384 + sw128(t, j));
+                uint4 v = *pw;
+                uint32_t* vw = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const __half2 r2 = __hmul2(*reinterpret_cast<const __half2*>(&vw[e]), w2);
+                    hmax = __hmax2(hmax, __habs2(r2));
+                    vw[e] = *reinterpret_cast<const uint32_t*>(&r2);
                 }
+                *pw = v;
             }
             tmem_wait_st();
             fence_proxy_async();

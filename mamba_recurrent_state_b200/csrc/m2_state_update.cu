@@ -109,6 +109,35 @@ __device__ __forceinline__ ConvIn load_conv_in(const AT* xrow, const AT* w, cons
     return in;
 }
 
+// K = 4 conv inputs of one quarter of a 16-byte channel vector: CQ = AV / 4
+// consecutive channels c0.. (two bf16 or one fp32), i.e. 4 bytes of raw input
+// and bias and the CQ x 4 weight block, one 16-byte vector ((e, k) at e*4 + k).
+struct QuadIn {
+    uint4 w;
+    uint32_t xin;
+    uint32_t bias;
+};
+
+template <typename AT>
+__device__ __forceinline__ QuadIn load_quad_in(const AT* xrow, const AT* w, const AT* bias, int64_t c0) {
+    QuadIn in;
+    in.xin = *reinterpret_cast<const uint32_t*>(xrow + c0);
+    in.bias = bias ? __ldg(reinterpret_cast<const uint32_t*>(bias + c0)) : 0u;
+    in.w = __ldg(reinterpret_cast<const uint4*>(w + c0 * 4));
+    return in;
+}
+
+// The 4 bytes of a quarter vector as floats: two bf16 (lo, hi) or one fp32.
+template <typename AT>
+__device__ __forceinline__ void unpack4(uint32_t u, float* out);
+template <>
+__device__ __forceinline__ void unpack4<bf16_t>(uint32_t u, float* out) {
+    out[0] = __uint_as_float(u << 16);
+    out[1] = __uint_as_float(u & 0xFFFF0000u);
+}
+template <>
+__device__ __forceinline__ void unpack4<float>(uint32_t u, float* out) { out[0] = __uint_as_float(u); }
+
 // Conv tap of AV consecutive channels c0.. for one row: the K-1 cached raw
 // inputs (staged in shared memory at `rows`, row pitch `pitch` elements,
 // oldest first) and the raw input; tap K-1 multiplies the newest input.
@@ -237,10 +266,30 @@ state_update_kernel(const StateUpdateArgs a) {
     const bool first_half = tid < kHalf;
     const int v_first = first_half ? tid : tid - kHalf;
     ConvIn cin_first{};
+    QuadIn qin_first{};
     float x_first = 0.f, b_first = 0.f, c_first = 0.f;
+    // K = 4: every thread takes a quarter of a channel vector (vector tid / 4)
+    constexpr int CQ = AV / 4;           // channels per quarter vector
+    constexpr int NVC = XV + 2 * BV;     // conv vectors: the tile's x channels, the group's B and C
+    auto quad_channel = [&](int q, bool& is_x, int& v, int& sub) -> int64_t {
+        v = q >> 2;
+        sub = q & 3;
+        is_x = v < XV;
+        if (is_x) return r0 + static_cast<int64_t>(v) * AV + sub * CQ;
+        const int u = v - XV;
+        return ((u / BV) ? cC : cB) + (u % BV) * AV + sub * CQ;
+    };
     if constexpr (FUSED) {
         const int nvec = first_half ? XV : 2 * BV;
-        if (v_first < nvec) {
+        if (K == 4) {
+            if (tid < 4 * NVC) {
+                bool is_x;
+                int v, sub;
+                const int64_t c0 = quad_channel(tid, is_x, v, sub);
+                qin_first = load_quad_in<AT>(static_cast<const AT*>(a.xBC) + b * a.xBC_stride,
+                                             static_cast<const AT*>(a.conv_w), static_cast<const AT*>(a.conv_b), c0);
+            }
+        } else if (v_first < nvec) {
             const int64_t c0 = first_half ? r0 + static_cast<int64_t>(v_first) * AV
                                           : ((v_first / BV) ? cC : cB) + (v_first % BV) * AV;
             cin_first = load_conv_in<AT>(static_cast<const AT*>(a.xBC) + b * a.xBC_stride,
@@ -326,6 +375,73 @@ state_update_kernel(const StateUpdateArgs a) {
         const AT* w = static_cast<const AT*>(a.conv_w);
         const AT* bias = static_cast<const AT*>(a.conv_b);
         const int nvec = first_half ? XV : 2 * BV;
+        if (K == 4) {
+            // every thread: a quarter of a 16-byte channel vector (CQ channels),
+            // so the conv's FMA and SiLU chains are short and no warp idles; per
+            // channel the same operations in the same order as conv_vec_k4
+            QuadIn qin = qin_first;  // the first quarter's inputs were loaded up front
+            for (int q = tid; q < 4 * NVC; q += kThreads) {
+                bool is_x;
+                int v, sub;
+                const int64_t c0 = quad_channel(q, is_x, v, sub);
+                const AT* rows;
+                int row_pitch;
+                if (is_x) {
+                    rows = s_cx + v * AV + sub * CQ;
+                    row_pitch = TILE;
+                } else {
+                    const int u = v - XV;
+                    rows = s_cbc + (u / BV) * N + (u % BV) * AV + sub * CQ;
+                    row_pitch = 2 * N;
+                }
+                if (q != tid) qin = load_quad_in<AT>(xrow, w, bias, c0);
+                float wf[4 * CQ], out[CQ], xv[CQ];
+                {
+                    float w8[8];
+                    unpack16<AT>(qin.w, w8);  // (e, k) at e*4 + k
+#pragma unroll
+                    for (int i = 0; i < 4 * CQ; ++i) wf[i] = w8[i];
+                }
+                unpack4<AT>(qin.bias, out);
+                if (!mbar_wait_bounded(bar_conv, 0, kWaitLimitNs)) {
+                    record_error(a.error, M2_ERR_TIMEOUT);
+                    s_fail = 1;
+                    break;
+                }
+                unpack4<AT>(qin.xin, xv);
+                uint32_t rr[3];
+#pragma unroll
+                for (int k = 0; k < 3; ++k) {
+                    rr[k] = *reinterpret_cast<const uint32_t*>(rows + k * row_pitch);
+                    float rv[CQ];
+                    unpack4<AT>(rr[k], rv);
+#pragma unroll
+                    for (int e = 0; e < CQ; ++e) out[e] = fmaf(wf[e * 4 + k], rv[e], out[e]);
+                }
+#pragma unroll
+                for (int e = 0; e < CQ; ++e) {
+                    out[e] = fmaf(wf[e * 4 + 3], xv[e], out[e]);
+                    if (a.activation) out[e] = silu_f32(out[e]);
+                }
+                if (is_x) {
+                    // roll the private x rows: row k <- row k+1, last row <- raw input
+                    *reinterpret_cast<uint32_t*>(conv0 + c0) = rr[1];
+                    *reinterpret_cast<uint32_t*>(conv0 + cd + c0) = rr[2];
+                    *reinterpret_cast<uint32_t*>(conv0 + 2 * cd + c0) = qin.xin;
+                    // the rows of one vector lie in one head (r0 and P are multiples of 8)
+                    const int hl = (rr0 + v * AV) / P;
+                    const float dtv = s_dt[hl], dAv = s_dA[hl], Dv = s_D[hl];
+#pragma unroll
+                    for (int e = 0; e < CQ; ++e)
+                        s_rp[v * AV + sub * CQ + e] = make_float4(dtv * out[e], dAv, Dv * out[e], 0.f);
+                } else {
+                    const int u = v - XV;
+                    float* dstf = (u / BV) ? s_C : s_B;
+#pragma unroll
+                    for (int e = 0; e < CQ; ++e) dstf[(u % BV) * AV + sub * CQ + e] = out[e];
+                }
+            }
+        } else {
         ConvIn cin = cin_first;  // the first vector's inputs were loaded up front
         for (int v = v_first; v < nvec; v += kHalf) {
             // channel c0 .. c0+AV-1 and where its cached rows sit in shared memory
@@ -373,6 +489,7 @@ state_update_kernel(const StateUpdateArgs a) {
 #pragma unroll
                 for (int e = 0; e < AV; ++e) dstf[(v % BV) * AV + e] = out[e];
             }
+        }
         }
         // every CTA of the group has read the B/C conv rows once it arrives here
         cluster_arrive();

@@ -12,7 +12,7 @@
 // after verification the caller adopts the slot of the last accepted token.
 //
 // Work decomposition: one CTA of 256 threads per 64 state rows (the rows of
-// 64/P heads) of one sequence. The CTA stages its state tile (16 KB for bf16,
+// 64/P heads) of one sequence, four CTAs per SM. The CTA stages its state tile (16 KB for bf16,
 // N = 128), the conv rows of its x channels and of the group's B/C channels
 // and their T raw input rows with bulk copies, computes the conv tap of every
 // (token, 16-byte channel vector) at once (the group's B/C conv is computed by
@@ -30,13 +30,22 @@
 namespace m2 {
 namespace {
 
+// Resident CTAs per SM the register budget is sized for (compile-time knob):
+// four (64 registers) where N <= 128 -- the phases between the block barriers
+// leave a CTA idle much of its time, and a fourth CTA per SM covers it
+// (Nemotron-H, 64 x 4 drafts: 155.7 us against 169.2 us at three) -- three for
+// N = 256, whose wider rows would spill at 64 registers.
+#ifndef M2_MT_MIN_BLOCKS
+#define M2_MT_MIN_BLOCKS 4
+#endif
+
 constexpr int kMtThreads = 256;
 constexpr int kMtRows = 64;   // state rows per CTA
 constexpr int kMtMaxHeads = kMtRows / 8 + 1;
 constexpr uint64_t kMtWaitNs = 1000000000ull;
 
 template <typename ST, typename AT, int N>
-__global__ void __launch_bounds__(kMtThreads, 3) mt_decode_kernel(const MtArgs a) {
+__global__ void __launch_bounds__(kMtThreads, N <= 128 ? M2_MT_MIN_BLOCKS : 3) mt_decode_kernel(const MtArgs a) {
     constexpr int EPV = Vec16<ST>::n;        // state elements per 16-byte vector
     constexpr int LPR = N / EPV;             // lanes per state row
     static_assert(LPR >= 1 && LPR <= 32 && 32 % LPR == 0, "row must fit a warp");
