@@ -920,9 +920,11 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
         const int t = quarter * 32 + lane;      // row (token) of this thread
         const int h2 = e1 >> 7;                 // column half
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-        float dt_raw_next = 0.f;
+        // the next chunk's dt_raw stays in its bf16 bits until it is used, so the
+        // load is waited for a chunk later, not where it is issued
+        bf16_t dt_raw_next = 0;
         if (h2 == 0 && c_begin * kQ + t < T)
-            dt_raw_next = to_f32(static_cast<const bf16_t*>(a.dt)[(row0 + c_begin * kQ + t) * a.dt_stride + h]);
+            dt_raw_next = static_cast<const bf16_t*>(a.dt)[(row0 + c_begin * kQ + t) * a.dt_stride + h];
         for (int i = 0; i < nloc; ++i) {
             const int c = c_begin + i;
             const int q = i & 1;
@@ -932,9 +934,9 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
             // dt and the cumulative decay (log2 units) of chunk c
             float dt = 0.f, cum = 0.f;
             if (h2 == 0) {
-                dt = (t < valid) ? softplus_f32(dt_raw_next + dt_bias) : 0.f;
+                dt = (t < valid) ? softplus_f32(to_f32(dt_raw_next) + dt_bias) : 0.f;
                 if (c + 1 < c_end && t < min(kQ, T - (c + 1) * kQ))
-                    dt_raw_next = to_f32(static_cast<const bf16_t*>(a.dt)[(row0 + (c + 1) * kQ + t) * a.dt_stride + h]);
+                    dt_raw_next = static_cast<const bf16_t*>(a.dt)[(row0 + (c + 1) * kQ + t) * a.dt_stride + h];
                 cum = dt * A2;
 #pragma unroll
                 for (int off = 1; off < 32; off <<= 1) {
