@@ -84,6 +84,50 @@ def _peak(key: str, fallback: float) -> tuple[float, str]:
         return fallback, "fallback"
 
 
+class _Cudart:
+    """The few CUDA runtime calls the end-to-end loop issues, bound by ctypes to
+    the libcudart that torch loaded (streams and events are shared with torch)."""
+
+    def __init__(self):
+        import ctypes
+        try:
+            lib = ctypes.CDLL("libcudart.so.12", mode=ctypes.RTLD_GLOBAL)
+        except OSError:
+            import nvidia.cuda_runtime as ncr
+            lib = ctypes.CDLL(os.path.join(list(ncr.__path__)[0], "lib", "libcudart.so.12"))
+        vp, sz, ci, cu = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_uint
+        self._ct = ctypes
+        self._lib = lib
+        for name, args in (("cudaMemcpyAsync", [vp, vp, sz, ci, vp]),
+                           ("cudaEventRecord", [vp, vp]),
+                           ("cudaStreamWaitEvent", [vp, vp, cu]),
+                           ("cudaEventCreateWithFlags", [ctypes.POINTER(vp), cu]),
+                           ("cudaEventDestroy", [vp])):
+            fn = getattr(lib, name)
+            fn.argtypes, fn.restype = args, ci
+            setattr(self, name, fn)
+
+    def event(self):
+        e = self._ct.c_void_p()
+        self.check(self.cudaEventCreateWithFlags(self._ct.byref(e), 2), "event")  # timing off
+        return e.value
+
+    @staticmethod
+    def check(status, what):
+        if status != 0:
+            raise RuntimeError(f"CUDA runtime error {status} in {what}")
+
+
+_CUDART = None
+
+
+def cudart() -> _Cudart:
+    global _CUDART
+    if _CUDART is None:
+        _CUDART = _Cudart()
+    return _CUDART
+
+
 def measured_peaks() -> tuple[float, str]:
     """HBM copy bandwidth, GB/s (measured on this machine, else the fallback)."""
     return _peak("hbm_gbs", 6650.0)
@@ -801,34 +845,43 @@ def run_ours(args, world, rank, local):
     set_ptrs = [ss.data_ptr() for ss in slot_sets]
     stream_ptr = stream.cuda_stream
 
+    # The loop's stream operations go to the CUDA runtime through ctypes (the
+    # same libcudart torch loaded), so that issuing a step costs the host a few
+    # microseconds instead of the tens that torch's Python wrappers take.
+    rt = cudart()
+    H2D, D2H = 1, 2
+    in_ptr = [hb.data_ptr() for hb in host_in]
+    hy_ptr = [hy.data_ptr() for hy in host_y]
+    dv_ptr = [d.data_ptr() for d in dev_in]
+    ys_ptr = [yy.data_ptr() for yy in ys]
+    s_in_p, s_out_p = s_in.cuda_stream, s_out.cuda_stream
+    ev = [[rt.event() for _ in range(ring)] for _ in range(3)]  # in_done, comp_done, out_done
+
     def e2e_loop(n, t_start=None, t_end=None):
-        in_done = [torch.cuda.Event() for _ in range(ring)]
-        comp_done = [torch.cuda.Event() for _ in range(ring)]
-        out_done = [torch.cuda.Event() for _ in range(ring)]
+        in_done, comp_done, out_done = ev
         if t_start is not None:
             t_start.record(stream)
         s_in.wait_stream(stream)
         s_out.wait_stream(stream)
+        memcpy, record, wait = rt.cudaMemcpyAsync, rt.cudaEventRecord, rt.cudaStreamWaitEvent
         for i in range(n):
             r = i % ring
             if i >= ring:
-                s_in.wait_event(comp_done[r])  # step i-ring has read this input buffer
-            with torch.cuda.stream(s_in):
-                dev_in[r].copy_(host_in[i % n_sets], non_blocking=True)
-            in_done[r].record(s_in)
-            stream.wait_event(in_done[r])
+                wait(s_in_p, comp_done[r], 0)  # step i-ring has read this input buffer
+            rt.check(memcpy(dv_ptr[r], in_ptr[i % n_sets], packed_bytes, H2D, s_in_p), "copy in")
+            record(in_done[r], s_in_p)
+            wait(stream_ptr, in_done[r], 0)
             if i >= ring:
-                stream.wait_event(out_done[r])  # y of step i-ring has been copied out
+                wait(stream_ptr, out_done[r], 0)  # y of step i-ring has been copied out
             xp, dtp, zp, yp = call_args[r]
             st = L.m2_state_update(cache_ref, sp_ref, cp_ref, w.batch, xp, m2.M2_BF16, cd, dtp, w.H, zp, hp,
                                    yp, hp, set_ptrs[i % len(set_ptrs)], stream_ptr)
             if st != m2.M2_OK:
                 raise m2.M2Error(st, "m2_state_update")
-            comp_done[r].record(stream)
-            s_out.wait_event(comp_done[r])
-            with torch.cuda.stream(s_out):
-                host_y[r].copy_(ys[r], non_blocking=True)
-            out_done[r].record(s_out)
+            record(comp_done[r], stream_ptr)
+            wait(s_out_p, comp_done[r], 0)
+            rt.check(memcpy(hy_ptr[r], ys_ptr[r], d2h, D2H, s_out_p), "copy out")
+            record(out_done[r], s_out_p)
         stream.wait_stream(s_in)
         stream.wait_stream(s_out)
         if t_end is not None:
@@ -846,6 +899,9 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = e_start.elapsed_time(e_end)
+    for e_ in ev:
+        for x_ in e_:
+            rt.cudaEventDestroy(x_)
     e2e_value, _ = job_throughput(w.batch * args.steps, e2e_ms, world)
     # the link itself on this machine: one step's packed inputs host -> device and
     # its y device -> host, each timed alone (CUDA events on its copy stream)
@@ -895,7 +951,8 @@ def run_ours(args, world, rank, local):
                                  "the kernel, so the slowest of the three bounds us_per_step"},
                 "how": "pinned host buffer (xBC|z|dt packed) -> device, one copy; m2_state_update "
                        "through the C ABI; y -> pinned host, one copy; every step, on two copy "
-                       "streams over a ring of 4 buffers, overlapping the steps"},
+                       "streams over a ring of 4 buffers, overlapping the steps; copies and "
+                       "stream waits issued through the CUDA runtime by ctypes"},
         "gpu_launches": args.steps,  # one fused decode launch per timed step (device-resident loop)
         "clocks": clocks,
     }
