@@ -185,8 +185,10 @@ conv1d_kernel(const ConvArgs a) {
 // time with packed f32x2 FMAs (per channel the same FMA chain as the other
 // conv kernels, so the outputs agree bit for bit). A CTA walks several tiles of
 // its sequence with two buffers: the next tile's rows land while the current
-// one is computed. Small tiles keep five CTAs on an SM (96 registers), which
-// the latency of the conv's FMA and SiLU chains needs.
+// one is computed. There is no block barrier between tiles: each warp arrives
+// on the buffer's "empty" mbarrier when it is done with it, and warp 0 refills
+// the buffer once all four have arrived. Small tiles keep five CTAs on an SM
+// (96 registers), which the latency of the conv's FMA and SiLU chains needs.
 constexpr int kTileThreads = 128;
 constexpr int kTileCh = 256;   // channels per CTA
 constexpr int kTileTok = 32;   // tokens per tile
@@ -207,6 +209,7 @@ __global__ void __launch_bounds__(kTileThreads, K <= 4 ? kTileMinBlocks : 3) con
     extern __shared__ __align__(128) uint8_t s_conv_dyn[];
     AT (*s_buf)[ROWS][kTileCh] = reinterpret_cast<AT (*)[ROWS][kTileCh]>(s_conv_dyn);
     __shared__ __align__(8) uint64_t s_bar[2];
+    __shared__ __align__(8) uint64_t s_empty[2];  // arrivals of the 4 warps done with buffer q
 
     const int tid = threadIdx.x;
     const int b = blockIdx.z;
@@ -250,6 +253,8 @@ __global__ void __launch_bounds__(kTileThreads, K <= 4 ? kTileMinBlocks : 3) con
     if (tid == 0) {
         mbar_init(&s_bar[0], 1);
         mbar_init(&s_bar[1], 1);
+        mbar_init(&s_empty[0], kTileThreads / 32);
+        mbar_init(&s_empty[1], kTileThreads / 32);
         fence_mbar_init();
     }
     __syncthreads();
@@ -283,9 +288,9 @@ __global__ void __launch_bounds__(kTileThreads, K <= 4 ? kTileMinBlocks : 3) con
         const uint32_t par = (phase >> q) & 1u;
         const bool ok = mbar_wait_bounded(&s_bar[q], par, kTileWaitNs);
         phase ^= 1u << q;
-        if (!__syncthreads_and(ok)) {
-            if (tid == 0) record_error(a.error, M2_ERR_TIMEOUT);
-            // let this CTA's copies land (bounded) before its shared memory goes:
+        if (!__all_sync(0xffffffffu, ok)) {
+            if ((tid & 31) == 0) record_error(a.error, M2_ERR_TIMEOUT);
+            // let this CTA's copies land (bounded) before this warp leaves:
             // this buffer's, and the next tile's in the other buffer if issued
             if (!ok) mbar_wait_bounded(&s_bar[q], par, kTileWaitNs);
             if (t0 + stride < T) mbar_wait_bounded(&s_bar[q ^ 1], (phase >> (q ^ 1)) & 1u, kTileWaitNs);
@@ -301,6 +306,7 @@ __global__ void __launch_bounds__(kTileThreads, K <= 4 ? kTileMinBlocks : 3) con
             for (int i = 0; i < TPT; ++i) {
                 const int t = t0 + tg * TPT + i;
                 if (t >= T) break;
+                OT* const optr = ob + t * a.out_stride + c0 + v * VEC;
                 float cur[VEC];
                 unpack16<AT>(*reinterpret_cast<const uint4*>(&s_rows[tg * TPT + i + K - 1][v * VEC]), cur);
                 float o[VEC];
@@ -321,9 +327,9 @@ __global__ void __launch_bounds__(kTileThreads, K <= 4 ? kTileMinBlocks : 3) con
                     const uint32_t pw[4] = {pk.x, pk.y, pk.z, pk.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) hmax = __hmax2(hmax, __habs2(*reinterpret_cast<const __half2*>(&pw[e])));
-                    *reinterpret_cast<uint4*>(ob + t * a.out_stride + c0 + v * VEC) = pk;
+                    *reinterpret_cast<uint4*>(optr) = pk;
                 } else {
-                    store_vec<OT, VEC>(ob + t * a.out_stride + c0 + v * VEC, o);
+                    store_vec<OT, VEC>(optr, o);
                 }
 #pragma unroll
                 for (int k = 0; k < K - 2; ++k) {
@@ -334,8 +340,20 @@ __global__ void __launch_bounds__(kTileThreads, K <= 4 ? kTileMinBlocks : 3) con
                 for (int e = 0; e < VEC; ++e) hist[K - 2][e] = cur[e];
             }
         }
-        __syncthreads();  // every thread is done with buffer q
-        if (t0 + 2 * stride < T) issue(t0 + 2 * stride, q);  // the tile after next lands in buffer q
+        // this warp is done with buffer q; warp 0 refills it once all four are
+        // (no block barrier: a warp that finishes early goes on to the next tile)
+        __syncwarp();
+        if ((tid & 31) == 0) mbar_arrive(&s_empty[q]);
+        if (tid < 32 && t0 + 2 * stride < T) {
+            const bool eok = mbar_wait_bounded(&s_empty[q], (j >> 1) & 1, kTileWaitNs);
+            if (!__all_sync(0xffffffffu, eok)) {
+                if (tid == 0) record_error(a.error, M2_ERR_TIMEOUT);
+                // the next tile's copies into the other buffer, if issued, land (bounded)
+                if (t0 + stride < T) mbar_wait_bounded(&s_bar[q ^ 1], (phase >> (q ^ 1)) & 1u, kTileWaitNs);
+                return;
+            }
+            issue(t0 + 2 * stride, q);  // the tile after next lands in buffer q
+        }
     }
     if (fmaxf(__low2float(hmax), __high2float(hmax)) >= 65520.f)
         record_error(a.error, M2_ERR_RANGE);  // beyond fp16 (rounds to inf)
