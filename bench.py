@@ -392,6 +392,18 @@ def measure_prefill(flush, peak_gbs: float, peak_tflops: float, reps: int = 10) 
         scan_step()
     conv_us = statistics.median(_time_us(conv_step, flush, reps))
     scan_us = statistics.median(_time_us(scan_step, flush, reps))
+    # the scan again, 12 launches back to back between one pair of events (no
+    # flush: 893 MB of operands per launch against a 126 MB L2); an ncu capture
+    # of these launches counts each launch's DRAM traffic including the
+    # write-back of its own output
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(12):
+        scan_step()
+    e1.record(stream)
+    e1.synchronize()
+    scan_b2b_us = 1e3 * e0.elapsed_time(e1) / 12
     if cache.device_error() != 0:
         raise RuntimeError("device error word set during the prefill benchmark")
     tokens = w.batch * T
@@ -409,7 +421,8 @@ def measure_prefill(flush, peak_gbs: float, peak_tflops: float, reps: int = 10) 
         "workload": "prefill: 8 seqs x 2048 tokens, Nemotron-H layer, bf16, zero initial state",
         "conv_us": conv_us, "conv_GBs": conv_bytes / conv_us / 1e3,
         "conv_frac_hbm": conv_bytes / conv_us / 1e3 / peak_gbs,
-        "scan_us": scan_us, "scan_bytes": scan_bytes, "scan_GBs": scan_bytes / scan_us / 1e3,
+        "scan_us": scan_us, "scan_b2b_us": scan_b2b_us, "scan_bytes": scan_bytes,
+        "scan_GBs": scan_bytes / scan_us / 1e3,
         "scan_frac_hbm": scan_bytes / scan_us / 1e3 / peak_gbs,
         "scan_alg_flops": alg_flops, "scan_exec_flops": exec_flops,
         "scan_alg_TFLOPs": alg_flops / scan_us / 1e6,
