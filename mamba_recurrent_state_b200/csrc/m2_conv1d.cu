@@ -191,9 +191,27 @@ conv1d_kernel(const ConvArgs a) {
 // (96 registers), which the latency of the conv's FMA and SiLU chains needs.
 constexpr int kTileThreads = 128;
 constexpr int kTileCh = 256;   // channels per CTA
-constexpr int kTileTok = 32;   // tokens per tile
-constexpr int kTileMinBlocks = 5;
-constexpr int kMaxTilesPerCta = 8;  // token tiles a CTA walks, double-buffered (at most)
+// Tuning knobs (compile-time): tokens per tile, tile buffers in flight per
+// CTA, resident CTAs per SM the register budget is sized for, tiles a CTA walks
+// at most. Measured on the 8 x 2048 Nemotron-H prefill: 32 tokens, 2 buffers,
+// 5 CTAs per SM 149.5-151.6 us; 32, 3, 4: 170-172 us; 16, 4, 5: 168-169 us;
+// 16, 3, 5: 169-170 us.
+#ifndef M2_CONV_TILE_TOK
+#define M2_CONV_TILE_TOK 32
+#endif
+#ifndef M2_CONV_NBUF
+#define M2_CONV_NBUF 2
+#endif
+#ifndef M2_CONV_MINB
+#define M2_CONV_MINB 5
+#endif
+#ifndef M2_CONV_MAXTILES
+#define M2_CONV_MAXTILES 8
+#endif
+constexpr int kTileTok = M2_CONV_TILE_TOK;   // tokens per tile
+constexpr int kTileBufs = M2_CONV_NBUF;      // tile buffers in flight per CTA
+constexpr int kTileMinBlocks = M2_CONV_MINB;
+constexpr int kMaxTilesPerCta = M2_CONV_MAXTILES;  // token tiles a CTA walks (at most)
 constexpr uint64_t kTileWaitNs = 1000000000ull;
 
 // (wider convs keep more taps per channel in registers: three CTAs per SM)
@@ -208,8 +226,8 @@ __global__ void __launch_bounds__(kTileThreads, K <= 4 ? kTileMinBlocks : 3) con
     // this one is computed
     extern __shared__ __align__(128) uint8_t s_conv_dyn[];
     AT (*s_buf)[ROWS][kTileCh] = reinterpret_cast<AT (*)[ROWS][kTileCh]>(s_conv_dyn);
-    __shared__ __align__(8) uint64_t s_bar[2];
-    __shared__ __align__(8) uint64_t s_empty[2];  // arrivals of the 4 warps done with buffer q
+    __shared__ __align__(8) uint64_t s_bar[kTileBufs];
+    __shared__ __align__(8) uint64_t s_empty[kTileBufs];  // arrivals of the 4 warps done with buffer q
 
     const int tid = threadIdx.x;
     const int b = blockIdx.z;
@@ -251,10 +269,11 @@ __global__ void __launch_bounds__(kTileThreads, K <= 4 ? kTileMinBlocks : 3) con
         bias[e] = (ok && a.b) ? to_f32(static_cast<const AT*>(a.b)[c]) : 0.f;
     }
     if (tid == 0) {
-        mbar_init(&s_bar[0], 1);
-        mbar_init(&s_bar[1], 1);
-        mbar_init(&s_empty[0], kTileThreads / 32);
-        mbar_init(&s_empty[1], kTileThreads / 32);
+#pragma unroll
+        for (int q = 0; q < kTileBufs; ++q) {
+            mbar_init(&s_bar[q], 1);
+            mbar_init(&s_empty[q], kTileThreads / 32);
+        }
         fence_mbar_init();
     }
     __syncthreads();
@@ -277,23 +296,27 @@ __global__ void __launch_bounds__(kTileThreads, K <= 4 ? kTileMinBlocks : 3) con
         }
     };
     const int first = blockIdx.y * kTileTok;
-    if (first < T) issue(first, 0);
-    if (first + stride < T) issue(first + stride, 1);
+#pragma unroll
+    for (int q = 0; q < kTileBufs; ++q)
+        if (first + q * stride < T) issue(first + q * stride, q);
+    // tiles j+1 .. j+kTileBufs-1 may be in flight into the other buffers: a
+    // warp that leaves early lets them land first (bounded)
+    auto drain = [&](int j, int t0) {
+        for (int i = 1; i < kTileBufs; ++i)
+            if (t0 + i * stride < T)
+                mbar_wait_bounded(&s_bar[(j + i) % kTileBufs], ((j + i) / kTileBufs) & 1, kTileWaitNs);
+    };
 
     __half2 hmax = __float2half2_rn(0.f);  // largest |fp16 output| (packed)
-    uint32_t phase = 0;  // bit q: parity of buffer q's next completion
 #pragma unroll 1
     for (int j = 0, t0 = first; t0 < T; ++j, t0 += stride) {
-        const int q = j & 1;
-        const uint32_t par = (phase >> q) & 1u;
+        const int q = j % kTileBufs;
+        const uint32_t par = (j / kTileBufs) & 1;  // tile j is buffer q's (j / kTileBufs)-th fill
         const bool ok = mbar_wait_bounded(&s_bar[q], par, kTileWaitNs);
-        phase ^= 1u << q;
         if (!__all_sync(0xffffffffu, ok)) {
             if ((tid & 31) == 0) record_error(a.error, M2_ERR_TIMEOUT);
-            // let this CTA's copies land (bounded) before this warp leaves:
-            // this buffer's, and the next tile's in the other buffer if issued
             if (!ok) mbar_wait_bounded(&s_bar[q], par, kTileWaitNs);
-            if (t0 + stride < T) mbar_wait_bounded(&s_bar[q ^ 1], (phase >> (q ^ 1)) & 1u, kTileWaitNs);
+            drain(j, t0);
             return;
         }
         AT (*s_rows)[kTileCh] = s_buf[q];
@@ -344,15 +367,14 @@ __global__ void __launch_bounds__(kTileThreads, K <= 4 ? kTileMinBlocks : 3) con
         // (no block barrier: a warp that finishes early goes on to the next tile)
         __syncwarp();
         if ((tid & 31) == 0) mbar_arrive(&s_empty[q]);
-        if (tid < 32 && t0 + 2 * stride < T) {
-            const bool eok = mbar_wait_bounded(&s_empty[q], (j >> 1) & 1, kTileWaitNs);
+        if (tid < 32 && t0 + kTileBufs * stride < T) {
+            const bool eok = mbar_wait_bounded(&s_empty[q], (j / kTileBufs) & 1, kTileWaitNs);
             if (!__all_sync(0xffffffffu, eok)) {
                 if (tid == 0) record_error(a.error, M2_ERR_TIMEOUT);
-                // the next tile's copies into the other buffer, if issued, land (bounded)
-                if (t0 + stride < T) mbar_wait_bounded(&s_bar[q ^ 1], (phase >> (q ^ 1)) & 1u, kTileWaitNs);
+                drain(j, t0);
                 return;
             }
-            issue(t0 + 2 * stride, q);  // the tile after next lands in buffer q
+            issue(t0 + kTileBufs * stride, q);  // tile j + kTileBufs lands in buffer q
         }
     }
     if (fmaxf(__low2float(hmax), __high2float(hmax)) >= 65520.f)
@@ -373,7 +395,7 @@ __global__ void __launch_bounds__(kTileThreads, K <= 4 ? kTileMinBlocks : 3) con
 
 template <typename OT, int K>
 cudaError_t conv_tile_launch(const ConvArgs& a, dim3 grid, cudaStream_t s) {
-    constexpr size_t smem = 2 * static_cast<size_t>(kTileTok + K - 1) * kTileCh * sizeof(bf16_t);
+    constexpr size_t smem = kTileBufs * static_cast<size_t>(kTileTok + K - 1) * kTileCh * sizeof(bf16_t);
     static AttrOnce attrs;
     const cudaError_t e = attrs.ensure([] {
         return cudaFuncSetAttribute(conv1d_tile_kernel<OT, K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
