@@ -188,7 +188,8 @@ m2_status m2_cache_zero_slots(const m2_cache* c, int32_t n, const int32_t* slot_
 namespace {
 
 m2_status conv1d_impl(const m2_cache* c, const m2_conv_params* conv, int32_t batch, int32_t seqlen,
-                      const int32_t* cu_seqlens, const void* xBC, int64_t xBC_row_stride, void* xBC_out,
+                      const int32_t* cu_seqlens, int64_t total_rows, const void* xBC, int64_t xBC_row_stride,
+                      void* xBC_out,
                       int32_t out_dtype, int64_t out_row_stride, const int32_t* slot_idx, m2_stream stream) {
     const m2_status st = cache_status(c);
     if (st != M2_OK) return st;
@@ -227,6 +228,7 @@ m2_status conv1d_impl(const m2_cache* c, const m2_conv_params* conv, int32_t bat
     a.out_stride = out_row_stride;
     a.slot_idx = slot_idx;
     a.cu_seqlens = cu_seqlens;
+    a.total_rows = total_rows;
     return from_cuda(m2::launch_conv1d_update(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -235,8 +237,8 @@ m2_status conv1d_impl(const m2_cache* c, const m2_conv_params* conv, int32_t bat
 m2_status m2_conv1d_update(const m2_cache* c, const m2_conv_params* conv, int32_t batch, int32_t seqlen,
                            const void* xBC, int64_t xBC_row_stride, void* xBC_out, int32_t out_dtype,
                            int64_t out_row_stride, const int32_t* slot_idx, m2_stream stream) {
-    return conv1d_impl(c, conv, batch, seqlen, nullptr, xBC, xBC_row_stride, xBC_out, out_dtype, out_row_stride,
-                       slot_idx, stream);
+    return conv1d_impl(c, conv, batch, seqlen, nullptr, static_cast<int64_t>(batch) * seqlen, xBC, xBC_row_stride,
+                       xBC_out, out_dtype, out_row_stride, slot_idx, stream);
 }
 
 m2_status m2_conv1d_update_varlen(const m2_cache* c, const m2_conv_params* conv, int32_t nseq,
@@ -248,8 +250,8 @@ m2_status m2_conv1d_update_varlen(const m2_cache* c, const m2_conv_params* conv,
     if (nseq > 0 && total_tokens > 0 && !cu_seqlens) return M2_ERR_INVALID_ARG;
     // no tokens: validate and return, as a zero-length fixed call does
     const int32_t len = (nseq == 0 || total_tokens == 0) ? 0 : std::max(max_seqlen, 1);
-    return conv1d_impl(c, conv, nseq, len, cu_seqlens, xBC, xBC_row_stride, xBC_out, out_dtype, out_row_stride,
-                       slot_idx, stream);
+    return conv1d_impl(c, conv, nseq, len, cu_seqlens, total_tokens, xBC, xBC_row_stride, xBC_out, out_dtype,
+                       out_row_stride, slot_idx, stream);
 }
 
 namespace {
@@ -661,8 +663,8 @@ m2_status m2_mixed_step(const m2_cache* c, const m2_ssm_params* ssm, const m2_co
         const m2_prefill_rows& p = *prefill;
         if (p.total_tokens > INT32_MAX) return M2_ERR_UNSUPPORTED;
         if (!p.cu_seqlens || !p.xBC_post) return M2_ERR_INVALID_ARG;
-        m2_status r = conv1d_impl(c, conv, p.nseq, std::max(p.max_seqlen, 1), p.cu_seqlens, p.xBC,
-                                  p.xBC_row_stride, p.xBC_post, p.xBC_post_dtype, p.xBC_post_row_stride,
+        m2_status r = conv1d_impl(c, conv, p.nseq, std::max(p.max_seqlen, 1), p.cu_seqlens, p.total_tokens,
+                                  p.xBC, p.xBC_row_stride, p.xBC_post, p.xBC_post_dtype, p.xBC_post_row_stride,
                                   p.slot_idx, stream);
         if (r != M2_OK) return r;
         m2::ScanArgs a{};

@@ -1186,26 +1186,21 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
     }
 }
 
-// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
-using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+}  // namespace
 
-EncodeFn encode_fn() {
+TensorMapEncodeFn tensor_map_encoder() {
     static std::once_flag once;
-    static EncodeFn fn = nullptr;
+    static TensorMapEncodeFn fn = nullptr;
     std::call_once(once, [] {
         void* p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeFn>(p);
+            fn = reinterpret_cast<TensorMapEncodeFn>(p);
         cudaGetLastError();
     });
     return fn;
 }
-
-}  // namespace
 
 bool chunk_scan_tc_supported(const ScanArgs& a) {
     return a.P == kP && a.N == kN && a.state_bf16 && a.act_bf16 &&
@@ -1245,7 +1240,7 @@ __global__ void __launch_bounds__(256) seg_combine_kernel(const ScanArgs a) {
 }
 
 cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t stream) {
-    EncodeFn enc = encode_fn();
+    TensorMapEncodeFn enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
     // xBC as a 2-D tensor (channel, packed token row), 64 x 128 boxes of 16-bit
     // elements, 128-byte swizzle; rows past the end of the buffer read as zeros

@@ -1,6 +1,7 @@
 // m2_device.cuh -- small device helpers shared by the libm2 kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
@@ -141,6 +142,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                      smem_addr(bar)),
                  "r"(bytes)
                  : "memory");
+}
+
+// One 2-D TMA tile load (no multicast) of the box at element coordinates
+// (x, y) of `map` into shared memory at `dst`, completing the box's bytes on
+// `bar`. x times the element size must be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_tile_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];\n" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y)
+        : "memory");
 }
 
 // Plain arrive (release): one of the barrier's expected arrivals.

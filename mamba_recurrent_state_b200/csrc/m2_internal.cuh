@@ -2,6 +2,7 @@
 // Not installed; the public ABI is include/m2.h.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -10,6 +11,14 @@
 #include "m2.h"
 
 namespace m2 {
+
+// cuTensorMapEncodeTiled, reached through the runtime's driver entry point (no
+// -lcuda); nullptr when the driver does not provide it.
+using TensorMapEncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                       const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                       CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                       CUtensorMapFloatOOBfill);
+TensorMapEncodeFn tensor_map_encoder();
 
 // Runs a kernel's one-time function-attribute setup once per device (the
 // attributes belong to the device's context). Concurrent first calls may both
@@ -80,6 +89,7 @@ struct ConvArgs {
     // variable-length batches: sequence b is packed rows cu_seqlens[b] ..
     // cu_seqlens[b+1]-1 (NULL: rows b*seqlen ..); seqlen then bounds the grid
     const int32_t* cu_seqlens;
+    int64_t total_rows;  // rows of x (batch * seqlen, or the packed total)
 };
 
 struct ZeroArgs {
