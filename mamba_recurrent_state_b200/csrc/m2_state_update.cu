@@ -12,10 +12,12 @@
 //  * A sequence's state [H, P, N] is a run of H*P rows of N elements. One CTA
 //    of 256 threads owns TILE consecutive rows, one contiguous block of the
 //    cache (64 KB in the main configuration), split in CHUNKS chunks.
-//  * Right after reading its slot index, one thread issues the whole tile as
-//    bulk asynchronous copies (cp.async.bulk) into shared memory, one
-//    mbarrier per chunk, so the tile's bytes are in flight while the CTA runs
-//    the conv tap and the per-head scalars. Registers are not used as the
+//  * Right after reading its slot index, one thread issues the slot's conv
+//    rows (fused: three 2-D TMA boxes, the tile's x rows and the group's B and
+//    C rows, where the shared-memory layout allows; else row by row) and the
+//    whole tile as bulk asynchronous copies (cp.async.bulk) into shared
+//    memory, one mbarrier per chunk, so the tile's bytes are in flight while
+//    the CTA runs the conv tap and the per-head scalars. Registers are not used as the
 //    staging buffer, which lets three CTAs share an SM.
 //  * A state row is handled by LPR = N*sizeof(state)/16 lanes, one 16-byte
 //    vector each, so every lane keeps the same EPV state columns n for all of
@@ -33,6 +35,8 @@
 //    reading the B/C conv rows, and only cluster rank 0 waits on it (at the
 //    very end) and then writes the rolled B/C rows.
 #include <cuda_runtime.h>
+
+#include <climits>
 
 #include "m2_device.cuh"
 #include "m2_internal.cuh"
@@ -194,9 +198,13 @@ __device__ __forceinline__ bool conv_vec_any(const ConvIn& in, const AT* w, int6
 // stored. The norm's channel group (the hpg*P rows of an SSM group) is exactly
 // the CTA cluster, so the group's sum of squares is exchanged through
 // distributed shared memory.
+// map_cx / map_cbc (fused, use_tma): the conv cache as (channel, slot*(K-1) + k)
+// with boxes of TILE and of N channels x K-1 rows, for the tile's x rows and
+// the group's B and C rows; use_tma = 0: every row is a bulk copy.
 template <typename ST, typename AT, typename XT, int N, int CHUNKS, int VPT, bool FUSED, bool NORM>
 __global__ void __launch_bounds__(kThreads, M2_DECODE_MIN_BLOCKS)
-state_update_kernel(const StateUpdateArgs a) {
+state_update_kernel(const __grid_constant__ CUtensorMap map_cx, const __grid_constant__ CUtensorMap map_cbc,
+                    const StateUpdateArgs a, const int use_tma) {
     static_assert(FUSED || !NORM, "the norm exchange needs the group cluster of the fused launch");
     constexpr int EPV = Vec16<ST>::n;       // state elements per 16-byte vector
     constexpr int LPR = N / EPV;            // lanes per state row
@@ -215,11 +223,11 @@ state_update_kernel(const StateUpdateArgs a) {
     constexpr uint32_t BROW_BYTES = N * sizeof(AT);
     constexpr int kHalf = kThreads / 2;     // x-conv threads | B/C-conv threads
 
-    // dynamic: [state tile | conv rows of the tile's x channels | conv rows of B, C]
+    // dynamic: [state tile | conv rows of the tile's x channels | conv rows of B, then of C]
     extern __shared__ __align__(128) uint8_t s_dyn[];
     uint8_t* s_tile = s_dyn;
     const AT* s_cx = reinterpret_cast<const AT*>(s_dyn + TILE_BYTES);                 // [K-1][TILE]
-    const AT* s_cbc = reinterpret_cast<const AT*>(s_dyn + TILE_BYTES + (a.K - 1) * XROW_BYTES);  // [K-1][2][N]
+    const AT* s_cbc = reinterpret_cast<const AT*>(s_dyn + TILE_BYTES + (a.K - 1) * XROW_BYTES);  // [2][K-1][N]
     __shared__ __align__(8) uint64_t s_bar[CHUNKS + 1];  // one per state chunk, one for the conv rows
     __shared__ __align__(16) float4 s_rp[TILE];          // per row: dt*x, dA, D*x
     __shared__ __align__(16) float s_B[N];
@@ -340,12 +348,18 @@ state_update_kernel(const StateUpdateArgs a) {
         if constexpr (FUSED) {
             mbar_arrive_expect_tx(bar_conv, (K - 1) * (XROW_BYTES + 2 * BROW_BYTES));
             uint8_t* dst = s_dyn + TILE_BYTES;
-            for (int k = 0; k < K - 1; ++k)
-                bulk_g2s(dst + k * XROW_BYTES, conv0 + k * cd + r0, XROW_BYTES, bar_conv);
-            dst += (K - 1) * XROW_BYTES;
-            for (int k = 0; k < K - 1; ++k) {
-                bulk_g2s(dst + (2 * k) * BROW_BYTES, conv0 + k * cd + cB, BROW_BYTES, bar_conv);
-                bulk_g2s(dst + (2 * k + 1) * BROW_BYTES, conv0 + k * cd + cC, BROW_BYTES, bar_conv);
+            uint8_t* dbc = dst + (K - 1) * XROW_BYTES;
+            if (use_tma) {  // three 2-D boxes: the x rows, the B rows, the C rows
+                const int crow = slot * (K - 1);
+                tma_load_tile_2d(dst, &map_cx, static_cast<int>(r0), crow, bar_conv);
+                tma_load_tile_2d(dbc, &map_cbc, static_cast<int>(cB), crow, bar_conv);
+                tma_load_tile_2d(dbc + (K - 1) * BROW_BYTES, &map_cbc, static_cast<int>(cC), crow, bar_conv);
+            } else {
+                for (int k = 0; k < K - 1; ++k) {
+                    bulk_g2s(dst + k * XROW_BYTES, conv0 + k * cd + r0, XROW_BYTES, bar_conv);
+                    bulk_g2s(dbc + k * BROW_BYTES, conv0 + k * cd + cB, BROW_BYTES, bar_conv);
+                    bulk_g2s(dbc + (K - 1 + k) * BROW_BYTES, conv0 + k * cd + cC, BROW_BYTES, bar_conv);
+                }
             }
         }
 #pragma unroll
@@ -391,8 +405,8 @@ state_update_kernel(const StateUpdateArgs a) {
                     row_pitch = TILE;
                 } else {
                     const int u = v - XV;
-                    rows = s_cbc + (u / BV) * N + (u % BV) * AV + sub * CQ;
-                    row_pitch = 2 * N;
+                    rows = s_cbc + (u / BV) * (K - 1) * N + (u % BV) * AV + sub * CQ;
+                    row_pitch = N;
                 }
                 if (q != tid) qin = load_quad_in<AT>(xrow, w, bias, c0);
                 float wf[4 * CQ], out[CQ], xv[CQ];
@@ -456,8 +470,8 @@ state_update_kernel(const StateUpdateArgs a) {
                 const int seg = v / BV;                        // 0 = B, 1 = C
                 const int j0 = (v % BV) * AV;
                 c0 = (seg ? cC : cB) + j0;
-                rows = s_cbc + seg * N + j0;
-                row_pitch = 2 * N;
+                rows = s_cbc + seg * (K - 1) * N + j0;
+                row_pitch = N;
             }
             if (v != v_first) cin = load_conv_in<AT>(xrow, w, bias, c0, K);
             const uint4 xin = cin.xin;
@@ -624,9 +638,9 @@ state_update_kernel(const StateUpdateArgs a) {
                 const int seg = v / BV;
                 const int j0 = (v % BV) * AV;
                 const int64_t c0 = (seg ? cC : cB) + j0;
-                const AT* rows = s_cbc + seg * N + j0;
+                const AT* rows = s_cbc + seg * (K - 1) * N + j0;
                 for (int k = 0; k < K - 1; ++k) {
-                    const uint4 nv = (k < K - 2) ? *reinterpret_cast<const uint4*>(rows + (k + 1) * 2 * N)
+                    const uint4 nv = (k < K - 2) ? *reinterpret_cast<const uint4*>(rows + (k + 1) * N)
                                                  : *reinterpret_cast<const uint4*>(xrow + c0);
                     *reinterpret_cast<uint4*>(conv0 + k * cd + c0) = nv;
                 }
@@ -672,7 +686,36 @@ cudaError_t launch_one(const StateUpdateArgs& a, const DecodePlan& plan, cudaStr
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, kern, a);
+    // fused: the slot's conv rows by three 2-D TMA boxes where the cache allows
+    // it (16-byte row pitch, row coordinates in 32 bits) and each box lands on
+    // a 128-byte boundary of shared memory, as a tensor copy requires (the B
+    // rows follow K-1 x rows of TILE channels, the C rows K-1 B rows);
+    // otherwise row by row
+    CUtensorMap map_cx{}, map_cbc{};
+    int use_tma = 0;
+    if constexpr (FUSED) {
+        const TensorMapEncodeFn enc = tensor_map_encoder();
+        const int64_t as = sizeof(AT);
+        const int64_t rows = a.num_slots * (a.K - 1);
+        const int64_t off_b = static_cast<int64_t>(TILE) * N * sizeof(ST) + (a.K - 1) * TILE * as;
+        const int64_t off_c = off_b + (a.K - 1) * N * as;
+        if (enc && (a.conv_dim * as) % 16 == 0 && rows <= INT32_MAX && off_b % 128 == 0 && off_c % 128 == 0) {
+            const CUtensorMapDataType dt =
+                sizeof(AT) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+            const cuuint64_t dims[2] = {static_cast<cuuint64_t>(a.conv_dim), static_cast<cuuint64_t>(rows)};
+            const cuuint64_t strides[1] = {static_cast<cuuint64_t>(a.conv_dim * as)};
+            const cuuint32_t estr[2] = {1, 1};
+            const cuuint32_t box_x[2] = {static_cast<cuuint32_t>(TILE), static_cast<cuuint32_t>(a.K - 1)};
+            const cuuint32_t box_bc[2] = {static_cast<cuuint32_t>(N), static_cast<cuuint32_t>(a.K - 1)};
+            use_tma = enc(&map_cx, dt, 2, a.conv, dims, strides, box_x, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS &&
+                      enc(&map_cbc, dt, 2, a.conv, dims, strides, box_bc, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+        }
+    }
+    return cudaLaunchKernelEx(&cfg, kern, map_cx, map_cbc, a, use_tma);
 }
 
 template <typename ST, typename AT, typename XT, int N, bool FUSED, bool NORM>
