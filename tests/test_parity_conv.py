@@ -92,3 +92,72 @@ def test_conv_fp16_range_error():
     m2.conv1d_update(cache, conv, x, torch.tensor([1], dtype=torch.int32, device="cuda"),
                      out_dtype=torch.float16)
     assert cache.device_error() == m2.M2_ERR_RANGE
+
+
+def _tile_case(index, K, batch, slots):
+    # conv_dim = 10*32 + 2*2*64 = 576: two full 256-channel blocks and a
+    # 64-channel partial one
+    return W.Workload(index, f"convtile{index}", 10, 32, 64, 2, K, S.BF16, S.BF16, slots, batch)
+
+
+@pytest.mark.parametrize("K,T,od", [(4, 33000, torch.float16), (2, 4133, torch.bfloat16),
+                                    (5, 70, torch.float32)],
+                         ids=["K4-ring-f16", "K2-bf16", "K5-short-f32"])
+def test_conv_tile_kernel(K, T, od):
+    """The shared-memory tile kernel (bf16 input, >= 32 tokens): a partial last
+    channel block, a ragged last tile, the first tile staged from the conv
+    cache, and -- at 33000 tokens -- several tiles per CTA, so the buffers are
+    refilled while the other is computed; the last tile's 2-D box reaches past
+    the sequence (into the next row's tokens, or past the buffer)."""
+    w = _tile_case(260 + K, K, batch=2, slots=5)
+    cache = make_cache(w)
+    conv0 = cache.conv.clone()
+    _, _, conv = layer_objs(w)
+    slot_list = [3, 1]
+    slots = torch.tensor(slot_list, dtype=torch.int32, device="cuda")
+    x = TI.step_tensors(w, 0, rows=w.batch * T)["xBC"].view(w.batch, T, w.conv_dim)
+    out = m2.conv1d_update(cache, conv, x, slots, out_dtype=od)
+    torch.cuda.synchronize()
+    assert cache.device_error() == 0
+    ol = OracleLayer(w)
+    out_code = {torch.float32: S.F32, torch.bfloat16: S.BF16, torch.float16: S.F16}[od]
+    tol = {S.F32: 1e-5, S.BF16: 2e-2, S.F16: 1e-3}[out_code]
+    for b, s in enumerate(slot_list):
+        state = ol.initial_conv(s)
+        xr = f64(W.step_rows(w, T_XBC, 0, np.arange(b * T, (b + 1) * T)), w.act_dtype)
+        ref = ol.orc.conv1d(state, xr, ol.conv_w, ol.conv_b, 1)
+        assert_close(f64(TI.to_storage_np(out[b]), out_code), ref, S.F32, f"row {b}", tol=tol)
+        assert np.array_equal(TI.to_storage_np(cache.conv[s]), S.to_storage(state, w.act_dtype))
+    keep = [s for s in range(w.num_slots) if s not in slot_list]
+    assert torch.equal(cache.conv[keep], conv0[keep])
+
+
+def test_conv_tile_kernel_varlen():
+    """Packed sequences of 4100, 31 (below one tile), 0 (empty) and 2050
+    tokens through the tile kernel: a tile's box may hold rows of the next
+    sequence, which are never read; the empty sequence leaves its slot
+    untouched."""
+    lens = [4100, 31, 0, 2050]
+    w = _tile_case(270, 4, batch=len(lens), slots=6)
+    cache = make_cache(w)
+    conv0 = cache.conv.clone()
+    _, _, conv = layer_objs(w)
+    slot_list = [5, 0, 2, 4]
+    slots = torch.tensor(slot_list, dtype=torch.int32, device="cuda")
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    total = int(cu[-1])
+    x = TI.step_tensors(w, 0, rows=total)["xBC"]
+    out = m2.conv1d_update_varlen(cache, conv, x, torch.from_numpy(cu).cuda(), slots, max(lens),
+                                  out_dtype=torch.float16)
+    torch.cuda.synchronize()
+    assert cache.device_error() == 0
+    ol = OracleLayer(w)
+    for b, s in enumerate(slot_list):
+        if lens[b] == 0:
+            assert torch.equal(cache.conv[s], conv0[s])
+            continue
+        state = ol.initial_conv(s)
+        xr = f64(W.step_rows(w, T_XBC, 0, np.arange(cu[b], cu[b + 1])), w.act_dtype)
+        ref = ol.orc.conv1d(state, xr, ol.conv_w, ol.conv_b, 1)
+        assert_close(f64(TI.to_storage_np(out[cu[b]:cu[b + 1]]), S.F16), ref, S.F32, f"seq {b}", tol=1e-3)
+        assert np.array_equal(TI.to_storage_np(cache.conv[s]), S.to_storage(state, w.act_dtype))
