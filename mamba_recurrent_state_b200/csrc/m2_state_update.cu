@@ -232,6 +232,8 @@ state_update_kernel(const __grid_constant__ CUtensorMap map_cx, const __grid_con
     __shared__ __align__(16) float4 s_rp[TILE];          // per row: dt*x, dA, D*x
     __shared__ __align__(16) float s_B[N];
     __shared__ __align__(16) float s_C[N];
+    // (fused, K = 4) the raw B and C inputs of this step, for cluster rank 0's roll
+    __shared__ __align__(16) uint32_t s_rawbc[2 * N * sizeof(AT) / 4];
     __shared__ float s_y[TILE];
     __shared__ float s_dt[kMaxHeadsPerTile];
     __shared__ float s_dA[kMaxHeadsPerTile];
@@ -321,9 +323,13 @@ state_update_kernel(const __grid_constant__ CUtensorMap map_cx, const __grid_con
         hs_alog = a.A_log[h];
         hs_D = a.D[h];
     }
-    // (c) z of this thread's first y row
+    // (c) z of this thread's first y row (and its norm weight)
     float z_first = 0.f;
     if (zrow && tid < TILE) z_first = to_f32(zrow[r0 + tid]);
+    float nw_first = 0.f;
+    if constexpr (NORM) {
+        if (tid < TILE) nw_first = to_f32(static_cast<const AT*>(a.norm_w)[r0 + tid]);
+    }
 
     const int32_t slot = a.slot_idx[b];
 
@@ -453,6 +459,7 @@ state_update_kernel(const __grid_constant__ CUtensorMap map_cx, const __grid_con
                     float* dstf = (u / BV) ? s_C : s_B;
 #pragma unroll
                     for (int e = 0; e < CQ; ++e) dstf[(u % BV) * AV + sub * CQ + e] = out[e];
+                    s_rawbc[((u / BV) * N + (u % BV) * AV + sub * CQ) * sizeof(AT) / 4] = qin.xin;
                 }
             }
         } else {
@@ -622,7 +629,7 @@ state_update_kernel(const __grid_constant__ CUtensorMap map_cx, const __grid_con
             const AT* nw = static_cast<const AT*>(a.norm_w);
             const float rstd = s_rstd;
             for (int i = tid; i < TILE; i += kThreads)
-                yrow[r0 + i] = from_f32<AT>(s_y[i] * rstd * to_f32(nw[r0 + i]));
+                yrow[r0 + i] = from_f32<AT>(s_y[i] * rstd * (i == tid ? nw_first : to_f32(nw[r0 + i])));
         }
     }
 
@@ -640,8 +647,11 @@ state_update_kernel(const __grid_constant__ CUtensorMap map_cx, const __grid_con
                 const int64_t c0 = (seg ? cC : cB) + j0;
                 const AT* rows = s_cbc + seg * (K - 1) * N + j0;
                 for (int k = 0; k < K - 1; ++k) {
-                    const uint4 nv = (k < K - 2) ? *reinterpret_cast<const uint4*>(rows + (k + 1) * N)
-                                                 : *reinterpret_cast<const uint4*>(xrow + c0);
+                    // the newest row is this step's raw input: staged by the K = 4 conv
+                    const uint4 nv =
+                        (k < K - 2) ? *reinterpret_cast<const uint4*>(rows + (k + 1) * N)
+                        : (K == 4)  ? *reinterpret_cast<const uint4*>(&s_rawbc[(seg * N + j0) * sizeof(AT) / 4])
+                                    : *reinterpret_cast<const uint4*>(xrow + c0);
                     *reinterpret_cast<uint4*>(conv0 + k * cd + c0) = nv;
                 }
             }
