@@ -147,6 +147,29 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Two blocks of 16 consecutive fp32 columns of this thread's TMEM lane (at
+// taddr_a and taddr_b), with one wait for both loads.
+__device__ __forceinline__ void tmem_ld16x2(uint32_t taddr_a, uint32_t taddr_b, float (&va)[16], float (&vb)[16]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%33];\n"
+        "tcgen05.wait::ld.sync.aligned;\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr_a), "r"(taddr_b)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        va[i] = __uint_as_float(r[i]);
+        vb[i] = __uint_as_float(r[16 + i]);
+    }
+}
+
 // 2^x with the hardware approximation (PTX ex2.approx, relative error about
 // 2^-22); the decay sums are kept in log2 units so exp(c) = 2^(c log2 e).
 __device__ __forceinline__ float ex2(float x) {
@@ -1130,8 +1153,7 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 float yd[16], yo[16];
-                tmem_ld16(tq + lane_base + 64 + h2 * 32 + 16 * hh, yd);
-                tmem_ld16(tq + lane_base + 192 + h2 * 32 + 16 * hh, yo);
+                tmem_ld16x2(tq + lane_base + 64 + h2 * 32 + 16 * hh, tq + lane_base + 192 + h2 * 32 + 16 * hh, yd, yo);
 #pragma unroll
                 for (int jh = 0; jh < 2; ++jh) {
                     const int jj = 2 * hh + jh;
