@@ -183,8 +183,8 @@ conv1d_kernel(const ConvArgs a) {
 // arrive in shared memory as one 2-D TMA box of x; the first tile of a
 // sequence, whose rows before the sequence start come from the slot's conv
 // cache, is staged row by row with bulk copies by warp 0 (as is every tile
-// when x's rows are not 16-byte aligned). One box instead of 35 row copies
-// per tile: 134 us instead of 151.6 us for 8 x 2048 Nemotron-H tokens, whose
+// when the box does not apply). One box instead of 35 row copies per tile:
+// 132-134 us instead of 151.6 us for 8 x 2048 Nemotron-H tokens, whose
 // 35 copies of 512 bytes per tile kept the copy engine, not DRAM, busy (the
 // copies alone, with no arithmetic, took 84 us). Every thread then computes 8
 // tokens of one 16-byte channel vector from shared memory, two channels at a
@@ -199,9 +199,10 @@ constexpr int kTileThreads = 128;
 constexpr int kTileCh = 256;   // channels per CTA
 // Tuning knobs (compile-time): tokens per tile, tile buffers in flight per
 // CTA, resident CTAs per SM the register budget is sized for, tiles a CTA walks
-// at most. Measured on the 8 x 2048 Nemotron-H prefill with row-by-row copies:
-// 32 tokens, 2 buffers, 5 CTAs per SM 149.5-151.6 us; 32, 3, 4: 170-172 us;
-// 16, 4, 5: 168-169 us; 16, 3, 5: 169-170 us.
+// at most. Measured on the 8 x 2048 Nemotron-H prefill with one box per tile:
+// 32 tokens, 2 buffers, 5 CTAs per SM, 8 tiles 132-134 us; 16 tiles 137 us;
+// 32, 2, 4: 143 us; 32, 3, 4: 144 us; 16, 4, 5: 145 us. (With row-by-row
+// copies: 149.5-151.6, 170-172 for 32, 3, 4, 168-170 for 16-token tiles.)
 #ifndef M2_CONV_TILE_TOK
 #define M2_CONV_TILE_TOK 32
 #endif
