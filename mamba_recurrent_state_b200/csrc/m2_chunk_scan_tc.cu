@@ -770,6 +770,7 @@ __global__ void __launch_bounds__(kP2Threads, 1)
 chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs a) {
     extern __shared__ uint8_t s_raw[];
     __shared__ __align__(8) uint64_t s_full[2], s_cb[2], s_m[2], s_d[2], s_yoff[2], s_free[2], s_tfree[2];
+    __shared__ __align__(8) uint64_t s_w[2];  // W of stage q is built (every epilogue-1 thread arrives)
     __shared__ __align__(8) uint64_t s_sready[2];  // state copy (i & 1) holds the state entering chunk i
     __shared__ __align__(8) uint64_t s_drain;
     __shared__ uint32_t s_tmem;
@@ -831,7 +832,8 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
         for (int q = 0; q < 2; ++q) {
             mbar_init(&s_full[q], 1);
             mbar_init(&s_cb[q], 1);
-            mbar_init(&s_m[q], 1);
+            mbar_init(&s_m[q], 256);  // every epilogue-1 thread, once its rows of M are in TMEM
+            mbar_init(&s_w[q], 256);
             mbar_init(&s_d[q], 1);
             mbar_init(&s_yoff[q], 1);
             mbar_init(&s_free[q], 1);
@@ -924,9 +926,11 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
                 mma_commit(&s_yoff[q]);
                 if (!p2_wait(&s_m[q], par, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                for (int k = 0; k < kQ / 16; ++k)  // Ydiag = M . X (M from TMEM)
+                for (int k = 0; k < kQ / 16; ++k)  // Ydiag = M . X (M from TMEM), while W is built
                     mma_f16_ta(tq + 64, tq + 128 + k * 8, sw128_desc(st + 65536 + k * 2048u, 16384, 1024), id_ydiag,
                                k > 0);
+                if (!p2_wait(&s_w[q], par, abort_flag)) { ok = false; break; }
+                tc_fence_after();
                 for (int k = 0; k < kQ / 16; ++k)  // dS^T = W^T . X
                     mma_f16(tq + 0, sw128_desc(st + 32768 + k * 2048u, 16384, 1024),
                             sw128_desc(st + 65536 + k * 2048u, 16384, 1024), id_ds, k > 0);
@@ -1044,6 +1048,10 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
                 }
                 tmem_st8(tq + lane_base + 128 + u0 / 2, hw);  // M row t, columns u0 .. u0+15 as fp16 pairs
             }
+            // this thread's rows of M are in TMEM: M . X may start while W is built
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive1(&s_m[q]);
             // W row t = w_t * B row t (fp16 pairs, in place)
             const float wu = (t < valid) ? ex2(cum_end - cum_t) * dt_c[t] : 0.f;
             const __half2 w2 = __float2half2_rn(wu);
@@ -1061,11 +1069,10 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
                 }
                 *pw = v;
             }
-            tmem_wait_st();
+            // W visible to the tensor cores; the next chunk's first role barrier
+            // orders this chunk's reads of s_gam and the decay sums before their reuse
             fence_proxy_async();
-            tc_fence_before();
-            role_sync_or(1, false);
-            if (e1 == 0) mbar_arrive1(&s_m[q]);
+            mbar_arrive1(&s_w[q]);
         }
     } else {
         // ------------------------------------------------------- epilogue 2
