@@ -837,7 +837,7 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
             mbar_init(&s_d[q], 1);
             mbar_init(&s_yoff[q], 1);
             mbar_init(&s_free[q], 1);
-            mbar_init(&s_tfree[q], 1);
+            mbar_init(&s_tfree[q], 256);  // every epilogue-2 thread, once it has read the stage's TMEM
         }
         mbar_init(&s_sready[0], 1);
         mbar_init(&s_sready[1], 1);
@@ -1178,10 +1178,9 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
                     if (row_ok) *reinterpret_cast<uint4*>(yrow + 8 * (h2 * 4 + jj)) = pack16<bf16_t>(out);
                 }
             }
-            // TMEM of stage q is read: chunk c+2 may reuse it
+            // this thread has read TMEM stage q: chunk c+2 may reuse it once all have
             tc_fence_before();
-            role_sync_or(2, false);
-            if (e2 == 0) mbar_arrive1(&s_tfree[q]);
+            mbar_arrive1(&s_tfree[q]);
         }
         if (ok && (!split || seg == nseg_s - 1)) {  // the sequence's final state, in place
 #pragma unroll
