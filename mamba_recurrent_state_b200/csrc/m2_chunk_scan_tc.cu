@@ -692,7 +692,7 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
 // and C S^T depend on the carried state, so here they form the sequential
 // chain while epilogue 1 of the next chunk runs beside them:
 //   warp 0        TMA producer: stage (c & 1) <- x, B, C tiles of chunk c
-//   warp 1        MMA issuer: CB, then M X and W^T X, then C S^T
+//   warp 1        MMA issuer: C S^T, M X, W^T X, then CB of the next chunk
 //   warps 2..9    epilogue 1 (256 threads): dt and decay sums, M (into TMEM,
 //                 as the A operand of M X, so the C tile stays intact for
 //                 C S^T) and W = w o B (in place in the B tile)
@@ -700,11 +700,14 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
 //                 and its fp16 copy for C S^T of chunk c+1 first, then y of
 //                 chunk c
 // Per chunk the issuer runs C S^T as soon as the state entering the chunk is
-// ready (normally while epilogue 1 still works on M), then M X and W^T X,
-// after which the stage's tiles are free for the load of chunk c+2, then CB of
-// chunk c+1. The state copy is double-buffered, so the carry (the only step
-// that must follow the previous chunk's) is not held up by C S^T of the
-// previous chunk, and y leaves the chain.
+// ready (normally while epilogue 1 still works on M), then M X as soon as
+// every epilogue-1 thread has written its rows of M (the last of them are
+// still scaling W), then W^T X once W is built, after which the stage's tiles
+// are free for the load of chunk c+2, then CB of chunk c+1 (once every
+// epilogue-2 thread has read the TMEM stage of chunk c-1). The state copy is
+// double-buffered, so the carry (the only step that must follow the previous
+// chunk's) is not held up by C S^T of the previous chunk, and y leaves the
+// chain.
 // One CTA per SM (two shared-memory stages of 80 KB and two 16 KB state
 // copies, 512 TMEM columns: per stage CB at 0..127, later dS at 0..63 and
 // Ydiag at 64..127, M at 128..191 (fp16 pairs), Yoff at 192..255). Every
