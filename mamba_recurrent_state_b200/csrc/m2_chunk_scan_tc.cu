@@ -782,6 +782,7 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
     __shared__ __align__(16) float s_dt[4][kQ];
     __shared__ __align__(16) float s_gam[192];
     __shared__ float s_wsum[kQ / 32];
+    __shared__ float s_dt0[kQ / 32];  // dt of the first row of each quarter of the chunk
     volatile int* abort_flag = &s_abort;
 
     const int tid = threadIdx.x;
@@ -955,6 +956,7 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
         bf16_t dt_raw_next = 0;
         if (h2 == 0 && c_begin * kQ + t < T)
             dt_raw_next = static_cast<const bf16_t*>(a.dt)[(row0 + c_begin * kQ + t) * a.dt_stride + h];
+        bool cb_fail = false;
         for (int i = 0; i < nloc; ++i) {
             const int c = c_begin + i;
             const int q = i & 1;
@@ -974,23 +976,30 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
                     if (lane >= off) cum += o;
                 }
                 if (lane == 31) s_wsum[quarter] = cum;
+                if (lane == 0) s_dt0[quarter] = dt;
             }
-            role_sync_or(1, false);
+            // a failed wait of the previous chunk is decided here, by all together
+            if (role_sync_or(1, cb_fail)) { s_abort = 1; break; }
             if (h2 == 0) {
                 for (int w = 0; w < quarter; ++w) cum += s_wsum[w];
                 s_cum[ring][t] = cum;
                 s_dt[ring][t] = dt;
+                // the factored decay of column t for the row quarters below it:
+                // exp(c_32bq - c_t) dt_t, c_32bq summed in the same order as row 32bq's own
+                for (int bq = quarter + 1; bq < 4; ++bq) {
+                    float cq = s_dt0[bq] * A2;
+                    for (int w = 0; w < bq; ++w) cq += s_wsum[w];
+                    s_gam[(bq == 1 ? 0 : (bq == 2 ? 32 : 96)) + t] = ex2(cq - cum) * dt;
+                }
             }
             role_sync_or(1, false);
             const float* cum_c = s_cum[ring];
             const float* dt_c = s_dt[ring];
-            if (e1 < 192) {
-                const int bq = e1 < 32 ? 1 : (e1 < 96 ? 2 : 3);
-                const int u = e1 - (bq == 1 ? 0 : (bq == 2 ? 32 : 96));
-                s_gam[e1] = ex2(cum_c[32 * bq] - cum_c[u]) * dt_c[u];
+            if (!p2_wait(&s_cb[q], par, abort_flag)) {  // the next chunk's first barrier decides
+                s_abort = 1;
+                cb_fail = true;
+                continue;
             }
-            const bool got = p2_wait(&s_cb[q], par, abort_flag);
-            if (role_sync_or(1, !got)) { s_abort = 1; break; }
             tc_fence_after();
             const uint32_t tq = tmem + q * 256;
             uint8_t* stB = sm + q * kP2Stage + 32768;
