@@ -161,3 +161,30 @@ def test_conv_tile_kernel_varlen():
         ref = ol.orc.conv1d(state, xr, ol.conv_w, ol.conv_b, 1)
         assert_close(f64(TI.to_storage_np(out[cu[b]:cu[b + 1]]), S.F16), ref, S.F32, f"seq {b}", tol=1e-3)
         assert np.array_equal(TI.to_storage_np(cache.conv[s]), S.to_storage(state, w.act_dtype))
+
+
+def test_conv_tile_kernel_strided_rows():
+    """The tile kernel on a column slice of a wider buffer (as when xBC is a
+    view of the in_proj output): rows xBC_row_stride apart, the 2-D box reading
+    only the conv_dim channels of each row."""
+    w = _tile_case(275, 4, batch=2, slots=4)
+    cache = make_cache(w)
+    _, _, conv = layer_objs(w)
+    slot_list = [2, 0]
+    slots = torch.tensor(slot_list, dtype=torch.int32, device="cuda")
+    T = 1000
+    x = TI.step_tensors(w, 0, rows=w.batch * T)["xBC"].view(w.batch, T, w.conv_dim)
+    wide = torch.full((w.batch, T, w.conv_dim + 64), 7.0, dtype=x.dtype, device="cuda")
+    wide[:, :, 32:32 + w.conv_dim] = x
+    xs = wide[:, :, 32:32 + w.conv_dim]
+    assert xs.stride(1) == w.conv_dim + 64
+    out = m2.conv1d_update(cache, conv, xs, slots, out_dtype=torch.float16)
+    torch.cuda.synchronize()
+    assert cache.device_error() == 0
+    ol = OracleLayer(w)
+    for b, s in enumerate(slot_list):
+        state = ol.initial_conv(s)
+        xr = f64(W.step_rows(w, T_XBC, 0, np.arange(b * T, (b + 1) * T)), w.act_dtype)
+        ref = ol.orc.conv1d(state, xr, ol.conv_w, ol.conv_b, 1)
+        assert_close(f64(TI.to_storage_np(out[b]), S.F16), ref, S.F32, f"row {b}", tol=1e-3)
+        assert np.array_equal(TI.to_storage_np(cache.conv[s]), S.to_storage(state, w.act_dtype))
