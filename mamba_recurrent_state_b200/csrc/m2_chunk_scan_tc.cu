@@ -719,7 +719,8 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
 constexpr int kP2Threads = 576;
 constexpr uint32_t kP2Stage = 81920;                       // C 32 KB | B 32 KB | X 16 KB
 constexpr uint32_t kP2OffS = 2 * kP2Stage;                 // two fp16 state copies, 16 KB each
-constexpr uint32_t kP2Smem = kP2OffS + 2 * 16384 + 1024;   // + alignment slack
+constexpr uint32_t kP2OffZ = kP2OffS + 2 * 16384;          // the z tile of a chunk (bf16, 16 KB)
+constexpr uint32_t kP2Smem = kP2OffZ + 16384 + 1024;       // + alignment slack
 constexpr uint32_t kP2TmemCols = 512;
 
 // D (TMEM) = A (TMEM, K-major fp16 pairs) . B (shared memory descriptor)
@@ -770,12 +771,14 @@ __device__ __forceinline__ void mbar_arrive1(uint64_t* bar) {
 
 template <typename ST>
 __global__ void __launch_bounds__(kP2Threads, 1)
-chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs a) {
+chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_z,
+                     const ScanArgs a) {
     extern __shared__ uint8_t s_raw[];
     __shared__ __align__(8) uint64_t s_full[2], s_cb[2], s_m[2], s_d[2], s_yoff[2], s_free[2], s_tfree[2];
     __shared__ __align__(8) uint64_t s_w[2];  // W of stage q is built (every epilogue-1 thread arrives)
     __shared__ __align__(8) uint64_t s_sready[2];  // state copy (i & 1) holds the state entering chunk i
     __shared__ __align__(8) uint64_t s_drain;
+    __shared__ __align__(8) uint64_t s_z;  // the z tile of the next chunk has landed
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     __shared__ __align__(16) float s_cum[4][kQ];  // ring of 4 chunks (E2 reads c & 3 while E1 writes ahead)
@@ -846,6 +849,7 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
         mbar_init(&s_sready[0], 1);
         mbar_init(&s_sready[1], 1);
         mbar_init(&s_drain, 1);
+        mbar_init(&s_z, 1);
         fence_mbar_init();
         asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
     }
@@ -864,6 +868,7 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
     float range_max = 0.f;
     __half2 hmax = __float2half2_rn(0.f);
     int loads_issued = 0;  // producer bookkeeping (lane 0 of warp 0)
+    int z_issued = 0;      // z tiles issued (epilogue-2 thread 0)
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer
@@ -1118,6 +1123,20 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
                 *reinterpret_cast<__half*>(sS + sw128(p0 + k + 1, j) + (n & 7) * 2) = __high2half(hv);
             }
         };
+        // z tile of chunk c (128 tokens x 64 channels, 128-byte swizzle) by TMA
+        // into one shared buffer, issued by e2 == 0 once every thread has read
+        // the previous one (the TMEM-free barrier of that chunk)
+        const bool gate = a.z != nullptr;
+        uint8_t* zt = sm + kP2OffZ;
+        auto load_z = [&](int c) {
+            mbar_arrive_expect_tx(&s_z, 16384u);
+            tma_load_2d(base + kP2OffZ, &tmap_z, xcol, static_cast<int>(row0 + static_cast<int64_t>(c) * kQ), &s_z);
+        };
+        bool z_fail = false;
+        if (gate && e2 == 0) {
+            load_z(c_begin);
+            z_issued = 1;
+        }
         write_state_copy(0);
         fence_proxy_async();
         role_sync_or(2, false);
@@ -1130,20 +1149,11 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
             const int ring = i & 3;
             const int t0 = c * kQ;
             const int valid = min(kQ, T - t0);
-            // z of this row half, loaded before the waits
-            uint4 zpre[4];
-            {
-                const bool zok = a.z != nullptr && t < valid;
-                const bf16_t* zr = zok ? static_cast<const bf16_t*>(a.z) + (row0 + t0 + t) * a.z_stride + xcol + 32 * h2
-                                       : nullptr;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) zpre[j] = zok ? *reinterpret_cast<const uint4*>(zr + 8 * j) : make_uint4(0, 0, 0, 0);
-            }
             // s_m: epilogue 1 of chunk c is done (its decay sums, read below, are
             // published by that release); s_d: dS and Ydiag are in TMEM
             bool got = p2_wait(&s_m[q], par, abort_flag);
             if (got) got = p2_wait(&s_d[q], par, abort_flag);
-            if (role_sync_or(2, !got)) { s_abort = 1; ok = false; break; }
+            if (role_sync_or(2, !got || z_fail)) { s_abort = 1; ok = false; break; }
             tc_fence_after();
             const uint32_t tq = tmem + q * 256;
             {
@@ -1162,11 +1172,11 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
                 if (e2 == 0) mbar_arrive1(&s_sready[(i + 1) & 1]);
             }
             got = p2_wait(&s_yoff[q], par, abort_flag);
+            if (got && gate) got = p2_wait(&s_z, i & 1, abort_flag);
             if (role_sync_or(2, !got)) { s_abort = 1; ok = false; break; }
             tc_fence_after();
             const float et = ex2(s_cum[ring][t]);
             const bool row_ok = t < valid;
-            const bool gate = a.z != nullptr;
             bf16_t* yrow = y + (row0 + t0 + t) * a.y_stride + xcol;
             const float2 et2 = make_float2(et, et);
 #pragma unroll
@@ -1178,7 +1188,7 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
                     const int jj = 2 * hh + jh;
                     float out[8];
                     float zv[8];
-                    unpack16<bf16_t>(zpre[jj], zv);
+                    if (gate) unpack16<bf16_t>(*reinterpret_cast<const uint4*>(zt + sw128(t, 4 * h2 + jj)), zv);
 #pragma unroll
                     for (int e = 0; e < 8; e += 2) {
                         float2 v = __ffma2_rn(et2, make_float2(yo[8 * jh + e], yo[8 * jh + e + 1]),
@@ -1190,9 +1200,20 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
                     if (row_ok) *reinterpret_cast<uint4*>(yrow + 8 * (h2 * 4 + jj)) = pack16<bf16_t>(out);
                 }
             }
-            // this thread has read TMEM stage q: chunk c+2 may reuse it once all have
+            // this thread has read TMEM stage q and the z tile: chunk c+2 may reuse
+            // the stage, chunk c+1's z may land, once all have
             tc_fence_before();
             mbar_arrive1(&s_tfree[q]);
+            if (gate && e2 == 0 && i + 1 < nloc) {
+                // (a failed wait here is decided by all at the next chunk's first barrier)
+                if (p2_wait(&s_tfree[q], par, abort_flag)) {
+                    load_z(c + 1);
+                    ++z_issued;
+                } else {
+                    s_abort = 1;
+                    z_fail = true;
+                }
+            }
         }
         if (ok && (!split || seg == nseg_s - 1)) {  // the sequence's final state, in place
 #pragma unroll
@@ -1211,6 +1232,7 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
             if (uses > 0) mbar_wait_bounded(&s_full[q], (uses - 1) & 1, kLimitNs);
         }
     }
+    if (tid == 320 && z_issued > 0) mbar_wait_bounded(&s_z, (z_issued - 1) & 1, kLimitNs);  // the last z tile
     __syncthreads();
     range_max = fmaxf(range_max, fmaxf(__low2float(hmax), __high2float(hmax)));
     if (s_abort) {
@@ -1331,7 +1353,18 @@ cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t stream) {
                                         static_cast<int>(kP2Smem));
         });
         if (e != cudaSuccess) return e;
-        chunk_scan_p2_kernel<bf16_t><<<grid, kP2Threads, kP2Smem, stream>>>(map, a);
+        // z (bf16) as (channel, packed token row), boxes of 64 x 128, 128-byte swizzle
+        CUtensorMap map_z{};
+        if (a.z) {
+            const cuuint64_t zd[2] = {static_cast<cuuint64_t>(a.H) * kP, static_cast<cuuint64_t>(a.total_tokens)};
+            const cuuint64_t zs[1] = {static_cast<cuuint64_t>(a.z_stride) * 2};
+            const cuuint32_t zb[2] = {64, static_cast<cuuint32_t>(kQ)};
+            if (enc(&map_z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.z), zd, zs, zb, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return cudaErrorInvalidValue;
+        }
+        chunk_scan_p2_kernel<bf16_t><<<grid, kP2Threads, kP2Smem, stream>>>(map, map_z, a);
         return cudaGetLastError();
     }
 #endif
