@@ -1133,6 +1133,7 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
             tma_load_2d(base + kP2OffZ, &tmap_z, xcol, static_cast<int>(row0 + static_cast<int64_t>(c) * kQ), &s_z);
         };
         bool z_fail = false;
+        bool e2_fail = false;
         if (gate && e2 == 0) {
             load_z(c_begin);
             z_issued = 1;
@@ -1153,7 +1154,8 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
             // published by that release); s_d: dS and Ydiag are in TMEM
             bool got = p2_wait(&s_m[q], par, abort_flag);
             if (got) got = p2_wait(&s_d[q], par, abort_flag);
-            if (role_sync_or(2, !got || z_fail)) { s_abort = 1; ok = false; break; }
+            // also decides, together, a failed wait of the previous chunk's y phase
+            if (role_sync_or(2, !got || z_fail || e2_fail)) { s_abort = 1; ok = false; break; }
             tc_fence_after();
             const uint32_t tq = tmem + q * 256;
             {
@@ -1173,7 +1175,12 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
             }
             got = p2_wait(&s_yoff[q], par, abort_flag);
             if (got && gate) got = p2_wait(&s_z, i & 1, abort_flag);
-            if (role_sync_or(2, !got)) { s_abort = 1; ok = false; break; }
+            if (!got) {  // decided at the next chunk's first barrier
+                s_abort = 1;
+                e2_fail = true;
+                ok = false;
+                continue;
+            }
             tc_fence_after();
             const float et = ex2(s_cum[ring][t]);
             const bool row_ok = t < valid;
