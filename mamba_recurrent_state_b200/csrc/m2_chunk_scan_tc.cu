@@ -203,6 +203,18 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
+// One 2-D TMA tile store (no multicast) from shared memory at `src` to the box
+// at element coordinates (x, y) of `map`, in the thread's bulk group.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int x, int y, uint32_t src) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];\n" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(src)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
+}
+// Waits until every bulk store of this thread has read its shared memory.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
+
 // Byte offset of 16-byte chunk j of row r in a 128-byte-swizzled tile.
 __device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t j) { return r * 128u + ((j ^ (r & 7u)) << 4); }
 
@@ -772,7 +784,7 @@ __device__ __forceinline__ void mbar_arrive1(uint64_t* bar) {
 template <typename ST>
 __global__ void __launch_bounds__(kP2Threads, 1)
 chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_z,
-                     const ScanArgs a) {
+                     const __grid_constant__ CUtensorMap tmap_y, const ScanArgs a) {
     extern __shared__ uint8_t s_raw[];
     __shared__ __align__(8) uint64_t s_full[2], s_cb[2], s_m[2], s_d[2], s_yoff[2], s_free[2], s_tfree[2];
     __shared__ __align__(8) uint64_t s_w[2];  // W of stage q is built (every epilogue-1 thread arrives)
@@ -1184,6 +1196,10 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
             tc_fence_after();
             const float et = ex2(s_cum[ring][t]);
             const bool row_ok = t < valid;
+            // a whole chunk with a gate: y goes in place of z into the tile and
+            // out as one TMA store (a partial chunk's rows past the sequence are
+            // another sequence's, so those chunks store row by row)
+            const bool ytile = gate && valid == kQ;
             bf16_t* yrow = y + (row0 + t0 + t) * a.y_stride + xcol;
             const float2 et2 = make_float2(et, et);
 #pragma unroll
@@ -1204,18 +1220,29 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
                         out[e] = v.x;
                         out[e + 1] = v.y;
                     }
-                    if (row_ok) *reinterpret_cast<uint4*>(yrow + 8 * (h2 * 4 + jj)) = pack16<bf16_t>(out);
+                    if (ytile)
+                        *reinterpret_cast<uint4*>(zt + sw128(t, 4 * h2 + jj)) = pack16<bf16_t>(out);
+                    else if (row_ok)
+                        *reinterpret_cast<uint4*>(yrow + 8 * (h2 * 4 + jj)) = pack16<bf16_t>(out);
                 }
             }
-            // this thread has read TMEM stage q and the z tile: chunk c+2 may reuse
-            // the stage, chunk c+1's z may land, once all have
+            if (ytile) fence_proxy_async();  // the y tile, for the TMA store
+            // this thread has read TMEM stage q and the z tile (and written its y
+            // rows): chunk c+2 may reuse the stage, the tile may go out and chunk
+            // c+1's z land, once all have
             tc_fence_before();
             mbar_arrive1(&s_tfree[q]);
-            if (gate && e2 == 0 && i + 1 < nloc) {
+            if (gate && e2 == 0 && (ytile || i + 1 < nloc)) {
                 // (a failed wait here is decided by all at the next chunk's first barrier)
                 if (p2_wait(&s_tfree[q], par, abort_flag)) {
-                    load_z(c + 1);
-                    ++z_issued;
+                    if (ytile) {
+                        tma_store_2d(&tmap_y, xcol, static_cast<int>(row0 + t0), base + kP2OffZ);
+                        bulk_wait_read();  // the tile is read out before z of the next chunk lands in it
+                    }
+                    if (i + 1 < nloc) {
+                        load_z(c + 1);
+                        ++z_issued;
+                    }
                 } else {
                     s_abort = 1;
                     z_fail = true;
@@ -1239,7 +1266,10 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
             if (uses > 0) mbar_wait_bounded(&s_full[q], (uses - 1) & 1, kLimitNs);
         }
     }
-    if (tid == 320 && z_issued > 0) mbar_wait_bounded(&s_z, (z_issued - 1) & 1, kLimitNs);  // the last z tile
+    if (tid == 320) {  // the last z tile has landed and the last y tile has been read out
+        if (z_issued > 0) mbar_wait_bounded(&s_z, (z_issued - 1) & 1, kLimitNs);
+        bulk_wait_read();
+    }
     __syncthreads();
     range_max = fmaxf(range_max, fmaxf(__low2float(hmax), __high2float(hmax)));
     if (s_abort) {
@@ -1371,7 +1401,18 @@ cudaError_t launch_chunk_scan_tc(const ScanArgs& a, cudaStream_t stream) {
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
                 return cudaErrorInvalidValue;
         }
-        chunk_scan_p2_kernel<bf16_t><<<grid, kP2Threads, kP2Smem, stream>>>(map, map_z, a);
+        // y (bf16), the same boxes, for the TMA stores of whole gated chunks
+        CUtensorMap map_y{};
+        if (a.z) {
+            const cuuint64_t yd[2] = {static_cast<cuuint64_t>(a.H) * kP, static_cast<cuuint64_t>(a.total_tokens)};
+            const cuuint64_t ys[1] = {static_cast<cuuint64_t>(a.y_stride) * 2};
+            const cuuint32_t yb[2] = {64, static_cast<cuuint32_t>(kQ)};
+            if (enc(&map_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.y, yd, ys, yb, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return cudaErrorInvalidValue;
+        }
+        chunk_scan_p2_kernel<bf16_t><<<grid, kP2Threads, kP2Smem, stream>>>(map, map_z, map_y, a);
         return cudaGetLastError();
     }
 #endif
