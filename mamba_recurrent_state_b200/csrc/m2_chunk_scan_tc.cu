@@ -705,30 +705,40 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
 // chain while epilogue 1 of the next chunk runs beside them:
 //   warp 0        TMA producer: stage (c & 1) <- x, B, C tiles of chunk c
 //   warp 1        MMA issuer: C S^T, M X, W^T X, then CB of the next chunk
-//   warps 2..9    epilogue 1 (256 threads): dt and decay sums, M (into TMEM,
-//                 as the A operand of M X, so the C tile stays intact for
-//                 C S^T) and W = w o B (in place in the B tile)
+//   warps 2..9    epilogue 1 (256 threads): dt and decay sums, M (into TMEM
+//                 in place of CB, as the A operand of M X, so the C tile
+//                 stays intact for C S^T) and W = w o B (in place in the B
+//                 tile)
 //   warps 10..17  epilogue 2 (256 threads): the fp32 state carry of chunk c
 //                 and its fp16 copy for C S^T of chunk c+1 first, then y of
 //                 chunk c
+//   warp 18       mover: the y tile of chunk c out and the z tile of chunk
+//                 c+1 in (TMA), off the epilogue-2 chain
 // Per chunk the issuer runs C S^T as soon as the state entering the chunk is
 // ready (normally while epilogue 1 still works on M), then M X as soon as
 // every epilogue-1 thread has written its rows of M (the last of them are
 // still scaling W), then W^T X once W is built, after which the stage's tiles
-// are free for the load of chunk c+2, then CB of chunk c+1 (once every
-// epilogue-2 thread has read the TMEM stage of chunk c-1). The state copy is
-// double-buffered, so the carry (the only step that must follow the previous
-// chunk's) is not held up by C S^T of the previous chunk, and y leaves the
-// chain.
-// One CTA per SM (two shared-memory stages of 80 KB and two 16 KB state
-// copies, 512 TMEM columns: per stage CB at 0..127, later dS at 0..63 and
-// Ydiag at 64..127, M at 128..191 (fp16 pairs), Yoff at 192..255). Every
-// hand-off is an mbarrier; every wait is bounded and a timeout ends all roles
-// with M2_ERR_TIMEOUT.
+// are free for the load of chunk c+2, then CB of chunk c+1 (once M X of chunk
+// c has read M). The state copy is double-buffered, so the carry (the only
+// step that must follow the previous chunk's) is not held up by C S^T of the
+// previous chunk, and y leaves the chain.
+// One CTA per SM: two shared-memory stages of 80 KB, two 16 KB state copies
+// (fp16, n-major like the x tile) and a 16 KB z / y tile. TMEM holds two
+// rings with their own lifetimes:
+//   ring A (columns 0..127, one stage): CB, then M in place of it. Each
+//     epilogue-1 thread writes the fp16 pairs of M's K-step k (its columns
+//     u = 16k..16k+15) into the first 8 of the 16 columns it read CB from,
+//     so no thread overwrites a column another thread has still to read.
+//     Free once M X has completed, which CB of the next chunk waits for.
+//   ring B (columns 128..511, two stages of 192): Ydiag at 0..63, dS^T at
+//     64..127, Yoff at 128..191 of a stage; free once every epilogue-2
+//     thread has read it.
+// Every hand-off is an mbarrier; every wait is bounded and a timeout ends all
+// roles with M2_ERR_TIMEOUT.
 #ifndef M2_SCAN_PIPELINED
 #define M2_SCAN_PIPELINED 1
 #endif
-constexpr int kP2Threads = 576;
+constexpr int kP2Threads = 608;
 constexpr uint32_t kP2Stage = 81920;                       // C 32 KB | B 32 KB | X 16 KB
 constexpr uint32_t kP2OffS = 2 * kP2Stage;                 // two fp16 state copies, 16 KB each
 constexpr uint32_t kP2OffZ = kP2OffS + 2 * 16384;          // the z tile of a chunk (bf16, 16 KB)
@@ -790,6 +800,7 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
     __shared__ __align__(8) uint64_t s_w[2];  // W of stage q is built (every epilogue-1 thread arrives)
     __shared__ __align__(8) uint64_t s_sready[2];  // state copy (i & 1) holds the state entering chunk i
     __shared__ __align__(8) uint64_t s_drain;
+    __shared__ __align__(8) uint64_t s_mx;  // M X of the last chunk has completed (TMEM ring A is free)
     __shared__ __align__(8) uint64_t s_z;  // the z tile of the next chunk has landed
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
@@ -861,6 +872,7 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
         mbar_init(&s_sready[0], 1);
         mbar_init(&s_sready[1], 1);
         mbar_init(&s_drain, 1);
+        mbar_init(&s_mx, 1);
         mbar_init(&s_z, 1);
         fence_mbar_init();
         asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
@@ -880,7 +892,7 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
     float range_max = 0.f;
     __half2 hmax = __float2half2_rn(0.f);
     int loads_issued = 0;  // producer bookkeeping (lane 0 of warp 0)
-    int z_issued = 0;      // z tiles issued (epilogue-2 thread 0)
+    int z_issued = 0;      // z tiles issued (the mover)
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer
@@ -906,7 +918,7 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
         // ------------------------------------------------------- MMA issuer
         if (lane == 0) {
             const uint32_t id_cb = idesc_f16(128, 128, false, false);
-            const uint32_t id_yoff = idesc_f16(128, 64, false, false);
+            const uint32_t id_yoff = idesc_f16(128, 64, false, true);
             const uint32_t id_ydiag = idesc_f16(128, 64, false, true);
             const uint32_t id_ds = idesc_f16(128, 64, true, true);
             // CB = C . B^T of chunk j into stage j & 1, once its tiles have landed
@@ -914,13 +926,13 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
             auto issue_cb = [&](int j) -> bool {
                 const int q = j & 1;
                 bool ok = p2_wait(&s_full[q], (j >> 1) & 1, abort_flag);
-                if (ok && j >= 2) ok = p2_wait(&s_tfree[q], ((j >> 1) - 1) & 1, abort_flag);
+                if (ok && j >= 1) ok = p2_wait(&s_mx, (j - 1) & 1, abort_flag);  // M of chunk j-1 read
                 if (!ok) return false;
                 tc_fence_after();
                 const uint32_t st = base + q * kP2Stage;
                 for (int k = 0; k < kN / 16; ++k) {
                     const uint32_t koff = (k >> 2) * 16384u + (k & 3) * 32u;
-                    mma_f16(tmem + q * 256, sw128_desc(st + koff, 16, 1024), sw128_desc(st + 32768 + koff, 16, 1024),
+                    mma_f16(tmem, sw128_desc(st + koff, 16, 1024), sw128_desc(st + 32768 + koff, 16, 1024),
                             id_cb, k > 0);
                 }
                 mma_commit(&s_cb[q]);
@@ -934,26 +946,28 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
                 const int q = i & 1;
                 const uint32_t par = (i >> 1) & 1;
                 const uint32_t st = base + q * kP2Stage;
-                const uint32_t tq = tmem + q * 256;
+                const uint32_t tq = tmem + 128 + q * 192;  // ring B: Ydiag, dS^T, Yoff
+                // ring-B stage q: epilogue 2 has read chunk i - 2's
+                if (i >= 2 && !p2_wait(&s_tfree[q], ((i >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
                 // the state entering chunk i, in copy q
                 if (!p2_wait(&s_sready[q], par, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 for (int k = 0; k < kN / 16; ++k) {  // Yoff = C . S^T
                     const uint32_t koff = (k >> 2) * 16384u + (k & 3) * 32u;
-                    const uint32_t soff = (k >> 2) * 8192u + (k & 3) * 32u;
-                    mma_f16(tq + 192, sw128_desc(st + koff, 16, 1024),
-                            sw128_desc(base + kP2OffS + q * 16384u + soff, 16, 1024), id_yoff, k > 0);
+                    mma_f16(tq + 128, sw128_desc(st + koff, 16, 1024),
+                            sw128_desc(base + kP2OffS + q * 16384u + k * 2048u, 16384, 1024), id_yoff, k > 0);
                 }
                 mma_commit(&s_yoff[q]);
                 if (!p2_wait(&s_m[q], par, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                for (int k = 0; k < kQ / 16; ++k)  // Ydiag = M . X (M from TMEM), while W is built
-                    mma_f16_ta(tq + 64, tq + 128 + k * 8, sw128_desc(st + 65536 + k * 2048u, 16384, 1024), id_ydiag,
+                for (int k = 0; k < kQ / 16; ++k)  // Ydiag = M . X (M from TMEM ring A), while W is built
+                    mma_f16_ta(tq + 0, tmem + k * 16, sw128_desc(st + 65536 + k * 2048u, 16384, 1024), id_ydiag,
                                k > 0);
+                mma_commit(&s_mx);
                 if (!p2_wait(&s_w[q], par, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 for (int k = 0; k < kQ / 16; ++k)  // dS^T = W^T . X
-                    mma_f16(tq + 0, sw128_desc(st + 32768 + k * 2048u, 16384, 1024),
+                    mma_f16(tq + 64, sw128_desc(st + 32768 + k * 2048u, 16384, 1024),
                             sw128_desc(st + 65536 + k * 2048u, 16384, 1024), id_ds, k > 0);
                 mma_commit(&s_d[q]);
                 mma_commit(&s_free[q]);
@@ -1018,7 +1032,7 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
                 continue;
             }
             tc_fence_after();
-            const uint32_t tq = tmem + q * 256;
+            const uint32_t ta = tmem;  // ring A: CB, then M in place
             uint8_t* stB = sm + q * kP2Stage + 32768;
             const float cum_t = cum_c[t];
             const float cum_end = cum_c[kQ - 1];
@@ -1034,7 +1048,7 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
 #pragma unroll
                     for (int e = 0; e < 16; ++e) m[e] = 0.f;
                 } else {
-                    tmem_ld16(tq + lane_base + u0, m);
+                    tmem_ld16(ta + lane_base + u0, m);
                     if (qb < wq) {
                         const float4* g4 = reinterpret_cast<const float4*>(gam + u0);
 #pragma unroll
@@ -1052,18 +1066,25 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
                     } else {
                         const float4* cu4 = reinterpret_cast<const float4*>(cum_c + u0);
                         const float4* du4 = reinterpret_cast<const float4*>(dt_c + u0);
+                        const float2 ct2 = make_float2(cum_t, cum_t);
 #pragma unroll
                         for (int i4 = 0; i4 < 4; ++i4) {
                             const float4 cu = cu4[i4], du = du4[i4];
-                            const float cuv[4] = {cu.x, cu.y, cu.z, cu.w};
-                            const float duv[4] = {du.x, du.y, du.z, du.w};
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int u = u0 + 4 * i4 + e;
-                                float v = m[4 * i4 + e] * ex2(cum_t - cuv[e]) * duv[e];
-                                if (u > t) v = 0.f;
-                                if (u == t) v += Dh;
-                                m[4 * i4 + e] = v;
+                            for (int hp = 0; hp < 2; ++hp) {  // a pair of columns, packed
+                                const float2 x = __fadd2_rn(ct2, hp ? make_float2(-cu.z, -cu.w) : make_float2(-cu.x, -cu.y));
+                                float2 v = __fmul2_rn(make_float2(m[4 * i4 + 2 * hp], m[4 * i4 + 2 * hp + 1]),
+                                                      make_float2(ex2(x.x), ex2(x.y)));
+                                v = __fmul2_rn(v, hp ? make_float2(du.z, du.w) : make_float2(du.x, du.y));
+                                const float vv[2] = {v.x, v.y};
+#pragma unroll
+                                for (int e = 0; e < 2; ++e) {
+                                    const int u = u0 + 4 * i4 + 2 * hp + e;
+                                    float w = vv[e];
+                                    if (u > t) w = 0.f;
+                                    if (u == t) w += Dh;
+                                    m[4 * i4 + 2 * hp + e] = w;
+                                }
                             }
                         }
                     }
@@ -1075,7 +1096,9 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
                     hmax = __hmax2(hmax, __habs2(hv));
                     hw[j] = *reinterpret_cast<const uint32_t*>(&hv);
                 }
-                tmem_st8(tq + lane_base + 128 + u0 / 2, hw);  // M row t, columns u0 .. u0+15 as fp16 pairs
+                // M row t, columns u0 .. u0+15 as fp16 pairs, into the first 8 of
+                // the 16 TMEM columns this thread read them from
+                tmem_st8(ta + lane_base + u0, hw);
             }
             // this thread's rows of M are in TMEM: M . X may start while W is built
             tmem_wait_st();
@@ -1085,6 +1108,9 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
             const float wu = (t < valid) ? ex2(cum_end - cum_t) * dt_c[t] : 0.f;
             const __half2 w2 = __float2half2_rn(wu);
             hmax = __hmax2(hmax, __habs2(w2));
+            // w <= 1 cannot take a finite fp16 B past the range: the products are
+            // checked only where it is larger
+            const bool wcheck = wu > 1.f;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 uint4* pw = reinterpret_cast<uint4*>(stB + h2 * 16384 + sw128(t, j));
@@ -1093,8 +1119,11 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const __half2 r2 = __hmul2(*reinterpret_cast<const __half2*>(&vw[e]), w2);
-                    hmax = __hmax2(hmax, __habs2(r2));
                     vw[e] = *reinterpret_cast<const uint32_t*>(&r2);
+                }
+                if (wcheck) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) hmax = __hmax2(hmax, __habs2(*reinterpret_cast<const __half2*>(&vw[e])));
                 }
                 *pw = v;
             }
@@ -1102,6 +1131,35 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
             // orders this chunk's reads of s_gam and the decay sums before their reuse
             fence_proxy_async();
             mbar_arrive1(&s_w[q]);
+        }
+    } else if (warp == 18) {
+        // --------------------------------------------------- y / z mover
+        // Chunk c's y tile leaves (one TMA store, in place of its z tile) and
+        // chunk c+1's z tile is loaded into the same buffer, once every
+        // epilogue-2 thread is done with chunk c (its TMEM-free arrival), so
+        // no epilogue-2 thread waits for the copies.
+        if (lane == 0 && a.z != nullptr) {
+            auto load_z = [&](int c) {
+                mbar_arrive_expect_tx(&s_z, 16384u);
+                tma_load_2d(base + kP2OffZ, &tmap_z, xcol, static_cast<int>(row0 + static_cast<int64_t>(c) * kQ),
+                            &s_z);
+                ++z_issued;
+            };
+            if (nloc > 0) load_z(c_begin);
+            for (int i = 0; i < nloc; ++i) {
+                const int c = c_begin + i;
+                const bool ytile = T - c * kQ >= kQ;  // a whole chunk: y leaves as one tile
+                if (!ytile && i + 1 >= nloc) break;
+                if (!p2_wait(&s_tfree[i & 1], (i >> 1) & 1, abort_flag)) {
+                    s_abort = 1;
+                    break;
+                }
+                if (ytile) {
+                    tma_store_2d(&tmap_y, xcol, static_cast<int>(row0 + static_cast<int64_t>(c) * kQ), base + kP2OffZ);
+                    bulk_wait_read();  // the tile is read out before z of the next chunk lands in it
+                }
+                if (i + 1 < nloc) load_z(c + 1);
+            }
         }
     } else {
         // ------------------------------------------------------- epilogue 2
@@ -1124,32 +1182,27 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
 #pragma unroll
             for (int k = 0; k < kPH; ++k) S[k] = init ? to_f32(state[(p0 + k) * kN + n]) : 0.f;
         }
+        // fp16 copy of the state as the B operand of C S^T, n-major like the x
+        // tile (row n: the 64 p values, 128-byte swizzle): four 16-byte stores
         auto write_state_copy = [&](int buf) {
-            uint8_t* sS = sm + kP2OffS + buf * 16384 + (n >> 6) * 8192;
-            const uint32_t j = (n & 63) >> 3;
+            uint8_t* sS = sm + kP2OffS + buf * 16384;
 #pragma unroll
-            for (int k = 0; k < kPH; k += 2) {
-                const __half2 hv = __floats2half2_rn(S[k], S[k + 1]);
-                hmax = __hmax2(hmax, __habs2(hv));
-                *reinterpret_cast<__half*>(sS + sw128(p0 + k, j) + (n & 7) * 2) = __low2half(hv);
-                *reinterpret_cast<__half*>(sS + sw128(p0 + k + 1, j) + (n & 7) * 2) = __high2half(hv);
+            for (int jj = 0; jj < 4; ++jj) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const __half2 hv = __floats2half2_rn(S[8 * jj + 2 * e], S[8 * jj + 2 * e + 1]);
+                    hmax = __hmax2(hmax, __habs2(hv));
+                    w[e] = *reinterpret_cast<const uint32_t*>(&hv);
+                }
+                *reinterpret_cast<uint4*>(sS + sw128(n, 4 * h2 + jj)) = make_uint4(w[0], w[1], w[2], w[3]);
             }
         };
-        // z tile of chunk c (128 tokens x 64 channels, 128-byte swizzle) by TMA
-        // into one shared buffer, issued by e2 == 0 once every thread has read
-        // the previous one (the TMEM-free barrier of that chunk)
+        // the z tile of chunk c (128 tokens x 64 channels, 128-byte swizzle)
+        // arrives by TMA in one shared buffer; the mover warp issues it
         const bool gate = a.z != nullptr;
         uint8_t* zt = sm + kP2OffZ;
-        auto load_z = [&](int c) {
-            mbar_arrive_expect_tx(&s_z, 16384u);
-            tma_load_2d(base + kP2OffZ, &tmap_z, xcol, static_cast<int>(row0 + static_cast<int64_t>(c) * kQ), &s_z);
-        };
-        bool z_fail = false;
         bool e2_fail = false;
-        if (gate && e2 == 0) {
-            load_z(c_begin);
-            z_issued = 1;
-        }
         write_state_copy(0);
         fence_proxy_async();
         role_sync_or(2, false);
@@ -1167,15 +1220,20 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
             bool got = p2_wait(&s_m[q], par, abort_flag);
             if (got) got = p2_wait(&s_d[q], par, abort_flag);
             // also decides, together, a failed wait of the previous chunk's y phase
-            if (role_sync_or(2, !got || z_fail || e2_fail)) { s_abort = 1; ok = false; break; }
+            if (role_sync_or(2, !got || e2_fail)) { s_abort = 1; ok = false; break; }
             tc_fence_after();
-            const uint32_t tq = tmem + q * 256;
+            const uint32_t tq = tmem + 128 + q * 192;
             {
                 const float eend = ex2(s_cum[ring][kQ - 1]);
                 float ds[32];
-                tmem_ld32(tq + lane_base + p0, ds);
+                tmem_ld32(tq + lane_base + 64 + p0, ds);
 #pragma unroll
-                for (int k = 0; k < kPH; ++k) S[k] = fmaf(eend, S[k], ds[k]);
+                for (int k = 0; k < kPH; k += 2) {
+                    const float2 r = __ffma2_rn(make_float2(eend, eend), make_float2(S[k], S[k + 1]),
+                                                make_float2(ds[k], ds[k + 1]));
+                    S[k] = r.x;
+                    S[k + 1] = r.y;
+                }
             }
             // the state leaving chunk c, for C S^T of chunk c+1: copy (i+1) & 1,
             // last read by C S^T of chunk c-1, which has completed (s_yoff, below)
@@ -1205,7 +1263,7 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 float yd[16], yo[16];
-                tmem_ld16x2(tq + lane_base + 64 + h2 * 32 + 16 * hh, tq + lane_base + 192 + h2 * 32 + 16 * hh, yd, yo);
+                tmem_ld16x2(tq + lane_base + h2 * 32 + 16 * hh, tq + lane_base + 128 + h2 * 32 + 16 * hh, yd, yo);
 #pragma unroll
                 for (int jh = 0; jh < 2; ++jh) {
                     const int jj = 2 * hh + jh;
@@ -1232,22 +1290,6 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
             // c+1's z land, once all have
             tc_fence_before();
             mbar_arrive1(&s_tfree[q]);
-            if (gate && e2 == 0 && (ytile || i + 1 < nloc)) {
-                // (a failed wait here is decided by all at the next chunk's first barrier)
-                if (p2_wait(&s_tfree[q], par, abort_flag)) {
-                    if (ytile) {
-                        tma_store_2d(&tmap_y, xcol, static_cast<int>(row0 + t0), base + kP2OffZ);
-                        bulk_wait_read();  // the tile is read out before z of the next chunk lands in it
-                    }
-                    if (i + 1 < nloc) {
-                        load_z(c + 1);
-                        ++z_issued;
-                    }
-                } else {
-                    s_abort = 1;
-                    z_fail = true;
-                }
-            }
         }
         if (ok && (!split || seg == nseg_s - 1)) {  // the sequence's final state, in place
 #pragma unroll
@@ -1266,7 +1308,7 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
             if (uses > 0) mbar_wait_bounded(&s_full[q], (uses - 1) & 1, kLimitNs);
         }
     }
-    if (tid == 320) {  // the last z tile has landed and the last y tile has been read out
+    if (tid == 576) {  // the mover: the last z tile has landed and the last y tile has been read out
         if (z_issued > 0) mbar_wait_bounded(&s_z, (z_issued - 1) & 1, kLimitNs);
         bulk_wait_read();
     }
