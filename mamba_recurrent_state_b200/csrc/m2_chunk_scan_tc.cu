@@ -700,15 +700,16 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
 // ---------------------------------------------------------------------------
 // Pipelined variant: warp-specialised, two chunks in flight (fp16 post-conv
 // input). The per-chunk chain of the kernel above is latency-bound (load, CB,
-// epilogue 1, M X and W^T X, epilogue 2, one after the other). Only epilogue 2
-// and C S^T depend on the carried state, so here they form the sequential
-// chain while epilogue 1 of the next chunk runs beside them:
+// epilogue 1, M X and the state MMA, epilogue 2, one after the other). Only
+// epilogue 2 and C S^T depend on the carried state, so here they form the
+// sequential chain while epilogue 1 of the next chunk runs beside them:
 //   warp 0        TMA producer: stage (c & 1) <- x, B, C tiles of chunk c
-//   warp 1        MMA issuer: C S^T, M X, W^T X, then CB of the next chunk
+//   warp 1        MMA issuer: C S^T, M X, dS^T = B^T (w o X), then CB of the
+//                 next chunk
 //   warps 2..9    epilogue 1 (256 threads): dt and decay sums, M (into TMEM
 //                 in place of CB, as the A operand of M X, so the C tile
-//                 stays intact for C S^T) and W = w o B (in place in the B
-//                 tile)
+//                 stays intact for C S^T) and w o x (the x tile scaled by
+//                 the decay-to-chunk-end weights w_t = exp(cum_end - cum_t) dt_t)
 //   warps 10..17  epilogue 2 (256 threads): the fp32 state carry of chunk c
 //                 and its fp16 copy for C S^T of chunk c+1 first, then y of
 //                 chunk c
@@ -717,14 +718,14 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
 // Per chunk the issuer runs C S^T as soon as the state entering the chunk is
 // ready (normally while epilogue 1 still works on M), then M X as soon as
 // every epilogue-1 thread has written its rows of M (the last of them are
-// still scaling W), then W^T X once W is built, after which the stage's tiles
-// are free for the load of chunk c+2, then CB of chunk c+1 (once M X of chunk
-// c has read M). The state copy is double-buffered, so the carry (the only
-// step that must follow the previous chunk's) is not held up by C S^T of the
-// previous chunk, and y leaves the chain.
-// One CTA per SM: two shared-memory stages of 80 KB, two 16 KB state copies
-// (fp16, n-major like the x tile) and a 16 KB z / y tile. TMEM holds two
-// rings with their own lifetimes:
+// still scaling x), then B^T (w o X) once w o x is built, after which the
+// stage's tiles are free for the load of chunk c+2, then CB of chunk c+1
+// (once M X of chunk c has read M). MMAs complete in issue order, so once dS
+// of chunk c is in, C S^T of chunk c has read the state copy and epilogue 2
+// overwrites it with the state leaving chunk c; y leaves the chain.
+// One CTA per SM: two shared-memory stages of 80 KB, a 16 KB fp16 state copy
+// (n-major like the x tile), the 16 KB w o x tile (fp16) and a 16 KB z / y
+// tile. TMEM holds two rings with their own lifetimes:
 //   ring A (columns 0..127, one stage): CB, then M in place of it. Each
 //     epilogue-1 thread writes the fp16 pairs of M's K-step k (its columns
 //     u = 16k..16k+15) into the first 8 of the 16 columns it read CB from,
@@ -740,8 +741,9 @@ chunk_scan_tc_kernel(const __grid_constant__ CUtensorMap tmap_x, const ScanArgs 
 #endif
 constexpr int kP2Threads = 608;
 constexpr uint32_t kP2Stage = 81920;                       // C 32 KB | B 32 KB | X 16 KB
-constexpr uint32_t kP2OffS = 2 * kP2Stage;                 // two fp16 state copies, 16 KB each
-constexpr uint32_t kP2OffZ = kP2OffS + 2 * 16384;          // the z tile of a chunk (bf16, 16 KB)
+constexpr uint32_t kP2OffS = 2 * kP2Stage;                 // the fp16 state copy (16 KB)
+constexpr uint32_t kP2OffXw = kP2OffS + 16384;             // w o x of a chunk (fp16, 16 KB)
+constexpr uint32_t kP2OffZ = kP2OffXw + 16384;             // the z tile of a chunk (bf16, 16 KB)
 constexpr uint32_t kP2Smem = kP2OffZ + 16384 + 1024;       // + alignment slack
 constexpr uint32_t kP2TmemCols = 512;
 
@@ -955,7 +957,7 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
                 for (int k = 0; k < kN / 16; ++k) {  // Yoff = C . S^T
                     const uint32_t koff = (k >> 2) * 16384u + (k & 3) * 32u;
                     mma_f16(tq + 128, sw128_desc(st + koff, 16, 1024),
-                            sw128_desc(base + kP2OffS + q * 16384u + k * 2048u, 16384, 1024), id_yoff, k > 0);
+                            sw128_desc(base + kP2OffS + k * 2048u, 16384, 1024), id_yoff, k > 0);
                 }
                 mma_commit(&s_yoff[q]);
                 if (!p2_wait(&s_m[q], par, abort_flag)) { ok = false; break; }
@@ -966,9 +968,9 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
                 mma_commit(&s_mx);
                 if (!p2_wait(&s_w[q], par, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                for (int k = 0; k < kQ / 16; ++k)  // dS^T = W^T . X
+                for (int k = 0; k < kQ / 16; ++k)  // dS^T = B^T . (w o X)
                     mma_f16(tq + 64, sw128_desc(st + 32768 + k * 2048u, 16384, 1024),
-                            sw128_desc(st + 65536 + k * 2048u, 16384, 1024), id_ds, k > 0);
+                            sw128_desc(base + kP2OffXw + k * 2048u, 16384, 1024), id_ds, k > 0);
                 mma_commit(&s_d[q]);
                 mma_commit(&s_free[q]);
                 if (i + 1 < nloc && !issue_cb(i + 1)) { ok = false; break; }
@@ -1033,7 +1035,7 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
             }
             tc_fence_after();
             const uint32_t ta = tmem;  // ring A: CB, then M in place
-            uint8_t* stB = sm + q * kP2Stage + 32768;
+            const uint8_t* stX = sm + q * kP2Stage + 65536;
             const float cum_t = cum_c[t];
             const float cum_end = cum_c[kQ - 1];
             const int wq = quarter;
@@ -1104,17 +1106,26 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive1(&s_m[q]);
-            // W row t = w_t * B row t (fp16 pairs, in place)
+            // (w o x) row t = w_t * x row t (fp16 pairs; this thread's 32 of the 64
+            // channels) into the one w o x buffer, once dS of the previous chunk
+            // has read it. B stays as loaded: dS^T = B^T (w o X) is the same sum
+            // as W^T X with W = w o B, and x has half the elements of B.
+            if (i >= 1 && !p2_wait(&s_d[(i - 1) & 1], ((i - 1) >> 1) & 1, abort_flag)) {
+                s_abort = 1;
+                cb_fail = true;  // decided at the next chunk's first barrier
+                continue;
+            }
             const float wu = (t < valid) ? ex2(cum_end - cum_t) * dt_c[t] : 0.f;
             const __half2 w2 = __float2half2_rn(wu);
             hmax = __hmax2(hmax, __habs2(w2));
-            // w <= 1 cannot take a finite fp16 B past the range: the products are
+            // w <= 1 cannot take a finite fp16 x past the range: the products are
             // checked only where it is larger
             const bool wcheck = wu > 1.f;
+            uint8_t* xw = sm + kP2OffXw;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                uint4* pw = reinterpret_cast<uint4*>(stB + h2 * 16384 + sw128(t, j));
-                uint4 v = *pw;
+            for (int jj = 0; jj < 4; ++jj) {
+                const int j = 4 * h2 + jj;
+                uint4 v = *reinterpret_cast<const uint4*>(stX + sw128(t, j));
                 uint32_t* vw = reinterpret_cast<uint32_t*>(&v);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -1125,9 +1136,9 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
 #pragma unroll
                     for (int e = 0; e < 4; ++e) hmax = __hmax2(hmax, __habs2(*reinterpret_cast<const __half2*>(&vw[e])));
                 }
-                *pw = v;
+                *reinterpret_cast<uint4*>(xw + sw128(t, j)) = v;
             }
-            // W visible to the tensor cores; the next chunk's first role barrier
+            // w o x visible to the tensor cores; the next chunk's first role barrier
             // orders this chunk's reads of s_gam and the decay sums before their reuse
             fence_proxy_async();
             mbar_arrive1(&s_w[q]);
@@ -1184,8 +1195,8 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
         }
         // fp16 copy of the state as the B operand of C S^T, n-major like the x
         // tile (row n: the 64 p values, 128-byte swizzle): four 16-byte stores
-        auto write_state_copy = [&](int buf) {
-            uint8_t* sS = sm + kP2OffS + buf * 16384;
+        auto write_state_copy = [&]() {
+            uint8_t* sS = sm + kP2OffS;
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj) {
                 uint32_t w[4];
@@ -1203,7 +1214,7 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
         const bool gate = a.z != nullptr;
         uint8_t* zt = sm + kP2OffZ;
         bool e2_fail = false;
-        write_state_copy(0);
+        write_state_copy();
         fence_proxy_async();
         role_sync_or(2, false);
         if (e2 == 0) mbar_arrive1(&s_sready[0]);
@@ -1235,10 +1246,11 @@ chunk_scan_p2_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_co
                     S[k + 1] = r.y;
                 }
             }
-            // the state leaving chunk c, for C S^T of chunk c+1: copy (i+1) & 1,
-            // last read by C S^T of chunk c-1, which has completed (s_yoff, below)
+            // the state leaving chunk c, for C S^T of chunk c+1, in the one copy:
+            // its last reader, C S^T of chunk c, was issued before dS of chunk c
+            // and has completed with it (s_d, above)
             if (i + 1 < nloc) {
-                write_state_copy((i + 1) & 1);
+                write_state_copy();
                 fence_proxy_async();
                 role_sync_or(2, false);
                 if (e2 == 0) mbar_arrive1(&s_sready[(i + 1) & 1]);
