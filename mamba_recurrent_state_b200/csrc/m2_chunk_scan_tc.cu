@@ -15,6 +15,8 @@
 //   MMA3  Yoff   [t,p] = C . S^T        A = C (K-major), B = S (K-major, fp16 copy)
 //   MMA2  Ydiag  [t,p] = M . X          A = M = CB o L o dt + D I (K-major), B = X (MN-major)
 //   MMA4  dS^T   [n,p] = W^T . X        A = W = w o B (MN-major), B = X (MN-major)
+//         (the pipelined kernel below forms the same sum as B^T . (w o X): x
+//         scaled per token into its own tile, B as loaded)
 // The state itself is carried exactly in fp32 registers (thread n holds column
 // n of S) and rounded once when the sequence ends. Only the chunk-to-chunk carry
 // is sequential. D x rides on the diagonal of M, so once MMA2 and MMA4 are
