@@ -359,7 +359,12 @@ __global__ void __launch_bounds__(kTileThreads, K <= 4 ? kTileMinBlocks : 3)
                     for (int k = 0; k < K - 1; ++k)
                         acc = __ffma2_rn(make_float2(w[e][k], w[e + 1][k]), make_float2(hist[k][e], hist[k][e + 1]), acc);
                     acc = __ffma2_rn(make_float2(w[e][K - 1], w[e + 1][K - 1]), make_float2(cur[e], cur[e + 1]), acc);
-                    if (a.activation) acc = silu2_f32(acc);
+                    if (a.activation) {
+                        if constexpr (std::is_same<OT, float>::value)
+                            acc = silu2_f32(acc);
+                        else
+                            acc = silu2_tanh_f32(acc);
+                    }
                     o[e] = acc.x;
                     o[e + 1] = acc.y;
                 }

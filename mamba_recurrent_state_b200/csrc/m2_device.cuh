@@ -251,11 +251,23 @@ constexpr float kNegLog2E = -1.4426950408889634f;  // -log2(e): exp(-v) = 2^(v *
 // reciprocal to 0, for v -> +inf it underflows to 0. silu2_f32 is the same
 // arithmetic on a pair, with packed f32x2 multiplies and adds (bit for bit
 // silu_f32 of each half; the conv kernels, bound by instruction issue, take
-// SiLUs in pairs). Every kernel uses these, so fused and unfused paths agree
-// bit for bit.
+// SiLUs in pairs). Every decode-side kernel uses these, so fused and unfused
+// decode paths agree bit for bit; the prefill tile conv takes the tanh form
+// below for its 16-bit outputs and these for fp32 outputs.
 __device__ __forceinline__ float silu_f32(float v) {
     const float d = 1.f + ex2_approx(v * kNegLog2E);
     return v * rcp_approx(d);
+}
+// silu on a pair in the tanh form: silu(v) = h + h tanh(h), h = v / 2, with
+// the hardware tanh (PTX tanh.approx, one special-function operation per
+// value instead of two; relative error about 2^-11). For outputs rounded to a
+// 16-bit type, whose own rounding is of that size.
+__device__ __forceinline__ float2 silu2_tanh_f32(float2 v) {
+    const float2 h = __fmul2_rn(v, make_float2(0.5f, 0.5f));
+    float ta, tb;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(ta) : "f"(h.x));
+    asm("tanh.approx.f32 %0, %1;" : "=f"(tb) : "f"(h.y));
+    return __ffma2_rn(h, make_float2(ta, tb), h);
 }
 __device__ __forceinline__ float2 silu2_f32(float2 v) {
     const float2 t = __fmul2_rn(v, make_float2(kNegLog2E, kNegLog2E));
