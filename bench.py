@@ -84,50 +84,6 @@ def _peak(key: str, fallback: float) -> tuple[float, str]:
         return fallback, "fallback"
 
 
-class _Cudart:
-    """The few CUDA runtime calls the end-to-end loop issues, bound by ctypes to
-    the libcudart that torch loaded (streams and events are shared with torch)."""
-
-    def __init__(self):
-        import ctypes
-        try:
-            lib = ctypes.CDLL("libcudart.so.12", mode=ctypes.RTLD_GLOBAL)
-        except OSError:
-            import nvidia.cuda_runtime as ncr
-            lib = ctypes.CDLL(os.path.join(list(ncr.__path__)[0], "lib", "libcudart.so.12"))
-        vp, sz, ci, cu = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_uint
-        self._ct = ctypes
-        self._lib = lib
-        for name, args in (("cudaMemcpyAsync", [vp, vp, sz, ci, vp]),
-                           ("cudaEventRecord", [vp, vp]),
-                           ("cudaStreamWaitEvent", [vp, vp, cu]),
-                           ("cudaEventCreateWithFlags", [ctypes.POINTER(vp), cu]),
-                           ("cudaEventDestroy", [vp])):
-            fn = getattr(lib, name)
-            fn.argtypes, fn.restype = args, ci
-            setattr(self, name, fn)
-
-    def event(self):
-        e = self._ct.c_void_p()
-        self.check(self.cudaEventCreateWithFlags(self._ct.byref(e), 2), "event")  # timing off
-        return e.value
-
-    @staticmethod
-    def check(status, what):
-        if status != 0:
-            raise RuntimeError(f"CUDA runtime error {status} in {what}")
-
-
-_CUDART = None
-
-
-def cudart() -> _Cudart:
-    global _CUDART
-    if _CUDART is None:
-        _CUDART = _Cudart()
-    return _CUDART
-
-
 def measured_peaks() -> tuple[float, str]:
     """HBM copy bandwidth, GB/s (measured on this machine, else the fallback)."""
     return _peak("hbm_gbs", 6650.0)
@@ -818,14 +774,14 @@ def run_ours(args, world, rank, local):
 
     # ---- end to end through the C ABI with host buffers: every step copies its
     # inputs from pinned host memory to the device, runs the step and copies y
-    # back to pinned host memory. A step's xBC, z and dt sit back to back in one
-    # pinned buffer and cross PCIe as one copy; y comes back as one copy. The
-    # copies run on two copy streams over a ring of four device buffers, so the
-    # inputs of later steps and the y of earlier ones cross PCIe while a step
-    # computes. The C entry point is called with arguments marshalled once per
-    # ring slot. The timed region is the whole K-step loop, from the first input
-    # copy to the last y landing in host memory (CUDA events); the host's own
-    # issue time for the loop is reported beside it.
+    # back to pinned host memory, all inside one C call (m2_state_update_host).
+    # A step's xBC, z and dt sit back to back in one pinned buffer and cross
+    # PCIe as one copy; y comes back as one copy. The library's staging ring of
+    # four device buffers and two copy streams lets the inputs of later steps
+    # and the y of earlier ones cross PCIe while a step computes. The timed
+    # region is the whole K-step loop, from the first input copy to the last y
+    # landing in host memory (CUDA events); the host's own issue time for the
+    # loop is reported beside it.
     import ctypes
     ring = 4
     parts = [("xBC", inputs[0]["xBC"]), ("z", inputs[0]["z"]), ("dt", inputs[0]["dt"])]
@@ -841,62 +797,31 @@ def run_ours(args, world, rank, local):
             n = v.numel() * v.element_size()
             hb[offs[k]:offs[k] + n].copy_(inp[k].contiguous().view(torch.uint8).view(-1).cpu())
         host_in.append(hb)
-    dev_in = [torch.empty(packed_bytes, dtype=torch.uint8, device="cuda") for _ in range(ring)]
-    ys = [torch.empty_like(y) for _ in range(ring)]
     host_y = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for _ in range(ring)]
     h2d = sum(v.numel() * v.element_size() for _, v in parts)  # bytes of the step's inputs
     d2h = host_y[0].numel() * host_y[0].element_size()
-    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    stage = m2.HostStage(ring, packed_bytes, d2h)
     L = m2.lib()
+    step_host, join = L.m2_state_update_host, L.m2_host_stage_join
     sp, cp = ssm.c(), conv.c()
     cache_ref, sp_ref, cp_ref = ctypes.byref(cache.c), ctypes.byref(sp), ctypes.byref(cp)
     hp, cd = w.H * w.P, w.conv_dim
-    call_args = []
-    for r in range(ring):
-        base = dev_in[r].data_ptr()
-        call_args.append((base + offs["xBC"], base + offs["dt"], base + offs["z"], ys[r].data_ptr()))
     set_ptrs = [ss.data_ptr() for ss in slot_sets]
     stream_ptr = stream.cuda_stream
-
-    # The loop's stream operations go to the CUDA runtime through ctypes (the
-    # same libcudart torch loaded), so that issuing a step costs the host a few
-    # microseconds instead of the tens that torch's Python wrappers take.
-    rt = cudart()
-    H2D, D2H = 1, 2
     in_ptr = [hb.data_ptr() for hb in host_in]
     hy_ptr = [hy.data_ptr() for hy in host_y]
-    dv_ptr = [d.data_ptr() for d in dev_in]
-    ys_ptr = [yy.data_ptr() for yy in ys]
-    s_in_p, s_out_p = s_in.cuda_stream, s_out.cuda_stream
-    ev = [[rt.event() for _ in range(ring)] for _ in range(3)]  # in_done, comp_done, out_done
+    off_x, off_dt, off_z = offs["xBC"], offs["dt"], offs["z"]
 
     def e2e_loop(n, t_start=None, t_end=None):
-        in_done, comp_done, out_done = ev
         if t_start is not None:
             t_start.record(stream)
-        s_in.wait_stream(stream)
-        s_out.wait_stream(stream)
-        memcpy, record, wait = rt.cudaMemcpyAsync, rt.cudaEventRecord, rt.cudaStreamWaitEvent
         for i in range(n):
-            r = i % ring
-            if i >= ring:
-                wait(s_in_p, comp_done[r], 0)  # step i-ring has read this input buffer
-            rt.check(memcpy(dv_ptr[r], in_ptr[i % n_sets], packed_bytes, H2D, s_in_p), "copy in")
-            record(in_done[r], s_in_p)
-            wait(stream_ptr, in_done[r], 0)
-            if i >= ring:
-                wait(stream_ptr, out_done[r], 0)  # y of step i-ring has been copied out
-            xp, dtp, zp, yp = call_args[r]
-            st = L.m2_state_update(cache_ref, sp_ref, cp_ref, w.batch, xp, m2.M2_BF16, cd, dtp, w.H, zp, hp,
-                                   yp, hp, set_ptrs[i % len(set_ptrs)], stream_ptr)
+            st = step_host(stage.ptr, cache_ref, sp_ref, cp_ref, w.batch, in_ptr[i % n_sets], off_x, cd, off_dt,
+                           w.H, off_z, hp, hy_ptr[i % ring], hp, set_ptrs[i % len(set_ptrs)], stream_ptr)
             if st != m2.M2_OK:
-                raise m2.M2Error(st, "m2_state_update")
-            record(comp_done[r], stream_ptr)
-            wait(s_out_p, comp_done[r], 0)
-            rt.check(memcpy(hy_ptr[r], ys_ptr[r], d2h, D2H, s_out_p), "copy out")
-            record(out_done[r], s_out_p)
-        stream.wait_stream(s_in)
-        stream.wait_stream(s_out)
+                raise m2.M2Error(st, "m2_state_update_host")
+        if join(stage.ptr, stream_ptr) != m2.M2_OK:
+            raise m2.M2Error(m2.M2_ERR_CUDA, "m2_host_stage_join")
         if t_end is not None:
             t_end.record(stream)
 
@@ -912,12 +837,14 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = e_start.elapsed_time(e_end)
-    for e_ in ev:
-        for x_ in e_:
-            rt.cudaEventDestroy(x_)
+    stage.close()
     e2e_value, _ = job_throughput(w.batch * args.steps, e2e_ms, world)
     # the link itself on this machine: one step's packed inputs host -> device and
-    # its y device -> host, each timed alone (CUDA events on its copy stream)
+    # its y device -> host, each timed alone (CUDA events on a copy stream)
+    dev_in = torch.empty(packed_bytes, dtype=torch.uint8, device="cuda")
+    dev_y = torch.empty_like(y)
+    s_copy = torch.cuda.Stream()
+
     def link_us(copy, strm, reps=20):
         with torch.cuda.stream(strm):
             for _ in range(3):
@@ -930,8 +857,8 @@ def run_ours(args, world, rank, local):
             b_.record(strm)
         torch.cuda.synchronize()
         return 1e3 * a_.elapsed_time(b_) / reps
-    h2d_us = link_us(lambda: dev_in[0].copy_(host_in[0], non_blocking=True), s_in)
-    d2h_us = link_us(lambda: host_y[0].copy_(ys[0], non_blocking=True), s_out)
+    h2d_us = link_us(lambda: dev_in.copy_(host_in[0], non_blocking=True), s_copy)
+    d2h_us = link_us(lambda: host_y[0].copy_(dev_y, non_blocking=True), s_copy)
     bytes_per_launch = W.bytes_per_unit(w) * w.batch + W.param_bytes_per_launch(w)
     avg_s = local_ms / args.steps / 1e3
     achieved = bytes_per_launch / avg_s / 1e9
@@ -962,10 +889,10 @@ def run_ours(args, world, rank, local):
                          "d2h_us_per_step": d2h_us, "d2h_GBs": d2h / d2h_us / 1e3,
                          "note": "each direction timed alone on this box; the steps overlap them with "
                                  "the kernel, so the slowest of the three bounds us_per_step"},
-                "how": "pinned host buffer (xBC|z|dt packed) -> device, one copy; m2_state_update "
-                       "through the C ABI; y -> pinned host, one copy; every step, on two copy "
-                       "streams over a ring of 4 buffers, overlapping the steps; copies and "
-                       "stream waits issued through the CUDA runtime by ctypes"},
+                "how": "m2_state_update_host through the C ABI, one call per step: pinned host "
+                       "buffer (xBC|z|dt packed) -> device, one copy; the fused step; y -> pinned "
+                       "host, one copy; the library's staging ring of 4 device buffers and two copy "
+                       "streams overlaps the copies with the steps"},
         "gpu_launches": args.steps,  # one fused decode launch per timed step (device-resident loop)
         "clocks": clocks,
     }

@@ -423,6 +423,47 @@ m2_status m2_mixed_step(const m2_cache* cache, const m2_ssm_params* ssm, const m
                         const m2_decode_rows* decode, const m2_prefill_rows* prefill,
                         m2_stream stream);
 
+/*
+ * Decode steps whose inputs and outputs live in host memory (vllm.cpp issue
+ * #1311, section "The divergence": the same fused step as m2_state_update,
+ * for a caller that produces the step's rows on the host and reads y back
+ * every step). An m2_host_stage owns `depth` device staging buffers of
+ * in_bytes and y_bytes, two copy streams and the events that order them; it
+ * is created and destroyed off the hot path (cudaMalloc / cudaFree, device of
+ * the current context). M2_ERR_INVALID_ARG for depth < 1 or a zero size,
+ * M2_ERR_OOM when the device is out of memory.
+ */
+typedef struct m2_host_stage m2_host_stage;
+m2_status m2_host_stage_create(int32_t depth, int64_t in_bytes, int64_t y_bytes, m2_host_stage** out);
+m2_status m2_host_stage_destroy(m2_host_stage* stage);
+
+/*
+ * One m2_state_update step (conv fused when conv is non-NULL) whose rows come
+ * from host memory. host_in (pinned, in_bytes of the stage) holds the step's
+ * xBC rows at byte offset off_xBC (act_dtype, xBC_row_stride elements), its
+ * dt rows at off_dt and its z rows at off_z (off_z < 0: no gate); every
+ * offset a multiple of 16. y (batch rows of y_row_stride elements, act_dtype)
+ * is copied into host_y (pinned) afterwards. slot_idx is on the device.
+ * The step takes the next staging buffer of the ring: its copy in (on the
+ * stage's input stream) waits until the step that last used the buffer has
+ * run, the step on `stream` waits for that copy and for the copy out of the
+ * buffer's previous y, and the copy out (on the stage's output stream)
+ * follows the step, so consecutive steps overlap their copies with each
+ * other's kernels. Everything is asynchronous to the host; host_in may be
+ * rewritten and host_y read only after m2_host_stage_join and a
+ * synchronisation of `stream`. Validation as for m2_state_update, plus the
+ * stage's sizes (M2_ERR_INVALID_ARG) before anything is enqueued.
+ */
+m2_status m2_state_update_host(m2_host_stage* stage, const m2_cache* cache, const m2_ssm_params* ssm,
+                               const m2_conv_params* conv, int32_t batch, const void* host_in,
+                               int64_t off_xBC, int64_t xBC_row_stride, int64_t off_dt,
+                               int64_t dt_row_stride, int64_t off_z, int64_t z_row_stride, void* host_y,
+                               int64_t y_row_stride, const int32_t* slot_idx, m2_stream stream);
+
+/* Makes `stream` wait for every copy the stage has issued so far; the next
+ * step's copy in then also waits for `stream`'s work issued before it. */
+m2_status m2_host_stage_join(m2_host_stage* stage, m2_stream stream);
+
 /* Debug/test path: synchronises `stream`, copies the cache's error word to
  * *out_code (0 or an m2_status value) and clears it. Not for hot loops. */
 m2_status m2_get_device_error(const m2_cache* cache, m2_stream stream, int32_t* out_code);

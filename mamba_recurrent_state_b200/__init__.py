@@ -141,6 +141,12 @@ SIGNATURES = {
     "m2_state_update_multi": (_I32, [ctypes.POINTER(m2_cache), ctypes.POINTER(m2_ssm_params),
                                      ctypes.POINTER(m2_conv_params), _I32, _I32, _P, _I64, _P, _I64, _P, _I64,
                                      _P, _I64, _P, _P, _P]),
+    "m2_host_stage_create": (_I32, [_I32, _I64, _I64, ctypes.POINTER(_P)]),
+    "m2_host_stage_destroy": (_I32, [_P]),
+    "m2_state_update_host": (_I32, [_P, ctypes.POINTER(m2_cache), ctypes.POINTER(m2_ssm_params),
+                                    ctypes.POINTER(m2_conv_params), _I32, _P, _I64, _I64, _I64, _I64, _I64,
+                                    _I64, _P, _I64, _P, _P]),
+    "m2_host_stage_join": (_I32, [_P, _P]),
     "m2_get_device_error": (_I32, [ctypes.POINTER(m2_cache), _P, ctypes.POINTER(_I32)]),
     "m2_status_string": (ctypes.c_char_p, [_I32]),
     "m2_version": (ctypes.c_char_p, []),
@@ -366,6 +372,53 @@ def state_update(cache: Cache, ssm: SSMParams, xBC: torch.Tensor, dt: torch.Tens
         _row_stride(y), slot_idx.data_ptr(), _stream_ptr() if stream is None else stream)
     _check(st, "m2_state_update")
     return y
+
+
+class HostStage:
+    """Device staging ring for decode steps whose rows live in pinned host
+    memory (m2_host_stage_create): ``depth`` buffers of ``in_bytes`` and
+    ``y_bytes``, two copy streams and their events."""
+
+    def __init__(self, depth: int, in_bytes: int, y_bytes: int):
+        ptr = ctypes.c_void_p()
+        _check(lib().m2_host_stage_create(depth, in_bytes, y_bytes, ctypes.byref(ptr)), "m2_host_stage_create")
+        self.ptr = ptr
+        self.in_bytes, self.y_bytes = in_bytes, y_bytes
+
+    def join(self, stream: Optional[int] = None) -> None:
+        """``stream`` waits for every copy the stage has issued."""
+        _check(lib().m2_host_stage_join(self.ptr, _stream_ptr() if stream is None else stream), "m2_host_stage_join")
+
+    def close(self) -> None:
+        if self.ptr is not None and self.ptr.value:
+            _check(lib().m2_host_stage_destroy(self.ptr), "m2_host_stage_destroy")
+        self.ptr = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def state_update_host(stage: HostStage, cache: Cache, ssm: SSMParams, conv: Optional[ConvParams], batch: int,
+                      host_in: torch.Tensor, off_xBC: int, xBC_row_stride: int, off_dt: int, dt_row_stride: int,
+                      off_z: int, z_row_stride: int, host_y: torch.Tensor, y_row_stride: int,
+                      slot_idx: torch.Tensor, stream: Optional[int] = None) -> None:
+    """One decode step from pinned host memory (m2_state_update_host): the
+    packed rows of ``host_in`` (byte offsets and element strides of xBC, dt and
+    z; ``off_z`` < 0 for no gate) are copied in, the step runs, y is copied
+    into ``host_y``. Asynchronous: read ``host_y`` after ``stage.join`` and a
+    synchronisation."""
+    if not host_in.is_pinned() or not host_y.is_pinned():
+        raise ValueError("host_in and host_y must be pinned host tensors")
+    sp = ssm.c()
+    cp = conv.c() if conv is not None else None
+    st = lib().m2_state_update_host(
+        stage.ptr, ctypes.byref(cache.c), ctypes.byref(sp), ctypes.byref(cp) if cp is not None else None, batch,
+        host_in.data_ptr(), off_xBC, xBC_row_stride, off_dt, dt_row_stride, off_z, z_row_stride,
+        host_y.data_ptr(), y_row_stride, slot_idx.data_ptr(), _stream_ptr() if stream is None else stream)
+    _check(st, "m2_state_update_host")
 
 
 def conv1d_update(cache: Cache, conv: ConvParams, xBC: torch.Tensor, slot_idx: torch.Tensor,

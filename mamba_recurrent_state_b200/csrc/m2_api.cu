@@ -10,6 +10,7 @@
 
 #include <cstdlib>
 #include <cstring>
+#include <new>
 #include <vector>
 
 #include "m2_internal.cuh"
@@ -256,11 +257,12 @@ m2_status m2_conv1d_update_varlen(const m2_cache* c, const m2_conv_params* conv,
 
 namespace {
 
+// check_only: validate the arguments and the launch plan, enqueue nothing.
 m2_status state_update_impl(const m2_cache* c, const m2_ssm_params* ssm, const m2_conv_params* conv,
                             const m2_norm_params* norm, int32_t batch, const void* xBC, int32_t xBC_dtype,
                             int64_t xBC_row_stride, const void* dt, int64_t dt_row_stride, const void* z,
                             int64_t z_row_stride, void* y, int64_t y_row_stride, const int32_t* slot_idx,
-                            m2_stream stream) {
+                            m2_stream stream, bool check_only = false) {
     const m2_status st = cache_status(c);
     if (st != M2_OK) return st;
     if (!ssm || !ssm->A_log || !ssm->dt_bias || !ssm->D || batch < 0 || !valid_buffer_dtype(xBC_dtype))
@@ -288,6 +290,7 @@ m2_status state_update_impl(const m2_cache* c, const m2_ssm_params* ssm, const m
     const m2_status ps = m2::plan_state_update(s.nheads, s.head_dim, s.d_state, s.ngroups,
                                                s.state_dtype == M2_BF16, conv != nullptr, &plan);
     if (ps != M2_OK) return ps;
+    if (check_only) return M2_OK;
     if (validate_mode()) {
         const m2_status v = validate_slots(slot_idx, batch, c->num_slots, reinterpret_cast<cudaStream_t>(stream));
         if (v != M2_OK) return v;
@@ -716,5 +719,145 @@ const char* m2_status_string(m2_status s) {
 }
 
 const char* m2_version(void) { return "m2 0.1"; }
+
+// ---------------------------------------------------------------------------
+// Host-staged decode steps: a ring of device staging buffers, two copy
+// streams and the events that order copy in, step and copy out.
+struct m2_host_stage {
+    int32_t depth = 0;
+    int64_t in_bytes = 0;
+    int64_t y_bytes = 0;
+    std::vector<void*> d_in, d_y;
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    std::vector<cudaEvent_t> in_done, comp_done, out_done;
+    cudaEvent_t start = nullptr;
+    std::vector<uint8_t> used;
+    int64_t next = 0;
+    bool fresh = true;  // the next step's copies first wait for the caller's stream
+};
+
+m2_status m2_host_stage_destroy(m2_host_stage* hs) {
+    if (!hs) return M2_ERR_INVALID_ARG;
+    m2_status st = M2_OK;
+    auto keep = [&](cudaError_t e) {
+        if (e != cudaSuccess && st == M2_OK) st = M2_ERR_CUDA;
+    };
+    if (hs->s_in) keep(cudaStreamSynchronize(hs->s_in));
+    if (hs->s_out) keep(cudaStreamSynchronize(hs->s_out));
+    for (void* p : hs->d_in) keep(cudaFree(p));
+    for (void* p : hs->d_y) keep(cudaFree(p));
+    for (auto* v : {&hs->in_done, &hs->comp_done, &hs->out_done})
+        for (cudaEvent_t e : *v) keep(cudaEventDestroy(e));
+    if (hs->start) keep(cudaEventDestroy(hs->start));
+    if (hs->s_in) keep(cudaStreamDestroy(hs->s_in));
+    if (hs->s_out) keep(cudaStreamDestroy(hs->s_out));
+    delete hs;
+    return st;
+}
+
+m2_status m2_host_stage_create(int32_t depth, int64_t in_bytes, int64_t y_bytes, m2_host_stage** out) {
+    if (!out) return M2_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (depth < 1 || depth > 64 || in_bytes <= 0 || y_bytes <= 0) return M2_ERR_INVALID_ARG;
+    auto* hs = new (std::nothrow) m2_host_stage();
+    if (!hs) return M2_ERR_OOM;
+    hs->depth = depth;
+    hs->in_bytes = in_bytes;
+    hs->y_bytes = y_bytes;
+    hs->used.assign(static_cast<size_t>(depth), 0);
+    auto fail = [&](cudaError_t e) {
+        m2_host_stage_destroy(hs);
+        return from_cuda(e);
+    };
+    for (int32_t r = 0; r < depth; ++r) {
+        void* p = nullptr;
+        cudaError_t e = cudaMalloc(&p, static_cast<size_t>(in_bytes));
+        if (e != cudaSuccess) return fail(e);
+        hs->d_in.push_back(p);
+        p = nullptr;
+        e = cudaMalloc(&p, static_cast<size_t>(y_bytes));
+        if (e != cudaSuccess) return fail(e);
+        hs->d_y.push_back(p);
+        for (auto* v : {&hs->in_done, &hs->comp_done, &hs->out_done}) {
+            cudaEvent_t ev = nullptr;
+            e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
+            if (e != cudaSuccess) return fail(e);
+            v->push_back(ev);
+        }
+    }
+    cudaError_t e = cudaEventCreateWithFlags(&hs->start, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&hs->s_in, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&hs->s_out, cudaStreamNonBlocking);
+    if (e != cudaSuccess) return fail(e);
+    *out = hs;
+    return M2_OK;
+}
+
+m2_status m2_state_update_host(m2_host_stage* hs, const m2_cache* c, const m2_ssm_params* ssm,
+                               const m2_conv_params* conv, int32_t batch, const void* host_in,
+                               int64_t off_xBC, int64_t xBC_row_stride, int64_t off_dt,
+                               int64_t dt_row_stride, int64_t off_z, int64_t z_row_stride, void* host_y,
+                               int64_t y_row_stride, const int32_t* slot_idx, m2_stream stream) {
+    if (!hs || !host_in || !host_y || batch < 0) return M2_ERR_INVALID_ARG;
+    const m2_status cs = cache_status(c);
+    if (cs != M2_OK) return cs;
+    if (batch == 0) return M2_OK;
+    const int64_t as = dsize(c->shape.act_dtype);
+    auto block_ok = [&](int64_t off, int64_t stride) {
+        return off >= 0 && off % 16 == 0 && stride > 0 && off + batch * stride * as <= hs->in_bytes;
+    };
+    if (!block_ok(off_xBC, xBC_row_stride) || !block_ok(off_dt, dt_row_stride) ||
+        (off_z >= 0 && !block_ok(off_z, z_row_stride)) || y_row_stride <= 0 ||
+        batch * y_row_stride * as > hs->y_bytes)
+        return M2_ERR_INVALID_ARG;
+    const int32_t r = static_cast<int32_t>(hs->next % hs->depth);
+    uint8_t* din = static_cast<uint8_t*>(hs->d_in[r]);
+    const void* xp = din + off_xBC;
+    const void* dtp = din + off_dt;
+    const void* zp = off_z >= 0 ? din + off_z : nullptr;
+    void* yp = hs->d_y[r];
+    m2_status st = state_update_impl(c, ssm, conv, nullptr, batch, xp, c->shape.act_dtype, xBC_row_stride, dtp,
+                                     dt_row_stride, zp, z_row_stride, yp, y_row_stride, slot_idx, stream, true);
+    if (st != M2_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaSuccess;
+    auto run = [&](cudaError_t x) {
+        if (e == cudaSuccess) e = x;
+    };
+    if (hs->fresh) {  // the copies follow what the caller enqueued on `stream` before
+        run(cudaEventRecord(hs->start, s));
+        run(cudaStreamWaitEvent(hs->s_in, hs->start, 0));
+        run(cudaStreamWaitEvent(hs->s_out, hs->start, 0));
+        hs->fresh = false;
+    }
+    if (hs->used[r]) run(cudaStreamWaitEvent(hs->s_in, hs->comp_done[r], 0));  // the buffer's last step has run
+    run(cudaMemcpyAsync(din, host_in, static_cast<size_t>(hs->in_bytes), cudaMemcpyHostToDevice, hs->s_in));
+    run(cudaEventRecord(hs->in_done[r], hs->s_in));
+    run(cudaStreamWaitEvent(s, hs->in_done[r], 0));
+    if (hs->used[r]) run(cudaStreamWaitEvent(s, hs->out_done[r], 0));  // the buffer's last y has left
+    if (e != cudaSuccess) return M2_ERR_CUDA;
+    st = state_update_impl(c, ssm, conv, nullptr, batch, xp, c->shape.act_dtype, xBC_row_stride, dtp,
+                           dt_row_stride, zp, z_row_stride, yp, y_row_stride, slot_idx, stream);
+    if (st != M2_OK) return st;
+    run(cudaEventRecord(hs->comp_done[r], s));
+    run(cudaStreamWaitEvent(hs->s_out, hs->comp_done[r], 0));
+    run(cudaMemcpyAsync(host_y, yp, static_cast<size_t>(batch * y_row_stride * as), cudaMemcpyDeviceToHost,
+                        hs->s_out));
+    run(cudaEventRecord(hs->out_done[r], hs->s_out));
+    hs->used[r] = 1;
+    ++hs->next;
+    return e == cudaSuccess ? M2_OK : M2_ERR_CUDA;
+}
+
+m2_status m2_host_stage_join(m2_host_stage* hs, m2_stream stream) {
+    if (!hs) return M2_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    for (int32_t r = 0; r < hs->depth; ++r) {
+        if (!hs->used[r]) continue;
+        if (cudaStreamWaitEvent(s, hs->out_done[r], 0) != cudaSuccess) return M2_ERR_CUDA;
+    }
+    hs->fresh = true;
+    return M2_OK;
+}
 
 }  // extern "C"

@@ -141,3 +141,24 @@ def test_newer_entry_points_validate_on_the_host(lib):
                              None) == m2.M2_ERR_INVALID_ARG
     assert lib.m2_mixed_step(ctypes.byref(cache), ctypes.byref(ssm), ctypes.byref(conv), None, None,
                              None) == m2.M2_OK
+
+
+def test_host_stage_validates_on_the_host(lib):
+    """The host-staged decode entry points refuse bad arguments before any
+    CUDA call: no stage is created for a zero depth or size, and a missing
+    stage or host buffer is an argument error."""
+    out = ctypes.c_void_p()
+    assert lib.m2_host_stage_create(0, 1024, 1024, ctypes.byref(out)) == m2.M2_ERR_INVALID_ARG
+    assert out.value is None
+    assert lib.m2_host_stage_create(4, 0, 1024, ctypes.byref(out)) == m2.M2_ERR_INVALID_ARG
+    assert lib.m2_host_stage_create(4, 1024, -1, ctypes.byref(out)) == m2.M2_ERR_INVALID_ARG
+    assert lib.m2_host_stage_create(4, 1024, 1024, None) == m2.M2_ERR_INVALID_ARG
+    assert lib.m2_host_stage_destroy(None) == m2.M2_ERR_INVALID_ARG
+    assert lib.m2_host_stage_join(None, None) == m2.M2_ERR_INVALID_ARG
+    shape = m2.Shape(128, 64, 128, 8, 4, m2.M2_BF16, m2.M2_BF16).c()
+    cache = m2.m2_cache()
+    assert lib.m2_cache_wrap(ctypes.byref(shape), 4, 0x100000, 0x200000, None, ctypes.byref(cache)) == m2.M2_OK
+    ssm = m2.m2_ssm_params(0x300000, 0x300100, 0x300200)
+    buf = 0x600000
+    assert lib.m2_state_update_host(None, ctypes.byref(cache), ctypes.byref(ssm), None, 1, buf, 0, 10240, 0, 128,
+                                    -1, 0, buf, 8192, buf, None) == m2.M2_ERR_INVALID_ARG
