@@ -430,8 +430,9 @@ m2_status m2_mixed_step(const m2_cache* cache, const m2_ssm_params* ssm, const m
  * every step). An m2_host_stage owns `depth` device staging buffers of
  * in_bytes and y_bytes, two copy streams and the events that order them; it
  * is created and destroyed off the hot path (cudaMalloc / cudaFree, device of
- * the current context). M2_ERR_INVALID_ARG for depth < 1 or a zero size,
- * M2_ERR_OOM when the device is out of memory.
+ * the current context; destroy first waits for every step and copy it issued).
+ * M2_ERR_INVALID_ARG for depth < 1 or a zero size, M2_ERR_OOM when the device
+ * is out of memory.
  */
 typedef struct m2_host_stage m2_host_stage;
 m2_status m2_host_stage_create(int32_t depth, int64_t in_bytes, int64_t y_bytes, m2_host_stage** out);

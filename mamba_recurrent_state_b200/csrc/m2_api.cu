@@ -742,6 +742,10 @@ m2_status m2_host_stage_destroy(m2_host_stage* hs) {
     auto keep = [&](cudaError_t e) {
         if (e != cudaSuccess && st == M2_OK) st = M2_ERR_CUDA;
     };
+    // every step that read a staging buffer and every copy are done before
+    // the buffers go
+    for (size_t r = 0; r < hs->used.size() && r < hs->comp_done.size(); ++r)
+        if (hs->used[r]) keep(cudaEventSynchronize(hs->comp_done[r]));
     if (hs->s_in) keep(cudaStreamSynchronize(hs->s_in));
     if (hs->s_out) keep(cudaStreamSynchronize(hs->s_out));
     for (void* p : hs->d_in) keep(cudaFree(p));
