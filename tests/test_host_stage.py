@@ -1,7 +1,8 @@
 """Decode steps from pinned host memory (m2_state_update_host): the staged
 copies around the same fused launch give the bits of the device-resident
-path, over more steps than the staging ring holds, with and without the gate,
-and the first step also against the oracle."""
+path, over more steps than the staging ring holds (and with a ring of one
+buffer, every step waiting for the last), with and without the gate, and the
+first step also against the oracle."""
 
 import numpy as np
 import pytest
@@ -36,10 +37,10 @@ def pack_steps(w, steps, gate):
     return bufs, offs, size
 
 
-@pytest.mark.parametrize("gate", [True, False], ids=["gate", "no-gate"])
-def test_host_steps_equal_device_steps_bitwise(gate):
+@pytest.mark.parametrize("gate,depth", [(True, 4), (False, 4), (True, 1)], ids=["gate", "no-gate", "depth1"])
+def test_host_steps_equal_device_steps_bitwise(gate, depth):
     w = W.WORKLOADS[1]
-    steps, depth = 6, 4
+    steps = 6
     a = make_cache(w)
     b = m2.Cache(shape_of(w), w.num_slots, ssm=a.ssm.clone(), conv=a.conv.clone())
     t, ssm, conv = layer_objs(w)
