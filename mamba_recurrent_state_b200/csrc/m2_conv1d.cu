@@ -199,18 +199,20 @@ constexpr int kTileThreads = 128;
 constexpr int kTileCh = 256;   // channels per CTA
 // Tuning knobs (compile-time): tokens per tile, tile buffers in flight per
 // CTA, resident CTAs per SM the register budget is sized for, tiles a CTA walks
-// at most. Measured on the 8 x 2048 Nemotron-H prefill with one box per tile:
-// 32 tokens, 2 buffers, 5 CTAs per SM, 8 tiles 132-134 us; 16 tiles 137 us;
-// 32, 2, 4: 143 us; 32, 3, 4: 144 us; 16, 4, 5: 145 us. (With row-by-row
-// copies: 149.5-151.6, 170-172 for 32, 3, 4, 168-170 for 16-token tiles.)
+// at most. Measured on the 8 x 2048 Nemotron-H prefill with one box per tile
+// and the tanh-form SiLU (the warps wait mostly for the next tile): 32 tokens,
+// 3 buffers, 4 CTAs per SM, 8 tiles 118.8 us; 32, 2, 5: 120.9 us; 64, 2, 3:
+// 120.8 us; 16, 4, 5: 125 us; 16 tiles 129 us; 16, 3, 6: 199 us (spills).
+// With the two-SFU SiLU, bound by its arithmetic, 32, 2, 5 was best
+// (132-134 us; 32, 3, 4: 144 us).
 #ifndef M2_CONV_TILE_TOK
 #define M2_CONV_TILE_TOK 32
 #endif
 #ifndef M2_CONV_NBUF
-#define M2_CONV_NBUF 2
+#define M2_CONV_NBUF 3
 #endif
 #ifndef M2_CONV_MINB
-#define M2_CONV_MINB 5
+#define M2_CONV_MINB 4
 #endif
 #ifndef M2_CONV_MAXTILES
 #define M2_CONV_MAXTILES 8
